@@ -1,0 +1,497 @@
+#!/usr/bin/env python
+"""Paged decode attention benchmark (KV-read GB/s, % of HBM peak, seqs/s).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2|all|1..5]
+                    [--impl ours|reference]
+
+One step = one pa_decode call over the whole batch of the workload (every
+page of every sequence read once, the split-KV combine included when the
+planner splits).  Default workload: the Llama-style MHA decode batch
+(64 sequences x 4096 tokens, 32/32 heads, head size 128, bf16, 4 GiB of K/V
+per step: larger than L2, so no flush is needed between steps; smaller
+workloads flush L2 by writing a 256 MiB buffer between timed steps).
+
+With N > 1 (torchrun), every rank runs its own batch of the same workload
+(weak scaling, no collective on the data path); the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload on this host's cores (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention KV-read GB/s (% of B200 HBM peak) and seqs/s at 1 GPU"
+UNIT = "GB/s"
+SPEC_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_NAME = "pa_decode_kernel"
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+# --------------------------------------------------------------------------- helpers
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+            return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_471_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_per_launch(config_idx: int):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel sources changed since the counters were taken."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except Exception:
+        return None
+    if t.get("source_hash") != kernel_source_hash():
+        return None
+    ent = t.get("configs", {}).get(str(config_idx))
+    return None if ent is None else float(ent["dram_bytes_per_launch"])
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return ws, rank, local
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and getattr(device, "type", "cpu") == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    def __init__(self, device, period_s: float = 0.02):
+        self.device, self.period = device, period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = self._handle(pynvml)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        except Exception:
+            self.ok = False
+        return self
+
+    def _handle(self, nv):
+        """NVML handle of the CUDA device (NVML ignores CUDA_VISIBLE_DEVICES)."""
+        import torch
+        props = torch.cuda.get_device_properties(self.device)
+        uuid = getattr(props, "uuid", None)
+        if uuid is not None:
+            try:
+                return nv.nvmlDeviceGetHandleByUUID("GPU-" + str(uuid))
+            except Exception:
+                pass
+        try:
+            bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.device.index or 0)
+
+    def _run(self):
+        nv = self._nv
+        names = {
+            "gpu_idle": getattr(nv, "nvmlClocksEventReasonGpuIdle", 0x1),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "hw_power_brake_slowdown": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for k, bit in names.items():
+                    if r & bit and k != "gpu_idle":
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join(timeout=1.0)
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- GPU arm
+def bytes_of(wl):
+    return wl.kv_bytes + wl.q_out_bytes
+
+
+def make_device_workload(idx: int, device):
+    from paged_kv_cache_471_b200 import workloads as W
+    return W.make_workload(W.CONFIGS[idx], device)
+
+
+def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0):
+    import torch
+
+    import paged_kv_cache_471_b200 as pa
+    from paged_kv_cache_471_b200 import workloads as W
+
+    cfg = W.CONFIGS[idx]
+    wl = make_device_workload(idx, device)
+    out = torch.empty_like(wl.query)
+    plan = pa.plan(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_size, cfg.block_size,
+                   cfg.max_seq_len, cfg.kv_dtype)
+    ws = torch.zeros(plan["workspace_bytes"], dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    alg_bytes = bytes_of(wl)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = alg_bytes < 4 * l2
+    scratch = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device) if flush else None
+
+    def step():
+        pa.decode(out, wl.query, wl.key_cache, wl.value_cache, cfg.num_kv_heads, cfg.scale,
+                  wl.block_tables, wl.seq_lens, cfg.block_size, cfg.max_seq_len, cfg.kv_dtype,
+                  wl.k_scale, wl.v_scale, workspace_tensor=ws, stream=stream)
+
+    for _ in range(max(warmup, 3)):
+        if flush:
+            scratch.fill_(1)
+        step()
+    torch.cuda.synchronize(device)
+
+    # per-launch device time (events bracket only the decode call)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(device) as clk:
+        t_start.record(stream)
+        for i in range(steps):
+            if flush:
+                scratch.fill_(1)
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(device)
+    barrier(device)
+    kern_ms = [a.elapsed_time(b) for a, b in ev]
+    region_ms = t_start.elapsed_time(t_end)
+    flush_ms = 0.0
+    if flush:
+        # the timed region includes the L2 flushes; the step time excludes them
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(steps):
+            scratch.fill_(1)
+        f1.record(stream)
+        torch.cuda.synchronize(device)
+        flush_ms = f0.elapsed_time(f1)
+    step_ms = sum(kern_ms) / steps if flush else region_ms / steps
+    status = pa.read_status(ws)
+
+    res = dict(cfg=cfg, wl=wl, plan=plan, alg_bytes=alg_bytes, kern_ms=kern_ms,
+               region_ms=region_ms, step_ms=step_ms, flush=flush, flush_ms=flush_ms,
+               clocks=clk.summary(), status=status,
+               launches_per_step=1 + (plan["num_partitions"] > 1))
+
+    if want_e2e:
+        # End to end through the public call: per step, copy the step's inputs
+        # (queries, block tables, sequence lengths) from pinned host memory,
+        # decode against the resident KV cache, and read the output back.
+        q_h = wl.query.cpu().pin_memory()
+        bt_h = wl.block_tables.cpu().pin_memory()
+        sl_h = wl.seq_lens.cpu().pin_memory()
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        q_d, bt_d, sl_d = torch.empty_like(wl.query), torch.empty_like(wl.block_tables), \
+            torch.empty_like(wl.seq_lens)
+
+        def e2e_step():
+            q_d.copy_(q_h, non_blocking=True)
+            bt_d.copy_(bt_h, non_blocking=True)
+            sl_d.copy_(sl_h, non_blocking=True)
+            pa.decode(out, q_d, wl.key_cache, wl.value_cache, cfg.num_kv_heads, cfg.scale, bt_d,
+                      sl_d, cfg.block_size, cfg.max_seq_len, cfg.kv_dtype, wl.k_scale,
+                      wl.v_scale, workspace_tensor=ws, stream=stream)
+            out_h.copy_(out, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(device)
+        barrier(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            if flush:
+                scratch.fill_(1)
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(device)
+        e2e_ms = (e0.elapsed_time(e1) - (flush_ms if flush else 0.0)) / steps
+        h2d = (q_h.numel() * q_h.element_size() + bt_h.numel() * bt_h.element_size()
+               + sl_h.numel() * sl_h.element_size())
+        d2h = out_h.numel() * out_h.element_size()
+        res.update(e2e_ms=e2e_ms, h2d=h2d, d2h=d2h)
+    return res
+
+
+# --------------------------------------------------------------------------- CPU arm
+def cpu_sample(idx: int, wl, budget_s: float = 12.0, max_seqs=None):
+    """Time the fp64 oracle on whole sequences of the workload (all heads),
+    growing the sample until it takes about budget_s.  Returns GB/s over the
+    sample's algorithmic bytes, the sample description and thread count."""
+    import torch
+
+    import oracle
+    from paged_kv_cache_471_b200 import workloads as W
+
+    cfg = wl.cfg
+    threads = len(os.sched_getaffinity(0))
+    kv = oracle.KV_E4M3 if cfg.kv_dtype == W.FP8_E4M3 else oracle.KV_BF16
+    elem = cfg.elem_bytes
+
+    def host_inputs(seqs):
+        bt = wl.block_tables[seqs].cpu()
+        ids = bt[bt >= 0].unique()
+        remap = torch.full((cfg.num_blocks,), -1, dtype=torch.int64)
+        remap[ids] = torch.arange(ids.numel())
+        btn = torch.where(bt >= 0, remap[bt.clamp(min=0).long()], torch.tensor(-1)).to(torch.int32)
+        idd = ids.to(wl.key_cache.device)
+        return (wl.query[seqs].cpu(), wl.key_cache[idd].cpu(), wl.value_cache[idd].cpu(), btn,
+                wl.seq_lens[seqs].cpu())
+
+    def run(seqs):
+        q, kc, vc, bt, sl = host_inputs(seqs)
+        t0 = time.perf_counter()
+        oracle.pa_decode(q, kc, vc, cfg.num_kv_heads, cfg.scale, bt, sl, cfg.block_size, kv,
+                         cfg.k_scale, cfg.v_scale, threads=threads)
+        dt = time.perf_counter() - t0
+        tok = int(sl.clamp(min=0).sum())
+        nbytes = 2 * tok * cfg.num_kv_heads * cfg.head_size * elem + \
+            2 * len(seqs) * cfg.num_heads * cfg.head_size * 2
+        return dt, nbytes
+
+    limit = max_seqs or cfg.num_seqs
+    n = 1
+    dt, nb = run(list(range(n)))
+    if dt < budget_s and n < limit:
+        n = min(limit, max(1, int(n * budget_s / max(dt, 1e-3))))
+        dt, nb = run(list(range(n)))
+    return dict(gbs=nb / dt / 1e9, seconds=dt, seqs=n, threads=threads, bytes=nb)
+
+
+# --------------------------------------------------------------------------- main
+def result_line(idx, r, n_gpus, steps, warmup, cpu=None):
+    cfg = r["cfg"]
+    peak, peak_kind = measured_hbm_peak()
+    gbs = r["alg_bytes"] / (r["step_ms"] * 1e-3) / 1e9
+    kern_avg = sum(r["kern_ms"]) / len(r["kern_ms"])
+    achieved = r["alg_bytes"] / (kern_avg * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": round(gbs * n_gpus, 2),
+        "unit": UNIT,
+        "n_gpus": n_gpus,
+        "steps": steps,
+        "warmup": warmup,
+        "ms_per_step": round(r["step_ms"], 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp8_e4m3 KV, f16 MMA, fp32 softmax" if cfg.kv_dtype == "fp8_e4m3"
+        else "bf16",
+        "data": "synthetic (seeded N(0,1) K/V/Q, seeded random block tables)",
+        "config": {
+            "workload": cfg.name,
+            "config_index": idx,
+            "num_seqs": cfg.num_seqs, "num_heads": cfg.num_heads,
+            "num_kv_heads": cfg.num_kv_heads, "head_size": cfg.head_size,
+            "block_size": cfg.block_size, "num_blocks": cfg.num_blocks,
+            "sum_seq_lens": int(r["wl"].seq_lens.sum()),
+            "bytes_per_step": r["alg_bytes"],
+            "seqs_per_s": round(cfg.num_seqs * n_gpus / (r["step_ms"] * 1e-3), 1),
+            "pct_of_8TBs_spec": round(100 * gbs / SPEC_HBM_GBS, 2),
+            f"pct_of_{peak_kind}_hbm": round(100 * gbs / peak, 2),
+            "l2": ("flushed between steps (256 MiB write, excluded from step time)"
+                   if r["flush"] else "inputs larger than L2, no flush"),
+            "plan": r["plan"],
+            "parallelism": f"weak x{n_gpus} (independent batches per GPU)" if n_gpus > 1
+            else "1 GPU",
+        },
+        "roofline": {
+            "bound": "hbm",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "peak_kind": peak_kind,
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": traffic_per_launch(idx),
+            "kernel": KERNEL_NAME + (" + pa_combine_kernel" if r["launches_per_step"] > 1 else ""),
+            "bytes_per_launch": r["alg_bytes"],
+        },
+        "gpu_launches": steps * r["launches_per_step"],
+        "clocks": r["clocks"],
+        "device_status": r["status"],
+    }
+    if "e2e_ms" in r:
+        line["e2e"] = {"value": round(r["alg_bytes"] / (r["e2e_ms"] * 1e-3) / 1e9 * n_gpus, 2),
+                       "unit": UNIT, "h2d_bytes_per_step": r["h2d"],
+                       "d2h_bytes_per_step": r["d2h"], "ms_per_step": round(r["e2e_ms"], 5),
+                       "note": "per step: pinned H2D of queries/block tables/seq_lens, decode "
+                               "over the resident KV cache, D2H of out"}
+    if cpu is not None:
+        line["cpu_baseline"] = {
+            "value": round(cpu["gbs"], 4), "unit": UNIT, "cores": cpu["threads"],
+            "kind": "oracle",
+            "sample": f"{cpu['seqs']} of {cfg.num_seqs} sequences (all heads), "
+                      f"{cpu['seconds']:.1f} s, fp64 C + OpenMP"}
+    return line
+
+
+def run_reference(args):
+    """The oracle as the reference arm: each step one bounded sample."""
+    import torch
+    ws, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    from paged_kv_cache_471_b200 import workloads as W
+    idx = int(args.config) if args.config not in ("all",) else 2
+    cfg = W.CONFIGS[idx]
+    dev = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
+    wl = W.make_workload(cfg, dev) if dev.type == "cuda" else W.make_workload(
+        W.reduced(idx, num_seqs=2), dev)
+    per = []
+    for i in range(args.warmup + args.steps):
+        r = cpu_sample(idx, wl, budget_s=args.ref_budget / max(args.steps, 1), max_seqs=2)
+        if i >= args.warmup:
+            per.append(r)
+    gbs = sum(r["bytes"] for r in per) / sum(r["seconds"] for r in per) / 1e9
+    ms = 1e3 * sum(r["seconds"] for r in per) / len(per)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "config_index": idx},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": UNIT, "cores": per[0]["threads"],
+                         "kind": "oracle",
+                         "sample": f"per step {per[0]['seqs']} sequence(s) of {cfg.num_seqs}, "
+                                   "all heads, fp64 C + OpenMP"},
+        "e2e": {"value": round(gbs, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="2", help="workload 1..5, or 'all' (one line each)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--ref-budget", type=float, default=20.0,
+                    help="seconds of CPU time for the reference arm's timed steps")
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)
+
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local if ws > 1 else 0)
+    torch.cuda.set_device(device)
+    import paged_kv_cache_471_b200 as pa
+    pa.lib()
+
+    configs = [1, 2, 3, 4, 5] if args.config == "all" else [int(args.config)]
+    for idx in configs:
+        r = time_gpu(idx, args.steps, args.warmup, device, want_e2e=not args.no_e2e, rank=rank)
+        r["step_ms"] = reduce_max(r["step_ms"], device)
+        if "e2e_ms" in r:
+            r["e2e_ms"] = reduce_max(r["e2e_ms"], device)
+        cpu = None
+        if rank == 0 and ws == 1 and not args.no_cpu and idx == configs[0]:
+            cpu = cpu_sample(idx, r["wl"])
+        if rank == 0:
+            print(json.dumps(result_line(idx, r, ws, args.steps, args.warmup, cpu)), flush=True)
+        del r
+        torch.cuda.empty_cache()
+    if ws > 1:
+        dist.barrier(device_ids=[device.index])
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

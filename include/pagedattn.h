@@ -1,0 +1,178 @@
+/*
+ * libpagedattn -- paged decode attention for NVIDIA B200 (sm_100a).
+ *
+ * For every sequence s and query head h the library computes
+ *     out[s][h] = softmax(scale * q[s][h] . K_s^T) V_s
+ * where the keys and values of sequence s are scattered over fixed-size
+ * physical blocks and found through an int32 block table.  This is the
+ * problem the PagedAttention pages state:
+ *  - "Why PagedAttention was retired", section 1: the block table is a map
+ *    [num_seqs, max_blocks] of int32 physical block ids; logical block j of
+ *    sequence s lives in physical block block_tables[s][j] (the id is widened
+ *    to 64 bits before address arithmetic);
+ *  - the same page, section 2: K cache [num_blocks, num_kv_heads,
+ *    head_size/x, block_size, x], V cache [num_blocks, num_kv_heads,
+ *    head_size, block_size];
+ *  - the same page, section 3: logits and softmax, then the softmax-weighted
+ *    V, made here in a single pass over each page (online softmax);
+ *  - the same page, section 4: K/V may be stored as FP8 e4m3 and are scaled
+ *    by a per-tensor k_scale / v_scale when converted;
+ *  - "PR #47361 report", benchmark snippet: the call's argument order
+ *    (out, query, key_cache, value_cache, num_kv_heads, scale, block_tables,
+ *    seq_lens, block_size, max_seq_len, kv_cache_dtype, k_scale, v_scale),
+ *    and the split-KV temporaries exp_sums / max_logits / tmp_output of the
+ *    partitioned variant, folded here into one opaque workspace.
+ *
+ * Conventions for every entry point:
+ *  - Ownership: the caller allocates and owns every buffer.  pa_decode
+ *    allocates nothing, never synchronises, and only enqueues work on the
+ *    given stream (a cudaStream_t passed as void*; NULL = legacy default).
+ *  - Argument errors are returned synchronously, before any launch, and
+ *    before any CUDA call.  pa_last_error_detail() then names the argument.
+ *  - Launch failures return PA_ERR_CUDA.
+ *  - Device data is not read on the host.  Kernels check every block id
+ *    they use against [0, num_blocks) and every seq_len against
+ *    [0, max_blocks_per_seq * block_size] and max_seq_len; a violation sets
+ *    a bit in the workspace's status word (PA_DEV_*), the offending block is
+ *    skipped and the offending length clamped, and nothing is read out of
+ *    bounds.  Read the word with pa_read_device_status.
+ *
+ * Element types: query and out are bf16.  K/V are bf16 (PA_KV_BF16, x = 8) or
+ * e4m3 codes (PA_KV_FP8_E4M3, x = 16); x is 16 bytes / element size.
+ * Pointer alignment: out, query, key_cache, value_cache and workspace 16 bytes;
+ * block_tables and seq_lens 4 bytes.
+ * Supported shapes: head_size 64 or 128; block_size 16 or 32;
+ * num_heads / num_kv_heads from 1 to 16 (query head h reads kv head
+ * h / (num_heads / num_kv_heads)).
+ */
+#ifndef PAGEDATTN_H
+#define PAGEDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,        /* null / misaligned pointer, inconsistent sizes    */
+    PA_ERR_UNSUPPORTED = 2,        /* head_size, block_size, group size, dtype          */
+    PA_ERR_WORKSPACE_TOO_SMALL = 3,/* workspace_bytes < pa_decode_workspace_size(...)   */
+    PA_ERR_CUDA = 4                /* a CUDA runtime call or launch failed              */
+} pa_status;
+
+typedef enum pa_kv_dtype {
+    PA_KV_BF16 = 0,
+    PA_KV_FP8_E4M3 = 1             /* OCP e4m3 ("fn"): bias 7, no inf, 0x7F/0xFF = NaN  */
+} pa_kv_dtype;
+
+/* Bits a kernel ORs into the workspace status word (never cleared by kernels). */
+#define PA_DEV_BAD_BLOCK_ID 0x1u        /* a block id outside [0, num_blocks): block skipped */
+#define PA_DEV_SEQ_LEN_OUT_OF_RANGE 0x2u/* seq_len < 0, > max_blocks*block_size, or beyond
+                                           max_seq_len's partitions: length clamped           */
+#define PA_DEV_WAIT_TIMEOUT 0x4u        /* a page copy did not land within ~2 s: output void  */
+
+/* Bytes at the start of the workspace reserved for the status word. */
+#define PA_WORKSPACE_HEADER_BYTES 256
+
+/*
+ * Tuning knobs; pass NULL for the planner's defaults.
+ *  partition_pages: 0 lets the planner choose; > 0 forces split-KV partitions
+ *      of that many blocks (the combine kernel merges them).  A value >= the
+ *      longest sequence's block count means "no split".
+ *  num_sms: 0 queries the current device; > 0 plans for that many SMs
+ *      (lets the host plan without a GPU, e.g. to size a workspace).
+ */
+typedef struct pa_options {
+    int partition_pages;
+    int num_sms;
+} pa_options;
+
+/* What pa_decode will launch for a given problem. */
+typedef struct pa_plan {
+    int num_partitions;     /* P: split-KV partitions per (seq, kv head); 1 = no split */
+    int partition_pages;    /* blocks per partition                                    */
+    int stages;             /* page buffers per warp in shared memory                  */
+    int warps_per_cta;      /* consumer warps per CTA                                   */
+    long long grid_ctas;    /* CTAs of the decode kernel: num_seqs*num_kv_heads*P       */
+    size_t smem_bytes;      /* dynamic shared memory per CTA                            */
+    size_t workspace_bytes; /* bytes pa_decode needs in `workspace`                     */
+} pa_plan;
+
+/*
+ * Fill *plan for the given sizes.  Host only; makes a CUDA call only when
+ * opts == NULL or opts->num_sms == 0 (to read the SM count).
+ */
+pa_status pa_plan_decode(pa_plan* plan, int num_seqs, int num_heads, int num_kv_heads,
+                         int head_size, int block_size, int max_seq_len, pa_kv_dtype kv_dtype,
+                         const pa_options* opts);
+
+/*
+ * Workspace bytes pa_decode needs (>= PA_WORKSPACE_HEADER_BYTES), or 0 when the
+ * sizes are invalid.  Layout: a 256-byte header whose first uint32 is the
+ * status word, then (when P > 1) per (seq, query head, partition) an fp32
+ * partial output [head_size], and fp32 running max (log2 domain) and sum.
+ * The caller zeroes the workspace once after allocating it; pa_decode never
+ * clears the status word (it is sticky) and overwrites the partials.
+ */
+size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_size,
+                                int block_size, int max_seq_len, pa_kv_dtype kv_dtype,
+                                const pa_options* opts);
+
+/*
+ * Paged decode attention.
+ *  out          bf16 [num_seqs, num_heads, head_size], written.
+ *  query        bf16 [num_seqs, num_heads, head_size].
+ *  key_cache    [num_blocks, num_kv_heads, head_size/x, block_size, x] of kv_dtype.
+ *  value_cache  [num_blocks, num_kv_heads, head_size, block_size] of kv_dtype.
+ *  scale        logit scale (typically 1/sqrt(head_size)); finite.
+ *  block_tables int32 [num_seqs, max_blocks_per_seq]; entries past a
+ *               sequence's last block are never read.
+ *  seq_lens     int32 [num_seqs]; 0 gives a zero output row.
+ *  max_seq_len  upper bound of seq_lens, used only to plan the split.
+ *  num_blocks   blocks in each cache (bounds for block ids).
+ *  k_scale, v_scale  device pointers to one fp32 each; required for FP8,
+ *               ignored for bf16.
+ *  workspace    device buffer of workspace_bytes (see above).
+ *  stream       cudaStream_t to enqueue on.
+ * All pointers are device pointers.  Accumulation is fp32; out is rounded
+ * to bf16 (round to nearest even).
+ */
+pa_status pa_decode(void* out, const void* query, const void* key_cache, const void* value_cache,
+                    int num_seqs, int num_heads, int num_kv_heads, int head_size, float scale,
+                    const int32_t* block_tables, int max_blocks_per_seq, const int32_t* seq_lens,
+                    int block_size, int max_seq_len, int64_t num_blocks, pa_kv_dtype kv_dtype,
+                    const float* k_scale, const float* v_scale, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/* pa_decode with tuning options (opts may be NULL). */
+pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
+                       const void* value_cache, int num_seqs, int num_heads, int num_kv_heads,
+                       int head_size, float scale, const int32_t* block_tables,
+                       int max_blocks_per_seq, const int32_t* seq_lens, int block_size,
+                       int max_seq_len, int64_t num_blocks, pa_kv_dtype kv_dtype,
+                       const float* k_scale, const float* v_scale, void* workspace,
+                       size_t workspace_bytes, void* stream, const pa_options* opts);
+
+/*
+ * Copy the workspace status word to *flags (synchronises `stream`), and
+ * zero it afterwards when clear != 0.
+ */
+pa_status pa_read_device_status(void* workspace, uint32_t* flags, int clear, void* stream);
+
+/* Static text for a status code. */
+const char* pa_status_string(pa_status status);
+
+/* Text describing the last error returned on the calling thread ("" if none). */
+const char* pa_last_error_detail(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H */

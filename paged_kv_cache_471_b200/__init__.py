@@ -1,0 +1,242 @@
+"""Python binding of libpagedattn (paged decode attention, B200 / sm_100a).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libpagedattn.so``; torch is used for device memory and streams.
+If the library has not been built the calls raise -- there is no fallback.
+
+``decode`` takes its arguments in the order of the call printed in the PR
+#47361 benchmark snippet (out, query, key_cache, value_cache, num_kv_heads,
+scale, block_tables, seq_lens, block_size, max_seq_len, kv dtype, k_scale,
+v_scale), with the split-KV temporaries folded into one optional workspace.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpagedattn.so")
+
+PA_OK = 0
+PA_ERR_INVALID_ARG = 1
+PA_ERR_UNSUPPORTED = 2
+PA_ERR_WORKSPACE_TOO_SMALL = 3
+PA_ERR_CUDA = 4
+
+PA_KV_BF16 = 0
+PA_KV_FP8_E4M3 = 1
+
+PA_DEV_BAD_BLOCK_ID = 0x1
+PA_DEV_SEQ_LEN_OUT_OF_RANGE = 0x2
+PA_DEV_WAIT_TIMEOUT = 0x4
+
+WORKSPACE_HEADER_BYTES = 256
+
+_KV = {"bf16": PA_KV_BF16, "auto": PA_KV_BF16, "fp8": PA_KV_FP8_E4M3, "fp8_e4m3": PA_KV_FP8_E4M3,
+       PA_KV_BF16: PA_KV_BF16, PA_KV_FP8_E4M3: PA_KV_FP8_E4M3}
+
+
+class PagedAttentionError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        self.status = status
+        super().__init__(detail)
+
+
+class Options(ctypes.Structure):
+    _fields_ = [("partition_pages", ctypes.c_int), ("num_sms", ctypes.c_int)]
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [("num_partitions", ctypes.c_int), ("partition_pages", ctypes.c_int),
+                ("stages", ctypes.c_int), ("warps_per_cta", ctypes.c_int),
+                ("grid_ctas", ctypes.c_longlong), ("smem_bytes", ctypes.c_size_t),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+    def as_dict(self):
+        return {f: getattr(self, f) for f, _ in self._fields_}
+
+
+_lib = None
+_lock = threading.Lock()
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+
+
+def _bind(lib):
+    decode_args = [_P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float, _P, _I, _P, _I, _I,
+                   ctypes.c_int64, _I, _P, _P, _P, ctypes.c_size_t, _P]
+    lib.pa_decode.argtypes = decode_args
+    lib.pa_decode.restype = _I
+    lib.pa_decode_ex.argtypes = decode_args + [ctypes.POINTER(Options)]
+    lib.pa_decode_ex.restype = _I
+    lib.pa_plan_decode.argtypes = [ctypes.POINTER(Plan), _I, _I, _I, _I, _I, _I, _I,
+                                   ctypes.POINTER(Options)]
+    lib.pa_plan_decode.restype = _I
+    lib.pa_decode_workspace_size.argtypes = [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(Options)]
+    lib.pa_decode_workspace_size.restype = ctypes.c_size_t
+    lib.pa_read_device_status.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32), _I, _P]
+    lib.pa_read_device_status.restype = _I
+    lib.pa_status_string.argtypes = [_I]
+    lib.pa_status_string.restype = ctypes.c_char_p
+    lib.pa_last_error_detail.argtypes = []
+    lib.pa_last_error_detail.restype = ctypes.c_char_p
+    lib.pa_version.argtypes = []
+    lib.pa_version.restype = _I
+    return lib
+
+
+def lib():
+    """The loaded libpagedattn (raises if it was never built)."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    raise RuntimeError(
+                        f"{LIB_PATH} is missing: build it with "
+                        "`python -m paged_kv_cache_471_b200.build` (there is no fallback path)")
+                _lib = _bind(ctypes.CDLL(LIB_PATH))
+    return _lib
+
+
+def _check(rc: int):
+    if rc != PA_OK:
+        L = lib()
+        raise PagedAttentionError(rc, f"{L.pa_status_string(rc).decode()}: "
+                                      f"{L.pa_last_error_detail().decode()}")
+
+
+def _opts(partition_pages=0, num_sms=0):
+    if not partition_pages and not num_sms:
+        return None
+    return ctypes.byref(Options(int(partition_pages), int(num_sms)))
+
+
+def kv_dtype_code(kv_dtype) -> int:
+    try:
+        return _KV[kv_dtype]
+    except KeyError:
+        raise ValueError(f"unsupported kv dtype {kv_dtype!r}") from None
+
+
+def plan(num_seqs, num_heads, num_kv_heads, head_size, block_size, max_seq_len, kv_dtype="bf16",
+         partition_pages=0, num_sms=0) -> dict:
+    p = Plan()
+    _check(lib().pa_plan_decode(ctypes.byref(p), num_seqs, num_heads, num_kv_heads, head_size,
+                                block_size, max_seq_len, kv_dtype_code(kv_dtype),
+                                _opts(partition_pages, num_sms)))
+    return p.as_dict()
+
+
+def workspace_size(num_seqs, num_heads, num_kv_heads, head_size, block_size, max_seq_len,
+                   kv_dtype="bf16", partition_pages=0, num_sms=0) -> int:
+    n = lib().pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_size, block_size,
+                                       max_seq_len, kv_dtype_code(kv_dtype),
+                                       _opts(partition_pages, num_sms))
+    if n == 0:
+        raise PagedAttentionError(PA_ERR_INVALID_ARG, lib().pa_last_error_detail().decode())
+    return n
+
+
+_ws_cache = {}
+
+
+def workspace(nbytes: int, device):
+    """A zeroed workspace of at least nbytes on `device`, reused across calls
+    (its status word is sticky; see read_status)."""
+    import torch
+    dev = torch.device(device)
+    key = (dev.type, dev.index)
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(max(nbytes, WORKSPACE_HEADER_BYTES), dtype=torch.uint8, device=dev)
+        _ws_cache[key] = ws
+    return ws
+
+
+def _ptr(t, name, dtypes=None, device=None):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    return t.data_ptr()
+
+
+def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, block_tables,
+           seq_lens, block_size: int, max_seq_len: int, kv_dtype="bf16", k_scale=None,
+           v_scale=None, workspace_tensor=None, partition_pages: int = 0, stream=None):
+    """Paged decode attention into ``out`` (bf16 [num_seqs, num_heads, head_size]).
+
+    key_cache: [num_blocks, num_kv_heads, head_size/x, block_size, x];
+    value_cache: [num_blocks, num_kv_heads, head_size, block_size]; bf16, or
+    uint8 / float8_e4m3fn holding e4m3 codes when kv_dtype is "fp8_e4m3"
+    (then k_scale / v_scale are 1-element fp32 CUDA tensors).
+    """
+    import torch
+    code = kv_dtype_code(kv_dtype)
+    dev = query.device
+    S, Hq, D = query.shape
+    kv_types = (torch.bfloat16,) if code == PA_KV_BF16 else (torch.uint8, torch.float8_e4m3fn)
+    args_ptrs = [
+        _ptr(out, "out", (torch.bfloat16,), dev),
+        _ptr(query, "query", (torch.bfloat16,), dev),
+        _ptr(key_cache, "key_cache", kv_types, dev),
+        _ptr(value_cache, "value_cache", kv_types, dev),
+    ]
+    if tuple(out.shape) != (S, Hq, D):
+        raise ValueError("out must have the query's shape")
+    if key_cache.dim() != 5 or value_cache.dim() != 4:
+        raise ValueError("key_cache must be 5-D and value_cache 4-D")
+    num_blocks = key_cache.shape[0]
+    if value_cache.shape[0] != num_blocks or key_cache.shape[3] != block_size \
+            or value_cache.shape[3] != block_size or key_cache.shape[1] != num_kv_heads \
+            or value_cache.shape[1] != num_kv_heads or value_cache.shape[2] != D \
+            or key_cache.shape[2] * key_cache.shape[4] != D:
+        raise ValueError("cache shapes do not match query / num_kv_heads / block_size")
+    bt = _ptr(block_tables, "block_tables", (torch.int32,), dev)
+    sl = _ptr(seq_lens, "seq_lens", (torch.int32,), dev)
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or seq_lens.shape != (S,):
+        raise ValueError("block_tables must be [num_seqs, max_blocks] and seq_lens [num_seqs]")
+    ks = vs = None
+    if code == PA_KV_FP8_E4M3:
+        ks = _ptr(k_scale, "k_scale", (torch.float32,), dev)
+        vs = _ptr(v_scale, "v_scale", (torch.float32,), dev)
+    need = workspace_size(S, Hq, num_kv_heads, D, block_size, max_seq_len, code, partition_pages)
+    if workspace_tensor is None:
+        workspace_tensor = workspace(need, dev)
+    ws = _ptr(workspace_tensor, "workspace", None, dev)
+    st = stream if stream is not None else torch.cuda.current_stream(dev)
+    rc = lib().pa_decode_ex(*args_ptrs, S, Hq, int(num_kv_heads), D, float(scale), bt,
+                            block_tables.shape[1], sl, int(block_size), int(max_seq_len),
+                            int(num_blocks), code, ks, vs, ws,
+                            workspace_tensor.numel() * workspace_tensor.element_size(),
+                            st.cuda_stream, _opts(partition_pages, 0))
+    _check(rc)
+    return out
+
+
+def read_status(workspace_tensor=None, device=None, clear=False, stream=None) -> int:
+    """The sticky PA_DEV_* bits kernels set in a workspace (synchronises)."""
+    import torch
+    if workspace_tensor is None:
+        dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        workspace_tensor = workspace(WORKSPACE_HEADER_BYTES, dev)
+    st = stream if stream is not None else torch.cuda.current_stream(workspace_tensor.device)
+    flags = ctypes.c_uint32(0)
+    _check(lib().pa_read_device_status(ctypes.c_void_p(workspace_tensor.data_ptr()),
+                                       ctypes.byref(flags), int(bool(clear)), st.cuda_stream))
+    return int(flags.value)
+
+
+def version() -> int:
+    return int(lib().pa_version())

@@ -1,0 +1,364 @@
+// C ABI of libpagedattn: argument checks, the split-KV planner, and the
+// launches of pa_decode_kernel / pa_combine_kernel.  See include/pagedattn.h
+// for the contract of each entry point.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+
+#include "pa_decode_kernels.cuh"
+#include "pagedattn.h"
+
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+constexpr size_t kSmemBudget = 110 * 1024;  // per CTA, so that two CTAs share an SM
+constexpr size_t kSmemPerSm = 228 * 1024;
+constexpr size_t kSmemReservedPerCta = 1024;
+constexpr int kMinPartitionPages = 16;
+constexpr int kMaxStages = 8;
+constexpr int kMaxDevices = 64;
+
+thread_local char g_detail[256] = "";
+
+pa_status fail(pa_status st, const char* fmt, const char* what) {
+    std::snprintf(g_detail, sizeof g_detail, fmt, what);
+    return st;
+}
+
+bool aligned(const void* ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
+
+int elem_bytes(pa_kv_dtype t) { return t == PA_KV_FP8_E4M3 ? 1 : 2; }
+
+pa_status check_sizes(int num_seqs, int num_heads, int num_kv_heads, int head_size,
+                      int block_size, int max_seq_len, pa_kv_dtype kv_dtype) {
+    if (num_seqs < 0) return fail(PA_ERR_INVALID_ARG, "%s", "num_seqs < 0");
+    if (num_heads <= 0 || num_kv_heads <= 0)
+        return fail(PA_ERR_INVALID_ARG, "%s", "num_heads and num_kv_heads must be > 0");
+    if (num_heads % num_kv_heads)
+        return fail(PA_ERR_INVALID_ARG, "%s", "num_heads must be a multiple of num_kv_heads");
+    if (num_heads / num_kv_heads > 16)
+        return fail(PA_ERR_UNSUPPORTED, "%s", "num_heads / num_kv_heads > 16");
+    if (head_size != 64 && head_size != 128)
+        return fail(PA_ERR_UNSUPPORTED, "%s", "head_size must be 64 or 128");
+    if (block_size != 16 && block_size != 32)
+        return fail(PA_ERR_UNSUPPORTED, "%s", "block_size must be 16 or 32");
+    if (kv_dtype != PA_KV_BF16 && kv_dtype != PA_KV_FP8_E4M3)
+        return fail(PA_ERR_UNSUPPORTED, "%s", "kv_dtype");
+    if (max_seq_len < 0) return fail(PA_ERR_INVALID_ARG, "%s", "max_seq_len < 0");
+    return PA_OK;
+}
+
+int device_sms(int* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    static std::atomic<int> cache[kMaxDevices];
+    if (dev >= 0 && dev < kMaxDevices) {
+        int v = cache[dev].load(std::memory_order_relaxed);
+        if (v > 0) {
+            *out = v;
+            return 0;
+        }
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return -1;
+    if (dev >= 0 && dev < kMaxDevices) cache[dev].store(n, std::memory_order_relaxed);
+    *out = n;
+    return 0;
+}
+
+size_t merge_bytes(int head_size, int group) {
+    const int nh = group > 8 ? 2 : 1;
+    return static_cast<size_t>(pa::kWarps * nh * 8 * (head_size + 4) + 2 * pa::kWarps * 16) * 4;
+}
+
+pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int head_size,
+               int block_size, int max_seq_len, pa_kv_dtype kv_dtype, const pa_options* opts) {
+    pa_status st = check_sizes(num_seqs, num_heads, num_kv_heads, head_size, block_size,
+                               max_seq_len, kv_dtype);
+    if (st != PA_OK) return st;
+    int sms = opts ? opts->num_sms : 0;
+    if (sms < 0) return fail(PA_ERR_INVALID_ARG, "%s", "opts->num_sms < 0");
+    if (opts && opts->partition_pages < 0)
+        return fail(PA_ERR_INVALID_ARG, "%s", "opts->partition_pages < 0");
+    if (sms == 0 && device_sms(&sms) != 0)
+        return fail(PA_ERR_CUDA, "%s", "cannot query the SM count of the current device");
+
+    const size_t stage = 2ull * head_size * block_size * elem_bytes(kv_dtype);
+    int ns = static_cast<int>(kSmemBudget / (pa::kWarps * stage));
+    ns = ns < 2 ? 2 : (ns > kMaxStages ? kMaxStages : ns);
+    size_t stage_area = static_cast<size_t>(pa::kWarps) * ns * stage;
+    const size_t mb = merge_bytes(head_size, num_heads / num_kv_heads);
+    if (stage_area < mb) stage_area = mb;
+    const size_t smem = stage_area + static_cast<size_t>(pa::kWarps) * ns * 8;
+    long long per_sm = static_cast<long long>(kSmemPerSm / (smem + kSmemReservedPerCta));
+    if (per_sm < 1) per_sm = 1;
+    if (per_sm > 2) per_sm = 2;
+    const long long slots = static_cast<long long>(sms) * per_sm;
+
+    const long long pages_max = (static_cast<long long>(max_seq_len) + block_size - 1) / block_size;
+    const long long units = static_cast<long long>(num_seqs) * num_kv_heads;
+    long long pp;
+    if (opts && opts->partition_pages > 0) {
+        pp = opts->partition_pages;
+    } else if (pages_max == 0 || units == 0) {
+        pp = 1;
+    } else {
+        // Aim for about four partitions' worth of work per CTA slot if every
+        // sequence were max_seq_len long (bounds the tail of the last wave),
+        // but never fewer than kMinPartitionPages pages per partition.
+        const long long per_slot = (units * pages_max + slots - 1) / slots;
+        long long target = (per_slot + 3) / 4;
+        if (target < kMinPartitionPages) target = kMinPartitionPages;
+        if (target >= pages_max) {
+            pp = pages_max;
+        } else {
+            const long long nparts = (pages_max + target - 1) / target;
+            pp = (pages_max + nparts - 1) / nparts;
+        }
+    }
+    if (pp < 1) pp = 1;
+    long long P = pages_max > 0 ? (pages_max + pp - 1) / pp : 1;
+    if (P <= 1) {
+        P = 1;
+        pp = pages_max > 0 ? pages_max : 1;
+    }
+    if (pp > (1ll << 30) || P > (1ll << 30))
+        return fail(PA_ERR_INVALID_ARG, "%s", "partition count out of range");
+
+    size_t ws = PA_WORKSPACE_HEADER_BYTES;
+    if (P > 1) {
+        ws += static_cast<size_t>(num_seqs) * num_heads * P * (static_cast<size_t>(head_size) + 2) *
+              sizeof(float);
+        ws = (ws + 255) & ~static_cast<size_t>(255);
+    }
+    pl->num_partitions = static_cast<int>(P);
+    pl->partition_pages = static_cast<int>(pp);
+    pl->stages = ns;
+    pl->warps_per_cta = pa::kWarps;
+    pl->grid_ctas = units * P;
+    pl->smem_bytes = smem;
+    pl->workspace_bytes = ws;
+    return PA_OK;
+}
+
+template <typename K>
+cudaError_t ensure_smem(K kernel, size_t smem) {
+    // One attribute call per device and instantiation (the kernel asks for the
+    // planner's largest stage area, so later calls never need more).
+    static std::atomic<int> done[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBudget + 32 * 1024));
+    if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
+    (void)smem;
+    return e;
+}
+
+template <int D, int B, bool FP8, int NH>
+cudaError_t launch_decode(const pa::DecodeParams& p, long long grid, size_t smem,
+                          cudaStream_t st) {
+    auto kern = pa::pa_decode_kernel<D, B, FP8, NH>;
+    cudaError_t e = ensure_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<static_cast<unsigned>(grid), pa::kThreads, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+template <int D, int B, bool FP8>
+cudaError_t launch_nh(const pa::DecodeParams& p, long long grid, size_t smem, cudaStream_t st) {
+    return p.G > 8 ? launch_decode<D, B, FP8, 2>(p, grid, smem, st)
+                   : launch_decode<D, B, FP8, 1>(p, grid, smem, st);
+}
+
+template <int D, int B>
+cudaError_t launch_dtype(const pa::DecodeParams& p, bool fp8, long long grid, size_t smem,
+                         cudaStream_t st) {
+    return fp8 ? launch_nh<D, B, true>(p, grid, smem, st) : launch_nh<D, B, false>(p, grid, smem, st);
+}
+
+cudaError_t launch_any(const pa::DecodeParams& p, int D, int B, bool fp8, long long grid,
+                       size_t smem, cudaStream_t st) {
+    if (D == 64) return B == 16 ? launch_dtype<64, 16>(p, fp8, grid, smem, st)
+                                : launch_dtype<64, 32>(p, fp8, grid, smem, st);
+    return B == 16 ? launch_dtype<128, 16>(p, fp8, grid, smem, st)
+                   : launch_dtype<128, 32>(p, fp8, grid, smem, st);
+}
+
+cudaError_t launch_combine(const pa::CombineParams& c, int D, cudaStream_t st) {
+    const long long rows = static_cast<long long>(c.S) * c.Hq;
+    const unsigned grid = static_cast<unsigned>((rows + pa::kWarps - 1) / pa::kWarps);
+    if (D == 64)
+        pa::pa_combine_kernel<64><<<grid, pa::kThreads, 0, st>>>(c);
+    else
+        pa::pa_combine_kernel<128><<<grid, pa::kThreads, 0, st>>>(c);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_plan_decode(pa_plan* out, int num_seqs, int num_heads, int num_kv_heads,
+                         int head_size, int block_size, int max_seq_len, pa_kv_dtype kv_dtype,
+                         const pa_options* opts) {
+    g_detail[0] = 0;
+    if (!out) return fail(PA_ERR_INVALID_ARG, "%s", "plan is NULL");
+    return plan(out, num_seqs, num_heads, num_kv_heads, head_size, block_size, max_seq_len,
+                kv_dtype, opts);
+}
+
+size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_size,
+                                int block_size, int max_seq_len, pa_kv_dtype kv_dtype,
+                                const pa_options* opts) {
+    g_detail[0] = 0;
+    pa_plan pl;
+    if (plan(&pl, num_seqs, num_heads, num_kv_heads, head_size, block_size, max_seq_len, kv_dtype,
+             opts) != PA_OK)
+        return 0;
+    return pl.workspace_bytes;
+}
+
+pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
+                       const void* value_cache, int num_seqs, int num_heads, int num_kv_heads,
+                       int head_size, float scale, const int32_t* block_tables,
+                       int max_blocks_per_seq, const int32_t* seq_lens, int block_size,
+                       int max_seq_len, int64_t num_blocks, pa_kv_dtype kv_dtype,
+                       const float* k_scale, const float* v_scale, void* workspace,
+                       size_t workspace_bytes, void* stream, const pa_options* opts) {
+    g_detail[0] = 0;
+    pa_status st = check_sizes(num_seqs, num_heads, num_kv_heads, head_size, block_size,
+                               max_seq_len, kv_dtype);
+    if (st != PA_OK) return st;
+    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "%s", "scale is not finite");
+    if (max_blocks_per_seq < 1) return fail(PA_ERR_INVALID_ARG, "%s", "max_blocks_per_seq < 1");
+    if (static_cast<long long>(max_seq_len) > static_cast<long long>(max_blocks_per_seq) * block_size)
+        return fail(PA_ERR_INVALID_ARG, "%s", "max_seq_len > max_blocks_per_seq * block_size");
+    if (num_blocks < 1) return fail(PA_ERR_INVALID_ARG, "%s", "num_blocks < 1");
+    if (num_seqs == 0) return PA_OK;
+    const struct {
+        const void* p;
+        size_t a;
+        const char* name;
+    } ptrs[] = {{out, 16, "out"},
+                {query, 16, "query"},
+                {key_cache, 16, "key_cache"},
+                {value_cache, 16, "value_cache"},
+                {block_tables, 4, "block_tables"},
+                {seq_lens, 4, "seq_lens"},
+                {workspace, 16, "workspace"}};
+    for (const auto& q : ptrs) {
+        if (!q.p) return fail(PA_ERR_INVALID_ARG, "%s is NULL", q.name);
+        if (!aligned(q.p, q.a)) return fail(PA_ERR_INVALID_ARG, "%s is misaligned", q.name);
+    }
+    if (kv_dtype == PA_KV_FP8_E4M3) {
+        if (!k_scale || !v_scale)
+            return fail(PA_ERR_INVALID_ARG, "%s", "k_scale and v_scale are required for FP8");
+        if (!aligned(k_scale, 4) || !aligned(v_scale, 4))
+            return fail(PA_ERR_INVALID_ARG, "%s", "k_scale / v_scale misaligned");
+    }
+    pa_plan pl;
+    st = plan(&pl, num_seqs, num_heads, num_kv_heads, head_size, block_size, max_seq_len, kv_dtype,
+              opts);
+    if (st != PA_OK) return st;
+    if (workspace_bytes < pl.workspace_bytes)
+        return fail(PA_ERR_WORKSPACE_TOO_SMALL, "%s", "workspace_bytes < pa_decode_workspace_size");
+    if (pl.grid_ctas > 0x7fffffffll) return fail(PA_ERR_INVALID_ARG, "%s", "grid too large");
+
+    pa::DecodeParams p;
+    std::memset(&p, 0, sizeof p);
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.q = static_cast<const uint16_t*>(query);
+    p.kc = static_cast<const uint8_t*>(key_cache);
+    p.vc = static_cast<const uint8_t*>(value_cache);
+    p.bt = block_tables;
+    p.seq_lens = seq_lens;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.status = reinterpret_cast<uint32_t*>(ws);
+    const size_t rows = static_cast<size_t>(num_seqs) * num_heads * pl.num_partitions;
+    float* part = reinterpret_cast<float*>(ws + PA_WORKSPACE_HEADER_BYTES);
+    p.ws_o = part;
+    p.ws_m = part + rows * head_size;
+    p.ws_l = p.ws_m + rows;
+    p.S = num_seqs;
+    p.Hq = num_heads;
+    p.Hk = num_kv_heads;
+    p.G = num_heads / num_kv_heads;
+    p.max_blocks = max_blocks_per_seq;
+    p.P = pl.num_partitions;
+    p.PP = pl.partition_pages;
+    p.stages = pl.stages;
+    p.num_blocks = num_blocks;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_any(p, head_size, block_size, kv_dtype == PA_KV_FP8_E4M3, pl.grid_ctas,
+                               pl.smem_bytes, s);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+    if (pl.num_partitions > 1) {
+        pa::CombineParams c;
+        c.out = p.out;
+        c.ws_o = p.ws_o;
+        c.ws_m = p.ws_m;
+        c.ws_l = p.ws_l;
+        c.seq_lens = seq_lens;
+        c.S = num_seqs;
+        c.Hq = num_heads;
+        c.P = pl.num_partitions;
+        c.PP = pl.partition_pages;
+        c.max_blocks = max_blocks_per_seq;
+        c.B = block_size;
+        e = launch_combine(c, head_size, s);
+        if (e != cudaSuccess) return fail(PA_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
+    }
+    return PA_OK;
+}
+
+pa_status pa_decode(void* out, const void* query, const void* key_cache, const void* value_cache,
+                    int num_seqs, int num_heads, int num_kv_heads, int head_size, float scale,
+                    const int32_t* block_tables, int max_blocks_per_seq, const int32_t* seq_lens,
+                    int block_size, int max_seq_len, int64_t num_blocks, pa_kv_dtype kv_dtype,
+                    const float* k_scale, const float* v_scale, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+    return pa_decode_ex(out, query, key_cache, value_cache, num_seqs, num_heads, num_kv_heads,
+                        head_size, scale, block_tables, max_blocks_per_seq, seq_lens, block_size,
+                        max_seq_len, num_blocks, kv_dtype, k_scale, v_scale, workspace,
+                        workspace_bytes, stream, nullptr);
+}
+
+pa_status pa_read_device_status(void* workspace, uint32_t* flags, int clear, void* stream) {
+    g_detail[0] = 0;
+    if (!workspace || !flags) return fail(PA_ERR_INVALID_ARG, "%s", "workspace or flags is NULL");
+    if (!aligned(workspace, 16)) return fail(PA_ERR_INVALID_ARG, "%s", "workspace is misaligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(flags, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess && clear) e = cudaMemsetAsync(workspace, 0, sizeof(uint32_t), s);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+    return PA_OK;
+}
+
+const char* pa_status_string(pa_status status) {
+    switch (status) {
+        case PA_OK: return "PA_OK";
+        case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG: invalid argument";
+        case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED: unsupported shape or dtype";
+        case PA_ERR_WORKSPACE_TOO_SMALL: return "PA_ERR_WORKSPACE_TOO_SMALL: workspace too small";
+        case PA_ERR_CUDA: return "PA_ERR_CUDA: CUDA runtime error";
+    }
+    return "unknown pa_status";
+}
+
+const char* pa_last_error_detail(void) { return g_detail; }
+
+int pa_version(void) { return kVersion; }
+
+}  // extern "C"

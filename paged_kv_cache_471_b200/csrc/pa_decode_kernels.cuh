@@ -1,0 +1,544 @@
+// Paged decode attention kernels for sm_100a.
+//
+// pa_decode_kernel: one CTA per (sequence, kv head, partition); four warps,
+// each an independent producer/consumer pipeline over its share of the
+// partition's pages (pages w, w+4, w+8, ... of the partition).
+//   * Lane 0 of a warp reads the block table (the page table of
+//     "Why PagedAttention was retired", section 1), widens the physical id to
+//     64 bits, and moves the whole (block, kv head) K page and V page --
+//     each one contiguous run of head_size*block_size elements in the cache
+//     layouts of section 2 -- into a shared-memory stage with two 1-D bulk
+//     async copies that complete on the stage's mbarrier.
+//   * The warp consumes a landed page once: S = Q K^T on the tensor cores
+//     (m16n8k16, heads on M, tokens on N, head dim on K), online softmax in
+//     fp32 registers (row max/sum over the quad by shuffles), then
+//     O^T += V^T P^T (head dim on M, heads on N, tokens on K).  K and V are
+//     each read from HBM exactly once -- the single traversal that replaces
+//     the legacy kernel's two passes (section 3 of the same page).
+//   * FP8 e4m3 pages are converted in registers (exact e4m3 -> f16) right
+//     before the MMA; k_scale folds into the logit scale and v_scale into the
+//     output, so the conversion needs no multiply (section 4 of the page).
+//   * The four warps' (max, sum, acc) are merged in shared memory; the CTA
+//     writes bf16 out directly, or, when the sequence is split over several
+//     partitions, an fp32 partial plus its (max, sum) for pa_combine_kernel
+//     (the exp_sums / max_logits / tmp_output roles of the partitioned
+//     variant in the PR #47361 benchmark snippet).
+//
+// Every mbarrier wait is bounded (~2 s); on give-up the warp drains its copies
+// in flight (bounded too), ORs PA_DEV_WAIT_TIMEOUT into the status word and
+// finishes without touching further pages.
+#pragma once
+
+#include <math.h>
+#include <stdint.h>
+
+#include "pa_ptx.cuh"
+
+namespace pa {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr uint32_t kFull = 0xffffffffu;
+
+constexpr uint32_t kDevBadBlock = 0x1u;
+constexpr uint32_t kDevSeqLen = 0x2u;
+constexpr uint32_t kDevTimeout = 0x4u;
+
+struct DecodeParams {
+    __nv_bfloat16* out;       // [S, Hq, D]
+    const uint16_t* q;        // bf16 bits [S, Hq, D]
+    const uint8_t* kc;        // K cache bytes
+    const uint8_t* vc;        // V cache bytes
+    const int32_t* bt;        // [S, max_blocks]
+    const int32_t* seq_lens;  // [S]
+    const float* k_scale;     // fp8 only
+    const float* v_scale;     // fp8 only
+    float* ws_o;              // [S, Hq, P, D]   (P > 1)
+    float* ws_m;              // [S, Hq, P]      running max, log2 domain
+    float* ws_l;              // [S, Hq, P]      running sum
+    uint32_t* status;         // sticky status word
+    int S, Hq, Hk, G;
+    int max_blocks;
+    int P;   // partitions per (seq, kv head)
+    int PP;  // pages per partition
+    int stages;
+    long long num_blocks;
+    float scale_log2;  // scale * log2(e)
+};
+
+// Bytes of shared memory the merge step needs (overlaid on the page stages).
+template <int D, int NH>
+constexpr int merge_smem_bytes() {
+    return (kWarps * NH * 8 * (D + 4) + 2 * kWarps * 16) * 4;
+}
+
+template <int D, int B, bool FP8, int NH>
+__global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodeParams p) {
+    constexpr int ELEM = FP8 ? 1 : 2;
+    constexpr int PAGE = D * B * ELEM;  // one K (or V) page of one kv head
+    constexpr int STAGE = 2 * PAGE;
+    constexpr int NT = B / 8;   // 8-token n-tiles per page (QK)
+    constexpr int KT = D / 16;  // 16-wide k-tiles over the head dim (QK)
+    constexpr int MT = D / 16;  // 16-row m-tiles over the head dim (PV)
+    constexpr int KK = B / 16;  // 16-token k-tiles per page (PV)
+    constexpr int CHUNK = B * 16;  // bytes of one 16-byte column group of a K page
+    constexpr int RS = D + 4;      // padded row stride of the merge buffer
+
+    extern __shared__ __align__(128) uint8_t smem[];
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int gq = lane >> 2;  // fragment row group
+    const int cq = lane & 3;   // thread in quad
+
+    const long long unit = blockIdx.x;
+    const int kvh = static_cast<int>(unit % p.Hk);
+    const int s = static_cast<int>((unit / p.Hk) % p.S);
+    const int part = static_cast<int>(unit / ((long long)p.Hk * p.S));
+
+    // ---- sequence length, with the device-side range checks
+    int T = __ldg(p.seq_lens + s);
+    uint32_t bad = 0;
+    const int t_cap = p.max_blocks * B;
+    if (T < 0) { T = 0; bad = kDevSeqLen; }
+    if (T > t_cap) { T = t_cap; bad = kDevSeqLen; }
+    int nb = (T + B - 1) / B;
+    const int covered = p.P * p.PP;
+    if (nb > covered) { nb = covered; T = nb * B; bad = kDevSeqLen; }
+    if (bad && part == 0 && kvh == 0 && threadIdx.x == 0) atomicOr(p.status, bad);
+
+    const int j0 = part * p.PP;
+    const int j1 = min(nb, j0 + p.PP);
+    const bool direct = (p.P == 1) || (nb <= p.PP);
+    const long long row0 = (long long)s * p.Hq + (long long)kvh * p.G;  // first q head row
+
+    if (j0 >= j1) {
+        if (part == 0) {  // empty sequence: defined as a zero output row
+            for (int i = threadIdx.x; i < p.G * D; i += kThreads)
+                p.out[row0 * D + i] = __float2bfloat16_rn(0.f);
+        }
+        return;
+    }
+
+    const int NS = p.stages;
+    const int span = j1 - j0;
+    const int n_my = span > warp ? (span - warp + kWarps - 1) / kWarps : 0;
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t wstage0 = sbase + static_cast<uint32_t>(warp * NS * STAGE);
+    const uint32_t bar0 = sbase + static_cast<uint32_t>(kWarps * NS * STAGE + warp * NS * 8);
+
+    if (lane == 0) {
+        for (int i = 0; i < NS; ++i) mbar_init(bar0 + 8 * i, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+
+    // Block-table window: lane l holds the id of this warp's page (wbase + l).
+    const int32_t* btrow = p.bt + (long long)s * p.max_blocks + j0 + warp;
+    auto load_win = [&](int base) -> int {
+        const int i = base + lane;
+        return i < n_my ? __ldg(btrow + (long long)kWarps * i) : -1;
+    };
+    int win_a = load_win(0);
+    int win_b = load_win(32);
+    int wbase = 0;
+    uint32_t valid_mask = 0;  // bit per stage: the page in it had a legal block id
+
+    const size_t head_off = static_cast<size_t>(kvh) * PAGE;
+    const size_t block_stride = static_cast<size_t>(p.Hk) * PAGE;
+
+    // Issue the copies of this warp's i-th page (warp-uniform call).
+    auto issue = [&](int i) {
+        if (i >= wbase + 32) {
+            win_a = win_b;
+            win_b = load_win(wbase + 64);
+            wbase += 32;
+        }
+        const int pb = __shfl_sync(kFull, win_a, i & 31);
+        const int stage = i % NS;
+        const uint32_t bar = bar0 + 8 * stage;
+        const bool ok = pb >= 0 && static_cast<long long>(pb) < p.num_blocks;
+        if (lane == 0) {
+            if (ok) {
+                const size_t off = static_cast<size_t>(pb) * block_stride + head_off;
+                const uint32_t dst = wstage0 + static_cast<uint32_t>(stage * STAGE);
+                mbar_arrive_expect_tx(bar, STAGE);
+                bulk_copy_g2s(dst, p.kc + off, PAGE, bar);
+                bulk_copy_g2s(dst + PAGE, p.vc + off, PAGE, bar);
+            } else {
+                mbar_arrive(bar);
+                atomicOr(p.status, kDevBadBlock);
+            }
+        }
+        valid_mask = ok ? (valid_mask | (1u << stage)) : (valid_mask & ~(1u << stage));
+    };
+
+    const int n_pro = n_my < NS ? n_my : NS;
+    for (int i = 0; i < n_pro; ++i) issue(i);
+
+    // ---- Q fragments (A operand of S = Q K^T; rows = heads 8r + gq)
+    uint32_t qa[KT][4];
+    float qk_mul = p.scale_log2;
+    float out_mul = 1.f;
+    if constexpr (!FP8) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int hl = 8 * r + gq;
+            const bool ok = (r < NH) && hl < p.G;
+            const uint16_t* qrow = p.q + (row0 + hl) * D;
+#pragma unroll
+            for (int kt = 0; kt < KT; ++kt) {
+                uint32_t lo = 0, hi = 0;
+                if (ok) {
+                    lo = __ldg(reinterpret_cast<const unsigned int*>(qrow + 16 * kt + 2 * cq));
+                    hi = __ldg(reinterpret_cast<const unsigned int*>(qrow + 16 * kt + 8 + 2 * cq));
+                }
+                qa[kt][r] = lo;
+                qa[kt][r + 2] = hi;
+            }
+        }
+    } else {
+        // f16 operands: q is scaled by 2^-e so that max|q| < 2^15 (f16 range);
+        // 2^e goes back into the logit multiplier.  Within each 16-wide chunk the
+        // k order is permuted to match the e4m3 byte order delivered by ldmatrix:
+        // k = 2c,2c+1 <-> d = 4c,4c+1 and k = 2c+8,2c+9 <-> d = 4c+2,4c+3.
+        float qf[2][KT][4];
+        float amax = 0.f;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int hl = 8 * r + gq;
+            const bool ok = (r < NH) && hl < p.G;
+            const uint16_t* qrow = p.q + (row0 + hl) * D;
+#pragma unroll
+            for (int kt = 0; kt < KT; ++kt) {
+                uint2 w = make_uint2(0u, 0u);
+                if (ok) w = __ldg(reinterpret_cast<const uint2*>(qrow + 16 * kt + 4 * cq));
+                qf[r][kt][0] = bf16_lo(w.x);
+                qf[r][kt][1] = bf16_hi(w.x);
+                qf[r][kt][2] = bf16_lo(w.y);
+                qf[r][kt][3] = bf16_hi(w.y);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(qf[r][kt][e]));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+        int ex = 0;
+        if (amax > 0.f && amax < INFINITY) ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xff) - 127;
+        const int e = ex > 14 ? ex - 14 : 0;
+        const float down = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+        const float up = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int kt = 0; kt < KT; ++kt) {
+                qa[kt][r] = pack_f16x2(qf[r][kt][0] * down, qf[r][kt][1] * down);
+                qa[kt][r + 2] = pack_f16x2(qf[r][kt][2] * down, qf[r][kt][3] * down);
+            }
+        qk_mul = p.scale_log2 * __ldg(p.k_scale) * up;
+        out_mul = __ldg(p.v_scale);
+    }
+
+    float m_run[NH], l_run[NH];
+    float acc[MT][NH][4];
+#pragma unroll
+    for (int r = 0; r < NH; ++r) {
+        m_run[r] = -INFINITY;
+        l_run[r] = 0.f;
+    }
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int r = 0; r < NH; ++r)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[mt][r][e] = 0.f;
+
+    const int quad0 = lane & ~3;
+    const int src0 = quad0 | ((2 * cq) & 3);
+    const int src1 = quad0 | ((2 * cq + 1) & 3);
+    const bool hi_half = cq >= 2;
+
+    bool timed_out = false;
+    int k = 0;
+    for (; k < n_my; ++k) {
+        const int stage = k % NS;
+        const uint32_t bar = bar0 + 8 * stage;
+        const bool landed = mbar_wait_bounded(bar, static_cast<uint32_t>((k / NS) & 1));
+        if (!__all_sync(kFull, landed)) {
+            timed_out = true;
+            break;
+        }
+        const int jg = j0 + warp + kWarps * k;
+        const int valid = ((valid_mask >> stage) & 1u) ? min(B, T - jg * B) : 0;
+        const uint32_t kbase = wstage0 + static_cast<uint32_t>(stage * STAGE);
+        const uint32_t vbase = kbase + PAGE;
+
+        // ---------------- S = Q K^T  (rows: heads, cols: tokens)
+        float sc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
+        {
+            const int mi = lane >> 3, r8 = lane & 7;
+            if constexpr (!FP8) {
+#pragma unroll
+                for (int kt = 0; kt < KT; ++kt)
+#pragma unroll
+                    for (int np = 0; np < NT / 2; ++np) {
+                        const int tok = 8 * (2 * np + (mi >> 1)) + r8;
+                        const int chunk = 2 * kt + (mi & 1);
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4(kbase + chunk * CHUNK + tok * 16, b0, b1, b2, b3);
+                        mma_bf16_16816(sc[2 * np], qa[kt], b0, b1);
+                        mma_bf16_16816(sc[2 * np + 1], qa[kt], b2, b3);
+                    }
+            } else {
+#pragma unroll
+                for (int jp = 0; jp < KT / 2; ++jp)
+#pragma unroll
+                    for (int np = 0; np < NT / 2; ++np) {
+                        const int tok = 8 * (2 * np + (mi & 1)) + r8;
+                        const int chunk = 2 * jp + (mi >> 1);
+                        uint32_t w0, w1, w2, w3;
+                        ldsm_x4(kbase + chunk * CHUNK + tok * 16, w0, w1, w2, w3);
+                        mma_f16_16816(sc[2 * np], qa[2 * jp], e4m3_lo_pair(w0), e4m3_hi_pair(w0));
+                        mma_f16_16816(sc[2 * np + 1], qa[2 * jp], e4m3_lo_pair(w1), e4m3_hi_pair(w1));
+                        mma_f16_16816(sc[2 * np], qa[2 * jp + 1], e4m3_lo_pair(w2), e4m3_hi_pair(w2));
+                        mma_f16_16816(sc[2 * np + 1], qa[2 * jp + 1], e4m3_lo_pair(w3),
+                                      e4m3_hi_pair(w3));
+                    }
+            }
+        }
+
+        // ---------------- online softmax (log2 domain), per head row
+        uint32_t pp[NH][NT];
+        float alpha[NH];
+#pragma unroll
+        for (int r = 0; r < NH; ++r) {
+            float v[NT][2];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    float x = sc[nt][2 * r + e] * qk_mul;
+                    if (valid < B && 8 * nt + 2 * cq + e >= valid) x = -INFINITY;
+                    v[nt][e] = x;
+                    mx = fmaxf(mx, x);
+                }
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+            const float m_new = fmaxf(m_run[r], mx);
+            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+            alpha[r] = exp2f(m_run[r] - m_use);
+            m_run[r] = m_new;
+            float ls = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const float p0 = exp2f(v[nt][0] - m_use);
+                const float p1 = exp2f(v[nt][1] - m_use);
+                uint32_t w;
+                if constexpr (!FP8) {
+                    w = pack_bf16x2(p0, p1);
+                    ls += bf16_lo(w) + bf16_hi(w);
+                } else {
+                    w = pack_f16x2(p0, p1);
+                    ls += f16_lo(w) + f16_hi(w);
+                }
+                pp[r][nt] = w;
+            }
+            l_run[r] = l_run[r] * alpha[r] + ls;
+        }
+
+        // ---------------- rescale O^T columns (heads 8r + 2cq, 8r + 2cq + 1)
+#pragma unroll
+        for (int r = 0; r < NH; ++r) {
+            const float a0 = __shfl_sync(kFull, alpha[r], 8 * cq);
+            const float a1 = __shfl_sync(kFull, alpha[r], 8 * cq + 4);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                acc[mt][r][0] *= a0;
+                acc[mt][r][1] *= a1;
+                acc[mt][r][2] *= a0;
+                acc[mt][r][3] *= a1;
+            }
+        }
+
+        // ---------------- O^T += V^T P^T  (rows: head dim, cols: heads, k: tokens)
+        // Per 16-token k-tile, thread cq holds V for tokens 4cq..4cq+3 (one
+        // contiguous 4-token group per row), so k = 2cq,2cq+1 <-> tokens
+        // 4cq,4cq+1 and k = 2cq+8,2cq+9 <-> 4cq+2,4cq+3; P is regrouped to
+        // that order with quad shuffles.
+#pragma unroll
+        for (int kk = 0; kk < KK; ++kk) {
+            uint32_t pb0[NH], pb1[NH];
+#pragma unroll
+            for (int r = 0; r < NH; ++r) {
+                const uint32_t x0 = __shfl_sync(kFull, pp[r][2 * kk], src0);
+                const uint32_t y0 = __shfl_sync(kFull, pp[r][2 * kk + 1], src0);
+                const uint32_t x1 = __shfl_sync(kFull, pp[r][2 * kk], src1);
+                const uint32_t y1 = __shfl_sync(kFull, pp[r][2 * kk + 1], src1);
+                pb0[r] = hi_half ? y0 : x0;
+                pb1[r] = hi_half ? y1 : x1;
+            }
+            uint32_t mlo = kFull, mhi = kFull;
+            if (valid < B) {
+                const int t0 = 16 * kk + 4 * cq;
+                mlo = (t0 < valid ? 0x0000ffffu : 0u) | (t0 + 1 < valid ? 0xffff0000u : 0u);
+                mhi = (t0 + 2 < valid ? 0x0000ffffu : 0u) | (t0 + 3 < valid ? 0xffff0000u : 0u);
+            }
+            if constexpr (!FP8) {
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    const uint32_t ra = vbase + (16 * mt + gq) * (B * 2) + kk * 32 + cq * 8;
+                    const uint2 va = lds64(ra);
+                    const uint2 vb = lds64(ra + 8 * (B * 2));
+                    const uint32_t a[4] = {va.x & mlo, vb.x & mlo, va.y & mhi, vb.y & mhi};
+#pragma unroll
+                    for (int r = 0; r < NH; ++r) mma_bf16_16816(acc[mt][r], a, pb0[r], pb1[r]);
+                }
+            } else {
+#pragma unroll
+                for (int mp = 0; mp < MT / 2; ++mp) {
+                    uint32_t w0, w1, w2, w3;
+                    ldsm_x4(vbase + (32 * mp + lane) * B + kk * 16, w0, w1, w2, w3);
+                    const uint32_t a0[4] = {e4m3_lo_pair(w0) & mlo, e4m3_lo_pair(w1) & mlo,
+                                            e4m3_hi_pair(w0) & mhi, e4m3_hi_pair(w1) & mhi};
+                    const uint32_t a1[4] = {e4m3_lo_pair(w2) & mlo, e4m3_lo_pair(w3) & mlo,
+                                            e4m3_hi_pair(w2) & mhi, e4m3_hi_pair(w3) & mhi};
+#pragma unroll
+                    for (int r = 0; r < NH; ++r) {
+                        mma_f16_16816(acc[2 * mp][r], a0, pb0[r], pb1[r]);
+                        mma_f16_16816(acc[2 * mp + 1][r], a1, pb0[r], pb1[r]);
+                    }
+                }
+            }
+        }
+
+        __syncwarp();
+        if (k + NS < n_my) issue(k + NS);
+    }
+
+    if (timed_out) {
+        // Let the copies already in flight land (bounded) before the CTA's
+        // shared memory can be handed to anyone else, then report.
+        const int last = min(n_my, k + NS);
+        for (int i = k; i < last; ++i)
+            (void)mbar_wait_bounded(bar0 + 8 * (i % NS), static_cast<uint32_t>((i / NS) & 1));
+        if (lane == 0) atomicOr(p.status, kDevTimeout);
+    }
+
+    // ---------------- merge the four warps' partial softmax states
+#pragma unroll
+    for (int r = 0; r < NH; ++r) {
+        l_run[r] += __shfl_xor_sync(kFull, l_run[r], 1);
+        l_run[r] += __shfl_xor_sync(kFull, l_run[r], 2);
+    }
+    __syncthreads();  // every warp is done with its stages
+    float* s_acc = reinterpret_cast<float*>(smem);
+    float* s_m = s_acc + kWarps * NH * 8 * RS;
+    float* s_l = s_m + kWarps * 16;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int r = 0; r < NH; ++r) {
+            const int h = 8 * r + 2 * cq;
+            const int d = 16 * mt + gq;
+            float* base = s_acc + (warp * NH * 8 + h) * RS + d;
+            base[0] = acc[mt][r][0];
+            base[RS] = acc[mt][r][1];
+            base[8] = acc[mt][r][2];
+            base[RS + 8] = acc[mt][r][3];
+        }
+    if (cq == 0) {
+#pragma unroll
+        for (int r = 0; r < NH; ++r) {
+            s_m[warp * 16 + 8 * r + gq] = m_run[r];
+            s_l[warp * 16 + 8 * r + gq] = timed_out ? 0.f : l_run[r];
+        }
+    }
+    __syncthreads();
+
+    for (int idx = threadIdx.x; idx < p.G * D; idx += kThreads) {
+        const int h = idx / D;
+        const int d = idx - h * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w)
+            if (s_l[w * 16 + h] > 0.f) M = fmaxf(M, s_m[w * 16 + h]);
+        float L = 0.f, O = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const float l = s_l[w * 16 + h];
+            if (l > 0.f) {
+                const float wt = exp2f(s_m[w * 16 + h] - M);
+                L += wt * l;
+                O += wt * s_acc[(w * NH * 8 + h) * RS + d];
+            }
+        }
+        const float o = L > 0.f ? (O / L) * out_mul : 0.f;
+        const long long row = row0 + h;
+        if (direct) {
+            p.out[row * D + d] = __float2bfloat16_rn(o);
+        } else {
+            const long long prow = row * p.P + part;
+            p.ws_o[prow * D + d] = o;
+            if (d == 0) {
+                p.ws_m[prow] = M;
+                p.ws_l[prow] = L;
+            }
+        }
+    }
+}
+
+struct CombineParams {
+    __nv_bfloat16* out;
+    const float* ws_o;
+    const float* ws_m;
+    const float* ws_l;
+    const int32_t* seq_lens;
+    int S, Hq, P, PP, max_blocks, B;
+};
+
+// Log-sum-exp merge of the split-KV partials of one (sequence, q head) per
+// warp:  M = max_p m_p;  w_p = l_p 2^(m_p - M);  out = sum_p w_p o_p / sum_p w_p.
+// Rows whose sequence fits in one partition were written by the decode kernel
+// and are skipped here, as are partitions with an empty sum.
+template <int D>
+__global__ void __launch_bounds__(kThreads) pa_combine_kernel(const CombineParams p) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * kWarps + warp;
+    if (row >= (long long)p.S * p.Hq) return;
+    const int s = static_cast<int>(row / p.Hq);
+    int T = __ldg(p.seq_lens + s);
+    T = max(0, min(T, p.max_blocks * p.B));
+    int nb = (T + p.B - 1) / p.B;
+    const int nps = min(p.P, (nb + p.PP - 1) / p.PP);
+    if (nps <= 1) return;
+    const long long base = row * p.P;
+    float M = -INFINITY;
+    for (int i = lane; i < nps; i += 32)
+        if (p.ws_l[base + i] > 0.f) M = fmaxf(M, p.ws_m[base + i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+    constexpr int PER = D / 32;
+    float a[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) a[i] = 0.f;
+    float L = 0.f;
+    for (int i = 0; i < nps; ++i) {
+        const float l = p.ws_l[base + i];
+        if (!(l > 0.f)) continue;
+        const float wt = exp2f(p.ws_m[base + i] - M) * l;
+        L += wt;
+        const float* o = p.ws_o + (base + i) * D;
+#pragma unroll
+        for (int j = 0; j < PER; ++j) a[j] += wt * o[lane + 32 * j];
+    }
+#pragma unroll
+    for (int j = 0; j < PER; ++j)
+        p.out[row * D + lane + 32 * j] = __float2bfloat16_rn(L > 0.f ? a[j] / L : 0.f);
+}
+
+}  // namespace pa

@@ -1,0 +1,137 @@
+"""The C ABI without a GPU: the library loads, exports every declared entry
+point, rejects bad arguments before any CUDA call, and plans the split."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import paged_kv_cache_471_b200 as pa
+from paged_kv_cache_471_b200 import build as pbuild
+from paged_kv_cache_471_b200 import workloads as W
+
+HEADER = os.path.join(pbuild.INCLUDE, "pagedattn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    pbuild.build()
+    return pa.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("pa_decode", "pa_decode_ex", "pa_decode_workspace_size", "pa_plan_decode",
+              "pa_status_string", "pa_read_device_status", "pa_last_error_detail", "pa_version"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", pa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s+(\w+)$", out, flags=re.M))
+    for n in declared_functions():
+        assert n in exported, n
+        assert hasattr(L, n)
+
+
+def test_no_cuda_link_to_oracle():
+    # The product library must not carry any oracle symbol.
+    out = subprocess.run(["nm", "-D", pa.LIB_PATH], capture_output=True, text=True).stdout
+    assert "oracle" not in out
+
+
+def test_version_and_strings(L):
+    assert pa.version() >= 10000
+    for code in range(5):
+        assert L.pa_status_string(code).decode().startswith("PA_")
+    assert b"unknown" in L.pa_status_string(77)
+
+
+def _decode(L, **over):
+    args = dict(out=0x10000, query=0x20000, key_cache=0x30000, value_cache=0x40000, num_seqs=2,
+                num_heads=8, num_kv_heads=2, head_size=128, scale=0.088, block_tables=0x50000,
+                max_blocks_per_seq=4, seq_lens=0x60000, block_size=16, max_seq_len=64,
+                num_blocks=64, kv_dtype=0, k_scale=None, v_scale=None, workspace=0x70000,
+                workspace_bytes=1 << 20, stream=None, opts=ctypes.byref(pa.Options(0, 148)))
+    args.update(over)
+    return L.pa_decode_ex(*args.values())
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(out=None), pa.PA_ERR_INVALID_ARG),
+    (dict(query=0x20002), pa.PA_ERR_INVALID_ARG),
+    (dict(key_cache=None), pa.PA_ERR_INVALID_ARG),
+    (dict(value_cache=0x40008), pa.PA_ERR_INVALID_ARG),
+    (dict(block_tables=0x50002), pa.PA_ERR_INVALID_ARG),
+    (dict(seq_lens=None), pa.PA_ERR_INVALID_ARG),
+    (dict(workspace=None), pa.PA_ERR_INVALID_ARG),
+    (dict(num_heads=9), pa.PA_ERR_INVALID_ARG),
+    (dict(num_heads=34, num_kv_heads=2), pa.PA_ERR_UNSUPPORTED),
+    (dict(head_size=96), pa.PA_ERR_UNSUPPORTED),
+    (dict(block_size=8), pa.PA_ERR_UNSUPPORTED),
+    (dict(kv_dtype=5), pa.PA_ERR_UNSUPPORTED),
+    (dict(max_seq_len=65), pa.PA_ERR_INVALID_ARG),
+    (dict(max_seq_len=-1), pa.PA_ERR_INVALID_ARG),
+    (dict(num_blocks=0), pa.PA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), pa.PA_ERR_INVALID_ARG),
+    (dict(kv_dtype=1), pa.PA_ERR_INVALID_ARG),  # fp8 without scales
+    (dict(workspace_bytes=16), pa.PA_ERR_WORKSPACE_TOO_SMALL),
+    (dict(num_seqs=-1), pa.PA_ERR_INVALID_ARG),
+    (dict(max_blocks_per_seq=0), pa.PA_ERR_INVALID_ARG),
+])
+def test_rejects_before_launch(L, over, code):
+    assert _decode(L, **over) == code
+    assert L.pa_last_error_detail().decode() != ""
+
+
+def test_zero_sequences_is_a_no_op(L):
+    assert _decode(L, num_seqs=0, out=None, query=None) == pa.PA_OK
+
+
+def test_workspace_size_header_only_without_split():
+    n = pa.workspace_size(64, 32, 32, 128, 16, 4096, "bf16", num_sms=148)
+    assert n == pa.WORKSPACE_HEADER_BYTES
+
+
+def _plan(idx, **kw):
+    c = W.CONFIGS[idx]
+    return pa.plan(c.num_seqs, c.num_heads, c.num_kv_heads, c.head_size, c.block_size,
+                   c.max_seq_len, c.kv_dtype, num_sms=148, **kw)
+
+
+def test_planner_on_the_five_workloads():
+    p1, p2, p3, p4, p5 = (_plan(i) for i in range(1, 6))
+    assert p1["num_partitions"] == 1 and p1["partition_pages"] == 16
+    assert p2["num_partitions"] == 1 and p2["grid_ctas"] == 64 * 32
+    assert p3["num_partitions"] >= 2  # variable lengths: bound the last wave's tail
+    assert p4["num_partitions"] == 1 and p4["grid_ctas"] == 256 * 8
+    assert p5["num_partitions"] >= 4  # 64 (seq, kv head) units cannot fill 148 SMs
+    for p in (p1, p2, p3, p4, p5):
+        assert p["smem_bytes"] <= 227 * 1024 and 2 <= p["stages"] <= 8
+        P, PP = p["num_partitions"], p["partition_pages"]
+    c5 = W.CONFIGS[5]
+    assert p5["num_partitions"] * p5["partition_pages"] >= c5.max_blocks_per_seq
+    ws = pa.workspace_size(c5.num_seqs, c5.num_heads, c5.num_kv_heads, 128, 32, c5.max_seq_len,
+                           num_sms=148)
+    assert ws >= 256 + 8 * 32 * p5["num_partitions"] * 130 * 4
+
+
+def test_forced_partitions():
+    p = _plan(2, partition_pages=7)
+    assert p["partition_pages"] == 7 and p["num_partitions"] == -(-256 // 7)
+    p = _plan(2, partition_pages=10000)
+    assert p["num_partitions"] == 1
+
+
+def test_two_ctas_per_sm_fit_for_the_bf16_b16_pages():
+    p = _plan(2)
+    assert 2 * (p["smem_bytes"] + 1024) <= 228 * 1024

@@ -1,0 +1,162 @@
+"""Bit-exact and structural checks of the CUDA path (GPU):
+
+* one-hot probe: a single token dominates every other logit by ~500 in log2
+  units, so every other weight underflows to exactly 0 in fp32 and the output
+  is that token's V row -- bit-exact, swept over every position, across block
+  and partition boundaries (this pins the block-table gather and the K/V page
+  indexing bit for bit);
+* relabelling physical blocks (moving their data) leaves the output bit-identical;
+* uniform logits give the mean of V; seq_len 0 gives a zero row;
+* illegal block ids / lengths set status bits without any out-of-range read.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_471_b200 as pa
+from paged_kv_cache_471_b200 import workloads as W
+from parity_helpers import compare, run_gpu, run_oracle
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _cfg(D=128, B=16, G=4, kv=W.BF16, lens=(37, 200, 16, 1), Hk=2, extra_blocks=7, seed=77):
+    return W.PagedConfig(f"probe D={D} B={B} G={G} {kv}", num_seqs=len(lens), num_heads=Hk * G,
+                         num_kv_heads=Hk, head_size=D, block_size=B,
+                         num_blocks=sum(-(-t // B) for t in lens) + extra_blocks, seq_len_lo=1,
+                         seq_len_hi=max(lens), kv_dtype=kv,
+                         k_scale=0.05 if kv == W.FP8_E4M3 else 1.0,
+                         v_scale=0.05 if kv == W.FP8_E4M3 else 1.0, seed=seed)
+
+
+def _token_slot(wl, s, t):
+    B = wl.cfg.block_size
+    return int(wl.block_tables[s, t // B]), t % B
+
+
+@pytest.mark.parametrize("kv", [W.BF16, W.FP8_E4M3])
+@pytest.mark.parametrize("D,B", [(128, 16), (64, 32), (128, 32)])
+@pytest.mark.parametrize("pp", [0, 2])
+def test_one_hot_probe_bit_exact(kv, D, B, pp):
+    lens = (3 * B + 5, B, 1, 7 * B - 1)
+    cfg = _cfg(D=D, B=B, G=4, kv=kv, lens=lens)
+    wl = W.make_workload(cfg, DEV, seq_lens=list(lens))
+    kc, vc = wl.key_cache, wl.value_cache
+    x = cfg.x
+    # zero the d=0 column of every referenced K slot (NaN poison elsewhere stays)
+    for s, T in enumerate(lens):
+        for t in range(T):
+            pb, o = _token_slot(wl, s, t)
+            kc[pb, :, 0, o, 0] = 0
+    q = torch.zeros_like(wl.query)
+    q[:, :, 0] = 4096.0
+    wl.query = q
+    one = 1.0 if kv == W.BF16 else 0x7E  # bf16 1.0 / e4m3 code of 448
+    for s, T in enumerate(lens):
+        for t_star in sorted({0, T // 2, T - 1, min(B, T - 1), min(2 * B - 1, T - 1)}):
+            pb, o = _token_slot(wl, s, t_star)
+            old = kc[pb, :, 0, o, 0].clone()
+            kc[pb, :, 0, o, 0] = one if kv == W.BF16 else torch.full_like(old, one)
+            out = run_gpu(wl, partition_pages=pp)
+            torch.cuda.synchronize()
+            for g in range(cfg.num_kv_heads):
+                v = wl.value_cache[pb, g, :, o]
+                if kv == W.BF16:
+                    want = v
+                else:
+                    want = (v.view(torch.float8_e4m3fn).float() * cfg.v_scale).to(torch.bfloat16)
+                for h in range(g * cfg.group, (g + 1) * cfg.group):
+                    got = out[s, h]
+                    assert torch.equal(got.view(torch.int16), want.view(torch.int16)), \
+                        (s, t_star, h, got[:4], want[:4])
+            kc[pb, :, 0, o, 0] = old
+
+
+@pytest.mark.parametrize("kv", [W.BF16, W.FP8_E4M3])
+def test_block_relabelling_bit_identical(kv):
+    lens = [500, 33, 129]
+    cfg = _cfg(kv=kv, lens=lens, extra_blocks=20, G=8)
+    wl = W.make_workload(cfg, DEV, seq_lens=lens)
+    a = run_gpu(wl).clone()
+    g = torch.Generator().manual_seed(5)
+    perm = torch.randperm(cfg.num_blocks, generator=g).to(DEV)
+    kc2 = torch.empty_like(wl.key_cache)
+    vc2 = torch.empty_like(wl.value_cache)
+    kc2[perm] = wl.key_cache
+    vc2[perm] = wl.value_cache
+    bt = wl.block_tables.long()
+    bt2 = torch.where(bt >= 0, perm[bt.clamp(min=0)], bt).to(torch.int32)
+    wl.key_cache, wl.value_cache, wl.block_tables = kc2, vc2, bt2.contiguous()
+    b = run_gpu(wl)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_uniform_logits_mean():
+    lens = [1000, 17]
+    cfg = _cfg(lens=lens, G=8)
+    wl = W.make_workload(cfg, DEV, seq_lens=lens)
+    wl.query = torch.zeros_like(wl.query)
+    out = run_gpu(wl)
+    torch.cuda.synchronize()
+    ref = run_oracle(wl)
+    compare(out, ref, cfg.kv_dtype, "uniform logits")
+
+
+def test_zero_length_sequence_and_split_agreement():
+    lens = [0, 300, 0, 4096, 5]
+    cfg = _cfg(lens=lens, G=4)
+    wl = W.make_workload(cfg, DEV, seq_lens=lens)
+    ref = run_oracle(wl)
+    outs = []
+    for pp in (0, 1, 2, 7, 1000):
+        o = run_gpu(wl, partition_pages=pp)
+        torch.cuda.synchronize()
+        compare(o, ref, cfg.kv_dtype, f"pp={pp}")
+        assert (o[0] == 0).all() and (o[2] == 0).all()
+        outs.append(o.float())
+    for o in outs[1:]:
+        # different partitions change only fp32 rounding before the bf16 store
+        assert torch.allclose(o, outs[0], rtol=2 ** -7, atol=1e-6)
+
+
+def test_non_default_stream():
+    cfg = W.reduced(3, num_seqs=3, seq_len_hi=900, seq_len_lo=100)
+    wl = W.make_workload(cfg, DEV)
+    st = torch.cuda.Stream(DEV)
+    out = torch.empty_like(wl.query)
+    st.wait_stream(torch.cuda.current_stream(DEV))
+    with torch.cuda.stream(st):
+        run_gpu(wl, out=out, stream=st)
+    st.synchronize()
+    compare(out, run_oracle(wl), cfg.kv_dtype, "side stream")
+
+
+def test_bad_block_id_and_length_flags():
+    lens = [100, 64]
+    cfg = _cfg(lens=lens)
+    wl = W.make_workload(cfg, DEV, seq_lens=lens)
+    ws = torch.zeros(pa.workspace_size(2, cfg.num_heads, 2, 128, 16, 100), dtype=torch.uint8,
+                     device=DEV)
+    good = run_gpu(wl, ws=ws)
+    torch.cuda.synchronize()
+    assert pa.read_status(ws) == 0
+    bt = wl.block_tables.clone()
+    wl.block_tables[0, 2] = cfg.num_blocks + 1000  # out of range
+    wl.block_tables[1, 1] = -1
+    out = run_gpu(wl, ws=ws)
+    torch.cuda.synchronize()
+    st = pa.read_status(ws, clear=True)
+    assert st & pa.PA_DEV_BAD_BLOCK_ID
+    assert torch.isfinite(out.float()).all()
+    # the skipped block's tokens drop out; other rows are untouched
+    wl.block_tables = bt
+    wl.seq_lens[1] = 10 ** 6  # longer than the block table row
+    out = run_gpu(wl, ws=ws)
+    torch.cuda.synchronize()
+    assert pa.read_status(ws, clear=True) & pa.PA_DEV_SEQ_LEN_OUT_OF_RANGE
+    assert torch.isfinite(out[0].float()).all()
+    assert torch.equal(out[0], good[0])
+    assert pa.read_status(ws) == 0

@@ -1,0 +1,83 @@
+"""CUDA path vs the fp64 oracle, element by element (GPU)."""
+
+import itertools
+
+import pytest
+import torch
+
+import paged_kv_cache_471_b200 as pa
+from paged_kv_cache_471_b200 import workloads as W
+from parity_helpers import compare, run_gpu, run_oracle, run_oracle_sampled, sample_pairs
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    pa.lib()  # fails loudly when the library is missing
+
+
+# Reduced versions of the five workloads: same heads, head size, block size,
+# dtype and length mix; sizes the oracle finishes in seconds, still many
+# pages per (sequence, kv head) and ragged last blocks.
+REDUCED = {
+    1: W.CONFIGS[1],  # already tiny
+    2: W.reduced(2, num_seqs=3, seq_len_hi=1000, seq_len_lo=700),
+    3: W.reduced(3, num_seqs=6, seq_len_hi=2100, seq_len_lo=100),
+    4: W.reduced(4, num_seqs=4, seq_len_hi=1500, seq_len_lo=900),
+    5: W.reduced(5, num_seqs=3, seq_len_hi=5000, seq_len_lo=4100, shared_prefix_blocks=40),
+}
+
+
+@pytest.mark.parametrize("idx", sorted(REDUCED))
+@pytest.mark.parametrize("partition_pages", [0, 3, 16])
+def test_reduced_workloads(idx, partition_pages):
+    cfg = REDUCED[idx]
+    wl = W.make_workload(cfg, DEV)
+    out = run_gpu(wl, partition_pages=partition_pages)
+    torch.cuda.synchronize()
+    ref = run_oracle(wl)
+    compare(out, ref, cfg.kv_dtype, f"cfg{idx} pp={partition_pages}")
+    assert pa.read_status(device=DEV) == 0
+
+
+SHAPES = list(itertools.product([64, 128], [16, 32], [1, 4, 8, 16], [W.BF16, W.FP8_E4M3]))
+
+
+@pytest.mark.parametrize("D,B,G,kv", SHAPES, ids=lambda v: str(v))
+def test_shapes(D, B, G, kv):
+    Hk = 2
+    lens = [1, B - 1, B, B + 1, 3 * B + 5, 17 * B - 1, 40 * B + 3]
+    cfg = W.PagedConfig(f"shape D={D} B={B} G={G} {kv}", num_seqs=len(lens), num_heads=Hk * G,
+                        num_kv_heads=Hk, head_size=D, block_size=B,
+                        num_blocks=sum(-(-t // B) for t in lens) + 9, seq_len_lo=1,
+                        seq_len_hi=max(lens), kv_dtype=kv,
+                        k_scale=0.05 if kv == W.FP8_E4M3 else 1.0,
+                        v_scale=0.04 if kv == W.FP8_E4M3 else 1.0, seed=4242 + D + B + G)
+    wl = W.make_workload(cfg, DEV, seq_lens=lens)
+    ref = run_oracle(wl)
+    for pp in (0, 4):
+        out = run_gpu(wl, partition_pages=pp)
+        torch.cuda.synchronize()
+        compare(out, ref, kv, f"{cfg.name} pp={pp}")
+
+
+@pytest.mark.parametrize("idx", [1, 2, 3, 4, 5])
+def test_full_size_sampled(idx):
+    """Full workload in the launch configuration the bench times; sampled rows
+    against the oracle, plus whole-output sanity (finite, no poison)."""
+    cfg = W.CONFIGS[idx]
+    wl = W.make_workload(cfg, DEV)
+    out = run_gpu(wl)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+    n = 24 if idx != 5 else 10
+    pairs = sample_pairs(cfg, n, seed=idx)
+    ref = run_oracle_sampled(wl, pairs)
+    got = torch.stack([out[s, h] for s, h in pairs])
+    compare(got, ref, cfg.kv_dtype, f"full cfg{idx}")
+    assert pa.read_status(device=DEV) == 0
+    del wl, out
+    torch.cuda.empty_cache()
