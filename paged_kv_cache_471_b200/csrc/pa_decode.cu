@@ -17,6 +17,7 @@ constexpr int kVersion = 10000;  // 1.0.0
 constexpr size_t kSmemBudget = 110 * 1024;  // per CTA, so that two CTAs share an SM
 constexpr size_t kSmemPerSm = 228 * 1024;
 constexpr size_t kSmemReservedPerCta = 1024;
+constexpr size_t kMaxSmemPerCta = 227 * 1024;  // opt-in limit of sm_100
 constexpr int kMinPartitionPages = 16;
 constexpr int kMaxStages = 8;
 constexpr int kMaxDevices = 64;
@@ -145,27 +146,29 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
     return PA_OK;
 }
 
+// Raise the kernel's dynamic shared-memory limit once per device.  `done` is
+// owned by the caller's template instantiation, so every kernel variant keeps
+// its own flags.
 template <typename K>
-cudaError_t ensure_smem(K kernel, size_t smem) {
-    // One attribute call per device and instantiation (the kernel asks for the
-    // planner's largest stage area, so later calls never need more).
-    static std::atomic<int> done[kMaxDevices];
+cudaError_t ensure_smem(K kernel, std::atomic<int>* done) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    const bool cached = dev >= 0 && dev < kMaxDevices;
+    if (cached && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBudget + 32 * 1024));
-    if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
-    (void)smem;
+                             static_cast<int>(kMaxSmemPerCta));
+    if (e == cudaSuccess && cached) done[dev].store(1, std::memory_order_release);
     return e;
 }
 
 template <int D, int B, bool FP8, int NH>
 cudaError_t launch_decode(const pa::DecodeParams& p, long long grid, size_t smem,
                           cudaStream_t st) {
+    static std::atomic<int> done[kMaxDevices];
     auto kern = pa::pa_decode_kernel<D, B, FP8, NH>;
-    cudaError_t e = ensure_smem(kern, smem);
+    if (smem > kMaxSmemPerCta) return cudaErrorInvalidValue;
+    cudaError_t e = ensure_smem(kern, done);
     if (e != cudaSuccess) return e;
     kern<<<static_cast<unsigned>(grid), pa::kThreads, smem, st>>>(p);
     return cudaGetLastError();

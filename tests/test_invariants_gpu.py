@@ -118,8 +118,11 @@ def test_zero_length_sequence_and_split_agreement():
         assert (o[0] == 0).all() and (o[2] == 0).all()
         outs.append(o.float())
     for o in outs[1:]:
-        # different partitions change only fp32 rounding before the bf16 store
-        assert torch.allclose(o, outs[0], rtol=2 ** -7, atol=1e-6)
+        # Each partitioning rounds the softmax weights to bf16 against its own
+        # running max, so results differ by O(2^-9 / sqrt(T)) absolute, not by
+        # a relative bf16 ulp; they must agree far inside the oracle tolerance.
+        d = (o - outs[0]).abs()
+        assert d.max().item() <= 2e-3 and d.mean().item() <= 1e-4, (d.max(), d.mean())
 
 
 def test_non_default_stream():
