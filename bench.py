@@ -180,22 +180,30 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- GPU arm
 def bytes_of(wl):
-    return wl.kv_bytes + wl.q_out_bytes
+    """Algorithmic bytes of one step: K+V of every token read once, plus Q and
+    out.  With a shared prefix the K/V of shared blocks count once (unique
+    bytes), the conservative figure; the logical count is reported beside it."""
+    kv = wl.unique_kv_bytes if wl.cfg.shared_prefix_blocks else wl.kv_bytes
+    return kv + wl.q_out_bytes
 
 
-def make_device_workload(idx: int, device):
+def workload_config(idx: int, num_seqs: int = 0):
+    """The named workload, or the same shape with fewer sequences and a pool
+    sized to them (used for small profiler captures)."""
     from paged_kv_cache_471_b200 import workloads as W
-    return W.make_workload(W.CONFIGS[idx], device)
+    if num_seqs and num_seqs < W.CONFIGS[idx].num_seqs:
+        return W.reduced(idx, num_seqs=num_seqs)
+    return W.CONFIGS[idx]
 
 
-def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0):
+def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, num_seqs=0):
     import torch
 
     import paged_kv_cache_471_b200 as pa
     from paged_kv_cache_471_b200 import workloads as W
 
-    cfg = W.CONFIGS[idx]
-    wl = make_device_workload(idx, device)
+    cfg = workload_config(idx, num_seqs)
+    wl = W.make_workload(cfg, device)
     out = torch.empty_like(wl.query)
     plan = pa.plan(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_size, cfg.block_size,
                    cfg.max_seq_len, cfg.kv_dtype)
@@ -370,6 +378,7 @@ def result_line(idx, r, n_gpus, steps, warmup, cpu=None):
             "block_size": cfg.block_size, "num_blocks": cfg.num_blocks,
             "sum_seq_lens": int(r["wl"].seq_lens.sum()),
             "bytes_per_step": r["alg_bytes"],
+            "logical_bytes_per_step": r["wl"].kv_bytes + r["wl"].q_out_bytes,
             "seqs_per_s": round(cfg.num_seqs * n_gpus / (r["step_ms"] * 1e-3), 1),
             "pct_of_8TBs_spec": round(100 * gbs / SPEC_HBM_GBS, 2),
             f"pct_of_{peak_kind}_hbm": round(100 * gbs / peak, 2),
@@ -454,6 +463,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--num-seqs", type=int, default=0,
+                    help="run the workload with fewer sequences (profiling captures only)")
     ap.add_argument("--ref-budget", type=float, default=20.0,
                     help="seconds of CPU time for the reference arm's timed steps")
     args = ap.parse_args(argv)
@@ -476,7 +487,8 @@ def main(argv=None):
 
     configs = [1, 2, 3, 4, 5] if args.config == "all" else [int(args.config)]
     for idx in configs:
-        r = time_gpu(idx, args.steps, args.warmup, device, want_e2e=not args.no_e2e, rank=rank)
+        r = time_gpu(idx, args.steps, args.warmup, device, want_e2e=not args.no_e2e, rank=rank,
+                     num_seqs=args.num_seqs)
         r["step_ms"] = reduce_max(r["step_ms"], device)
         if "e2e_ms" in r:
             r["e2e_ms"] = reduce_max(r["e2e_ms"], device)

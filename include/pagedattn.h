@@ -84,10 +84,13 @@ typedef enum pa_kv_dtype {
  *      longest sequence's block count means "no split".
  *  num_sms: 0 queries the current device; > 0 plans for that many SMs
  *      (lets the host plan without a GPU, e.g. to size a workspace).
+ *  stages: 0 lets the planner choose; 2..16 forces that many page buffers
+ *      per warp (shared memory grows with it; more than fits is rejected).
  */
 typedef struct pa_options {
     int partition_pages;
     int num_sms;
+    int stages;
 } pa_options;
 
 /* What pa_decode will launch for a given problem. */

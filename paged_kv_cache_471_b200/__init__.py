@@ -45,7 +45,8 @@ class PagedAttentionError(RuntimeError):
 
 
 class Options(ctypes.Structure):
-    _fields_ = [("partition_pages", ctypes.c_int), ("num_sms", ctypes.c_int)]
+    _fields_ = [("partition_pages", ctypes.c_int), ("num_sms", ctypes.c_int),
+                ("stages", ctypes.c_int)]
 
 
 class Plan(ctypes.Structure):
@@ -109,10 +110,10 @@ def _check(rc: int):
                                       f"{L.pa_last_error_detail().decode()}")
 
 
-def _opts(partition_pages=0, num_sms=0):
-    if not partition_pages and not num_sms:
+def _opts(partition_pages=0, num_sms=0, stages=0):
+    if not partition_pages and not num_sms and not stages:
         return None
-    return ctypes.byref(Options(int(partition_pages), int(num_sms)))
+    return ctypes.byref(Options(int(partition_pages), int(num_sms), int(stages)))
 
 
 def kv_dtype_code(kv_dtype) -> int:
@@ -123,11 +124,11 @@ def kv_dtype_code(kv_dtype) -> int:
 
 
 def plan(num_seqs, num_heads, num_kv_heads, head_size, block_size, max_seq_len, kv_dtype="bf16",
-         partition_pages=0, num_sms=0) -> dict:
+         partition_pages=0, num_sms=0, stages=0) -> dict:
     p = Plan()
     _check(lib().pa_plan_decode(ctypes.byref(p), num_seqs, num_heads, num_kv_heads, head_size,
                                 block_size, max_seq_len, kv_dtype_code(kv_dtype),
-                                _opts(partition_pages, num_sms)))
+                                _opts(partition_pages, num_sms, stages)))
     return p.as_dict()
 
 
@@ -174,7 +175,8 @@ def _ptr(t, name, dtypes=None, device=None):
 
 def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, block_tables,
            seq_lens, block_size: int, max_seq_len: int, kv_dtype="bf16", k_scale=None,
-           v_scale=None, workspace_tensor=None, partition_pages: int = 0, stream=None):
+           v_scale=None, workspace_tensor=None, partition_pages: int = 0, stream=None,
+           stages: int = 0):
     """Paged decode attention into ``out`` (bf16 [num_seqs, num_heads, head_size]).
 
     key_cache: [num_blocks, num_kv_heads, head_size/x, block_size, x];
@@ -220,7 +222,7 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
                             block_tables.shape[1], sl, int(block_size), int(max_seq_len),
                             int(num_blocks), code, ks, vs, ws,
                             workspace_tensor.numel() * workspace_tensor.element_size(),
-                            st.cuda_stream, _opts(partition_pages, 0))
+                            st.cuda_stream, _opts(partition_pages, 0, stages))
     _check(rc)
     return out
 

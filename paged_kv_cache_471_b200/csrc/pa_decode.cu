@@ -14,12 +14,13 @@
 namespace {
 
 constexpr int kVersion = 10000;  // 1.0.0
-constexpr size_t kSmemBudget = 110 * 1024;  // per CTA, so that two CTAs share an SM
 constexpr size_t kSmemPerSm = 228 * 1024;
 constexpr size_t kSmemReservedPerCta = 1024;
 constexpr size_t kMaxSmemPerCta = 227 * 1024;  // opt-in limit of sm_100
 constexpr int kMinPartitionPages = 16;
-constexpr int kMaxStages = 8;
+constexpr int kDefaultStages = 2;
+constexpr long long kMaxCtasPerSm = 3;
+constexpr int kMaxForcedStages = 16;
 constexpr int kMaxDevices = 64;
 
 thread_local char g_detail[256] = "";
@@ -88,16 +89,22 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
     if (sms == 0 && device_sms(&sms) != 0)
         return fail(PA_ERR_CUDA, "%s", "cannot query the SM count of the current device");
 
+    if (opts && (opts->stages < 0 || opts->stages == 1 || opts->stages > kMaxForcedStages))
+        return fail(PA_ERR_INVALID_ARG, "%s", "opts->stages must be 0 or 2..16");
+    // Two page buffers per warp: measured on B200, more resident CTAs beat
+    // deeper per-warp rings for the same bytes in flight.
     const size_t stage = 2ull * head_size * block_size * elem_bytes(kv_dtype);
-    int ns = static_cast<int>(kSmemBudget / (pa::kWarps * stage));
-    ns = ns < 2 ? 2 : (ns > kMaxStages ? kMaxStages : ns);
+    int ns = kDefaultStages;
+    if (opts && opts->stages > 0) ns = opts->stages;
     size_t stage_area = static_cast<size_t>(pa::kWarps) * ns * stage;
     const size_t mb = merge_bytes(head_size, num_heads / num_kv_heads);
     if (stage_area < mb) stage_area = mb;
     const size_t smem = stage_area + static_cast<size_t>(pa::kWarps) * ns * 8;
+    if (smem > kMaxSmemPerCta)
+        return fail(PA_ERR_INVALID_ARG, "%s", "too many stages for shared memory");
     long long per_sm = static_cast<long long>(kSmemPerSm / (smem + kSmemReservedPerCta));
     if (per_sm < 1) per_sm = 1;
-    if (per_sm > 2) per_sm = 2;
+    if (per_sm > kMaxCtasPerSm) per_sm = kMaxCtasPerSm;  // register limit
     const long long slots = static_cast<long long>(sms) * per_sm;
 
     const long long pages_max = (static_cast<long long>(max_seq_len) + block_size - 1) / block_size;
@@ -117,8 +124,23 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         if (target >= pages_max) {
             pp = pages_max;
         } else {
-            const long long nparts = (pages_max + target - 1) / target;
-            pp = (pages_max + nparts - 1) / nparts;
+            // Among P0..2*P0 partitions pick the one whose last wave of CTAs is
+            // fullest (CTAs of equal length run in whole waves of `slots`).
+            const long long p0 = (pages_max + target - 1) / target;
+            long long best = p0;
+            double best_eff = -1.0;
+            for (long long np = p0; np <= 2 * p0; ++np) {
+                const long long ppc = (pages_max + np - 1) / np;
+                const long long npe = (pages_max + ppc - 1) / ppc;  // partitions really used
+                if (npe != np) continue;
+                const double waves = static_cast<double>(units * np) / static_cast<double>(slots);
+                const double eff = waves / std::ceil(waves) - 0.002 * static_cast<double>(np - p0);
+                if (eff > best_eff + 1e-9) {
+                    best_eff = eff;
+                    best = np;
+                }
+            }
+            pp = (pages_max + best - 1) / best;
         }
     }
     if (pp < 1) pp = 1;

@@ -32,6 +32,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "pa_ptx.cuh"
 
 namespace pa {
@@ -147,7 +149,10 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
     const size_t head_off = static_cast<size_t>(kvh) * PAGE;
     const size_t block_stride = static_cast<size_t>(p.Hk) * PAGE;
 
-    // Issue the copies of this warp's i-th page (warp-uniform call).
+    // Issue the copies of this warp's i-th page (warp-uniform call, pages in
+    // increasing order).  Page i lives in stage i mod NS; `issue_stage` tracks
+    // that without a division.
+    int issue_stage = 0;
     auto issue = [&](int i) {
         if (i >= wbase + 32) {
             win_a = win_b;
@@ -155,7 +160,8 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
             wbase += 32;
         }
         const int pb = __shfl_sync(kFull, win_a, i & 31);
-        const int stage = i % NS;
+        const int stage = issue_stage;
+        issue_stage = (issue_stage + 1 == NS) ? 0 : issue_stage + 1;
         const uint32_t bar = bar0 + 8 * stage;
         const bool ok = pb >= 0 && static_cast<long long>(pb) < p.num_blocks;
         if (lane == 0) {
@@ -258,19 +264,10 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
     const int src1 = quad0 | ((2 * cq + 1) & 3);
     const bool hi_half = cq >= 2;
 
-    bool timed_out = false;
-    int k = 0;
-    for (; k < n_my; ++k) {
-        const int stage = k % NS;
-        const uint32_t bar = bar0 + 8 * stage;
-        const bool landed = mbar_wait_bounded(bar, static_cast<uint32_t>((k / NS) & 1));
-        if (!__all_sync(kFull, landed)) {
-            timed_out = true;
-            break;
-        }
-        const int jg = j0 + warp + kWarps * k;
-        const int valid = ((valid_mask >> stage) & 1u) ? min(B, T - jg * B) : 0;
-        const uint32_t kbase = wstage0 + static_cast<uint32_t>(stage * STAGE);
+    // One landed page: S = Q K^T, online softmax, O^T += V^T P^T.  FULL pages
+    // (every slot a token) skip all masking.
+    auto page = [&](auto full_tag, const uint32_t kbase, const int valid) {
+        constexpr bool FULL = decltype(full_tag)::value;
         const uint32_t vbase = kbase + PAGE;
 
         // ---------------- S = Q K^T  (rows: heads, cols: tokens)
@@ -314,6 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
         // ---------------- online softmax (log2 domain), per head row
         uint32_t pp[NH][NT];
         float alpha[NH];
+        bool grew = false;
 #pragma unroll
         for (int r = 0; r < NH; ++r) {
             float v[NT][2];
@@ -323,7 +321,9 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     float x = sc[nt][2 * r + e] * qk_mul;
-                    if (valid < B && 8 * nt + 2 * cq + e >= valid) x = -INFINITY;
+                    if constexpr (!FULL) {
+                        if (8 * nt + 2 * cq + e >= valid) x = -INFINITY;
+                    }
                     v[nt][e] = x;
                     mx = fmaxf(mx, x);
                 }
@@ -331,13 +331,14 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
             mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
             const float m_new = fmaxf(m_run[r], mx);
             const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-            alpha[r] = exp2f(m_run[r] - m_use);
+            grew |= m_new > m_run[r];
+            alpha[r] = fast_exp2(m_run[r] - m_use);
             m_run[r] = m_new;
             float ls = 0.f;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                const float p0 = exp2f(v[nt][0] - m_use);
-                const float p1 = exp2f(v[nt][1] - m_use);
+                const float p0 = fast_exp2(v[nt][0] - m_use);
+                const float p1 = fast_exp2(v[nt][1] - m_use);
                 uint32_t w;
                 if constexpr (!FP8) {
                     w = pack_bf16x2(p0, p1);
@@ -351,17 +352,20 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
             l_run[r] = l_run[r] * alpha[r] + ls;
         }
 
-        // ---------------- rescale O^T columns (heads 8r + 2cq, 8r + 2cq + 1)
+        // ---------------- rescale O^T columns (heads 8r + 2cq, 8r + 2cq + 1),
+        // only when some row maximum of the warp moved.
+        if (__any_sync(kFull, grew)) {
 #pragma unroll
-        for (int r = 0; r < NH; ++r) {
-            const float a0 = __shfl_sync(kFull, alpha[r], 8 * cq);
-            const float a1 = __shfl_sync(kFull, alpha[r], 8 * cq + 4);
+            for (int r = 0; r < NH; ++r) {
+                const float a0 = __shfl_sync(kFull, alpha[r], 8 * cq);
+                const float a1 = __shfl_sync(kFull, alpha[r], 8 * cq + 4);
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                acc[mt][r][0] *= a0;
-                acc[mt][r][1] *= a1;
-                acc[mt][r][2] *= a0;
-                acc[mt][r][3] *= a1;
+                for (int mt = 0; mt < MT; ++mt) {
+                    acc[mt][r][0] *= a0;
+                    acc[mt][r][1] *= a1;
+                    acc[mt][r][2] *= a0;
+                    acc[mt][r][3] *= a1;
+                }
             }
         }
 
@@ -382,8 +386,10 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
                 pb0[r] = hi_half ? y0 : x0;
                 pb1[r] = hi_half ? y1 : x1;
             }
+            // Slots past the sequence end may hold anything (even NaN); their
+            // weights are 0, but 0 * NaN is NaN, so their V is zeroed.
             uint32_t mlo = kFull, mhi = kFull;
-            if (valid < B) {
+            if constexpr (!FULL) {
                 const int t0 = 16 * kk + 4 * cq;
                 mlo = (t0 < valid ? 0x0000ffffu : 0u) | (t0 + 1 < valid ? 0xffff0000u : 0u);
                 mhi = (t0 + 2 < valid ? 0x0000ffffu : 0u) | (t0 + 3 < valid ? 0xffff0000u : 0u);
@@ -394,7 +400,13 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
                     const uint32_t ra = vbase + (16 * mt + gq) * (B * 2) + kk * 32 + cq * 8;
                     const uint2 va = lds64(ra);
                     const uint2 vb = lds64(ra + 8 * (B * 2));
-                    const uint32_t a[4] = {va.x & mlo, vb.x & mlo, va.y & mhi, vb.y & mhi};
+                    uint32_t a[4] = {va.x, vb.x, va.y, vb.y};
+                    if constexpr (!FULL) {
+                        a[0] &= mlo;
+                        a[1] &= mlo;
+                        a[2] &= mhi;
+                        a[3] &= mhi;
+                    }
 #pragma unroll
                     for (int r = 0; r < NH; ++r) mma_bf16_16816(acc[mt][r], a, pb0[r], pb1[r]);
                 }
@@ -403,10 +415,20 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
                 for (int mp = 0; mp < MT / 2; ++mp) {
                     uint32_t w0, w1, w2, w3;
                     ldsm_x4(vbase + (32 * mp + lane) * B + kk * 16, w0, w1, w2, w3);
-                    const uint32_t a0[4] = {e4m3_lo_pair(w0) & mlo, e4m3_lo_pair(w1) & mlo,
-                                            e4m3_hi_pair(w0) & mhi, e4m3_hi_pair(w1) & mhi};
-                    const uint32_t a1[4] = {e4m3_lo_pair(w2) & mlo, e4m3_lo_pair(w3) & mlo,
-                                            e4m3_hi_pair(w2) & mhi, e4m3_hi_pair(w3) & mhi};
+                    uint32_t a0[4] = {e4m3_lo_pair(w0), e4m3_lo_pair(w1), e4m3_hi_pair(w0),
+                                      e4m3_hi_pair(w1)};
+                    uint32_t a1[4] = {e4m3_lo_pair(w2), e4m3_lo_pair(w3), e4m3_hi_pair(w2),
+                                      e4m3_hi_pair(w3)};
+                    if constexpr (!FULL) {
+                        a0[0] &= mlo;
+                        a0[1] &= mlo;
+                        a0[2] &= mhi;
+                        a0[3] &= mhi;
+                        a1[0] &= mlo;
+                        a1[1] &= mlo;
+                        a1[2] &= mhi;
+                        a1[3] &= mhi;
+                    }
 #pragma unroll
                     for (int r = 0; r < NH; ++r) {
                         mma_f16_16816(acc[2 * mp][r], a0, pb0[r], pb1[r]);
@@ -415,17 +437,44 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
                 }
             }
         }
+    };
 
+    bool timed_out = false;
+    int k = 0;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (; k < n_my; ++k) {
+        const bool landed = mbar_wait_bounded(bar0 + 8 * stage, phase);
+        if (!__all_sync(kFull, landed)) {
+            timed_out = true;
+            break;
+        }
+        const int jg = j0 + warp + kWarps * k;
+        const int valid = ((valid_mask >> stage) & 1u) ? min(B, T - jg * B) : 0;
+        const uint32_t kbase = wstage0 + static_cast<uint32_t>(stage * STAGE);
+        if (valid == B)
+            page(std::true_type{}, kbase, valid);
+        else
+            page(std::false_type{}, kbase, valid);
         __syncwarp();
         if (k + NS < n_my) issue(k + NS);
+        if (++stage == NS) {
+            stage = 0;
+            phase ^= 1u;
+        }
     }
 
     if (timed_out) {
         // Let the copies already in flight land (bounded) before the CTA's
         // shared memory can be handed to anyone else, then report.
         const int last = min(n_my, k + NS);
-        for (int i = k; i < last; ++i)
-            (void)mbar_wait_bounded(bar0 + 8 * (i % NS), static_cast<uint32_t>((i / NS) & 1));
+        for (int i = k; i < last; ++i) {
+            (void)mbar_wait_bounded(bar0 + 8 * stage, phase);
+            if (++stage == NS) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
         if (lane == 0) atomicOr(p.status, kDevTimeout);
     }
 
