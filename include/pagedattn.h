@@ -160,6 +160,40 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
                        size_t workspace_bytes, void* stream, const pa_options* opts);
 
 /*
+ * pa_decode without a caller-supplied workspace, for callers that cannot
+ * allocate device memory at the point of the call -- for example code that
+ * runs inside an allocator callback, a runtime whose memory pool is owned and
+ * fully reserved by someone else, or a plugin whose host framework forbids
+ * device allocations after start-up.  The decoding pages state no such need;
+ * this entry point has no counterpart there.
+ *
+ * Scratch (the split-KV partials) lives in one fixed array of
+ * PA_NOALLOC_SCRATCH_BYTES in the library's own device memory, reserved on
+ * every GPU that loads the library until the process exits.  Problems whose
+ * plan needs more than that (pa_decode_workspace_size > PA_NOALLOC_SCRATCH_BYTES)
+ * are rejected with PA_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ * No allocation is made: no cudaMalloc, cudaFree or allocating library call.
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * Every call on a device shares the one array and it keeps the last call's
+ * contents; calls that can overlap on the GPU (other streams, other host
+ * threads) race on it and must be serialised by the caller.  Nothing in the
+ * array needs to start at zero: each call writes every partial it reads.  The
+ * device-side range-check bits (PA_DEV_*) of this entry point are recorded in
+ * the array but are not reported; use pa_decode with a workspace to read them.
+ * Other arguments, pointers and errors are those of pa_decode.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+pa_status pa_decode_noalloc(void* out, const void* query, const void* key_cache,
+                            const void* value_cache, int num_seqs, int num_heads, int num_kv_heads,
+                            int head_size, float scale, const int32_t* block_tables,
+                            int max_blocks_per_seq, const int32_t* seq_lens, int block_size,
+                            int max_seq_len, int64_t num_blocks, pa_kv_dtype kv_dtype,
+                            const float* k_scale, const float* v_scale, void* stream);
+
+/*
  * Copy the workspace status word to *flags (synchronises `stream`), and
  * zero it afterwards when clear != 0.
  */

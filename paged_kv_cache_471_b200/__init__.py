@@ -33,6 +33,7 @@ PA_DEV_SEQ_LEN_OUT_OF_RANGE = 0x2
 PA_DEV_WAIT_TIMEOUT = 0x4
 
 WORKSPACE_HEADER_BYTES = 256
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 _KV = {"bf16": PA_KV_BF16, "auto": PA_KV_BF16, "fp8": PA_KV_FP8_E4M3, "fp8_e4m3": PA_KV_FP8_E4M3,
        PA_KV_BF16: PA_KV_BF16, PA_KV_FP8_E4M3: PA_KV_FP8_E4M3}
@@ -73,6 +74,8 @@ def _bind(lib):
     lib.pa_decode.restype = _I
     lib.pa_decode_ex.argtypes = decode_args + [ctypes.POINTER(Options)]
     lib.pa_decode_ex.restype = _I
+    lib.pa_decode_noalloc.argtypes = decode_args[:18] + [_P]
+    lib.pa_decode_noalloc.restype = _I
     lib.pa_plan_decode.argtypes = [ctypes.POINTER(Plan), _I, _I, _I, _I, _I, _I, _I,
                                    ctypes.POINTER(Options)]
     lib.pa_plan_decode.restype = _I
@@ -223,6 +226,35 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
                             int(num_blocks), code, ks, vs, ws,
                             workspace_tensor.numel() * workspace_tensor.element_size(),
                             st.cuda_stream, _opts(partition_pages, 0, stages))
+    _check(rc)
+    return out
+
+
+def decode_noalloc(out, query, key_cache, value_cache, num_kv_heads: int, scale: float,
+                   block_tables, seq_lens, block_size: int, max_seq_len: int, kv_dtype="bf16",
+                   k_scale=None, v_scale=None, stream=None):
+    """``decode`` for callers that may not allocate device memory when they
+    call: the split-KV scratch is the library's own fixed device array
+    (NOALLOC_SCRATCH_BYTES per GPU), so nothing is allocated here.  Calls that
+    overlap on the GPU share that array and must be serialised by the caller;
+    the first call on a device should come before any stream capture."""
+    import torch
+    code = kv_dtype_code(kv_dtype)
+    dev = query.device
+    S, Hq, D = query.shape
+    kv_types = (torch.bfloat16,) if code == PA_KV_BF16 else (torch.uint8, torch.float8_e4m3fn)
+    ks = vs = None
+    if code == PA_KV_FP8_E4M3:
+        ks = _ptr(k_scale, "k_scale", (torch.float32,), dev)
+        vs = _ptr(v_scale, "v_scale", (torch.float32,), dev)
+    st = stream if stream is not None else torch.cuda.current_stream(dev)
+    rc = lib().pa_decode_noalloc(
+        _ptr(out, "out", (torch.bfloat16,), dev), _ptr(query, "query", (torch.bfloat16,), dev),
+        _ptr(key_cache, "key_cache", kv_types, dev), _ptr(value_cache, "value_cache", kv_types, dev),
+        S, Hq, int(num_kv_heads), D, float(scale),
+        _ptr(block_tables, "block_tables", (torch.int32,), dev), block_tables.shape[1],
+        _ptr(seq_lens, "seq_lens", (torch.int32,), dev), int(block_size), int(max_seq_len),
+        int(key_cache.shape[0]), code, ks, vs, st.cuda_stream)
     _check(rc)
     return out
 

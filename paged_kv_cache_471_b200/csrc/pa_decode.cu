@@ -226,6 +226,36 @@ cudaError_t launch_combine(const pa::CombineParams& c, int D, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+// Scratch of pa_decode_noalloc: one fixed array per device, in the
+// library's own device memory (no allocation at call time).
+constexpr size_t kNoallocScratchBytes = PA_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device with that device current, and cached.
+pa_status noalloc_scratch(void** out) {
+    static std::atomic<void*> addr[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    const bool cached = dev >= 0 && dev < kMaxDevices;
+    if (cached) {
+        void* p = addr[dev].load(std::memory_order_acquire);
+        if (p) {
+            *out = p;
+            return PA_OK;
+        }
+    }
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+        return fail(PA_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    if (cached) addr[dev].store(p, std::memory_order_release);
+    *out = p;
+    return PA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -357,6 +387,36 @@ pa_status pa_decode(void* out, const void* query, const void* key_cache, const v
                         head_size, scale, block_tables, max_blocks_per_seq, seq_lens, block_size,
                         max_seq_len, num_blocks, kv_dtype, k_scale, v_scale, workspace,
                         workspace_bytes, stream, nullptr);
+}
+
+pa_status pa_decode_noalloc(void* out, const void* query, const void* key_cache,
+                            const void* value_cache, int num_seqs, int num_heads, int num_kv_heads,
+                            int head_size, float scale, const int32_t* block_tables,
+                            int max_blocks_per_seq, const int32_t* seq_lens, int block_size,
+                            int max_seq_len, int64_t num_blocks, pa_kv_dtype kv_dtype,
+                            const float* k_scale, const float* v_scale, void* stream) {
+    g_detail[0] = 0;
+    pa_status st = check_sizes(num_seqs, num_heads, num_kv_heads, head_size, block_size,
+                               max_seq_len, kv_dtype);
+    if (st != PA_OK) return st;
+    if (num_seqs == 0) return PA_OK;
+    pa_plan pl;
+    st = plan(&pl, num_seqs, num_heads, num_kv_heads, head_size, block_size, max_seq_len, kv_dtype,
+              nullptr);
+    if (st != PA_OK) return st;
+    if (pl.workspace_bytes > kNoallocScratchBytes) {
+        std::snprintf(g_detail, sizeof g_detail,
+                      "this problem needs %zu bytes of scratch; the built-in scratch holds %zu",
+                      pl.workspace_bytes, kNoallocScratchBytes);
+        return PA_ERR_WORKSPACE_TOO_SMALL;
+    }
+    void* scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != PA_OK) return st;
+    return pa_decode_ex(out, query, key_cache, value_cache, num_seqs, num_heads, num_kv_heads,
+                        head_size, scale, block_tables, max_blocks_per_seq, seq_lens, block_size,
+                        max_seq_len, num_blocks, kv_dtype, k_scale, v_scale, scratch,
+                        kNoallocScratchBytes, stream, nullptr);
 }
 
 pa_status pa_read_device_status(void* workspace, uint32_t* flags, int clear, void* stream) {
