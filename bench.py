@@ -54,9 +54,11 @@ def measured_hbm_peak():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the device-code sources (the .cuh kernel headers); host-side
+    ABI code does not change what the kernels read or write."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_471_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(n for n in os.listdir(csrc) if n.endswith(".cuh")):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
