@@ -18,7 +18,10 @@ constexpr size_t kSmemPerSm = 228 * 1024;
 constexpr size_t kSmemReservedPerCta = 1024;
 constexpr size_t kMaxSmemPerCta = 227 * 1024;  // opt-in limit of sm_100
 constexpr int kMinPartitionPages = 16;
+constexpr long long kLongPartitionPages = 256;
 constexpr int kDefaultStages = 2;
+constexpr int kMaxShortStages = 4;
+constexpr size_t kShortStagesSmem = 96 * 1024;  // keep >= 2 CTAs per SM
 constexpr long long kMaxCtasPerSm = 3;
 constexpr int kMaxForcedStages = 16;
 constexpr int kMaxDevices = 64;
@@ -72,9 +75,9 @@ int device_sms(int* out) {
     return 0;
 }
 
-size_t merge_bytes(int head_size, int group) {
+size_t merge_bytes(int head_size, int group, int warps) {
     const int nh = group > 8 ? 2 : 1;
-    return static_cast<size_t>(pa::kWarps * nh * 8 * (head_size + 4) + 2 * pa::kWarps * 16) * 4;
+    return static_cast<size_t>(warps * nh * 8 * (head_size + 4) + 2 * warps * 16) * 4;
 }
 
 pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int head_size,
@@ -94,12 +97,13 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
     // Two page buffers per warp: measured on B200, more resident CTAs beat
     // deeper per-warp rings for the same bytes in flight.
     const size_t stage = 2ull * head_size * block_size * elem_bytes(kv_dtype);
+    const int W = pa::decode_warps(static_cast<long long>(stage));
     int ns = kDefaultStages;
     if (opts && opts->stages > 0) ns = opts->stages;
-    size_t stage_area = static_cast<size_t>(pa::kWarps) * ns * stage;
-    const size_t mb = merge_bytes(head_size, num_heads / num_kv_heads);
+    size_t stage_area = static_cast<size_t>(W) * ns * stage;
+    const size_t mb = merge_bytes(head_size, num_heads / num_kv_heads, W);
     if (stage_area < mb) stage_area = mb;
-    const size_t smem = stage_area + static_cast<size_t>(pa::kWarps) * ns * 8;
+    size_t smem = stage_area + static_cast<size_t>(W) * ns * 8;
     if (smem > kMaxSmemPerCta)
         return fail(PA_ERR_INVALID_ARG, "%s", "too many stages for shared memory");
     long long per_sm = static_cast<long long>(kSmemPerSm / (smem + kSmemReservedPerCta));
@@ -115,39 +119,42 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
     } else if (pages_max == 0 || units == 0) {
         pp = 1;
     } else {
-        // Aim for about four partitions' worth of work per CTA slot if every
-        // sequence were max_seq_len long (bounds the tail of the last wave),
-        // but never fewer than kMinPartitionPages pages per partition.
+        // Split count:
+        //  * enough partitions to balance uneven lengths: about four partitions
+        //    of work per CTA slot if every sequence were max_seq_len long, each
+        //    at least kMinPartitionPages;
+        //  * but no partition shorter than kLongPartitionPages unless that is
+        //    needed to give every CTA slot a partition (long partitions
+        //    amortise each CTA's start-up and merge; measured on B200).
         const long long per_slot = (units * pages_max + slots - 1) / slots;
         long long target = (per_slot + 3) / 4;
         if (target < kMinPartitionPages) target = kMinPartitionPages;
-        if (target >= pages_max) {
-            pp = pages_max;
-        } else {
-            // Among P0..2*P0 partitions pick the one whose last wave of CTAs is
-            // fullest (CTAs of equal length run in whole waves of `slots`).
-            const long long p0 = (pages_max + target - 1) / target;
-            long long best = p0;
-            double best_eff = -1.0;
-            for (long long np = p0; np <= 2 * p0; ++np) {
-                const long long ppc = (pages_max + np - 1) / np;
-                const long long npe = (pages_max + ppc - 1) / ppc;  // partitions really used
-                if (npe != np) continue;
-                const double waves = static_cast<double>(units * np) / static_cast<double>(slots);
-                const double eff = waves / std::ceil(waves) - 0.002 * static_cast<double>(np - p0);
-                if (eff > best_eff + 1e-9) {
-                    best_eff = eff;
-                    best = np;
-                }
-            }
-            pp = (pages_max + best - 1) / best;
-        }
+        const long long p_bal = (pages_max + target - 1) / target;
+        const long long p_fill = (slots + units - 1) / units;
+        const long long p_long = pages_max / kLongPartitionPages > 1 ? pages_max / kLongPartitionPages : 1;
+        long long np = p_bal < (p_fill > p_long ? p_fill : p_long)
+                           ? p_bal
+                           : (p_fill > p_long ? p_fill : p_long);
+        if (np < 1) np = 1;
+        pp = (pages_max + np - 1) / np;
     }
     if (pp < 1) pp = 1;
     long long P = pages_max > 0 ? (pages_max + pp - 1) / pp : 1;
     if (P <= 1) {
         P = 1;
         pp = pages_max > 0 ? pages_max : 1;
+    }
+    // Short partitions: give each warp a buffer for every page it will read
+    // (up to 4), so all copies are in flight after one block-table read.
+    if (!(opts && opts->stages > 0)) {
+        const long long per_warp = (pp + W - 1) / W;
+        const size_t want = static_cast<size_t>(W) * per_warp * (stage + 8);
+        if (per_warp > ns && per_warp <= kMaxShortStages && want <= kShortStagesSmem) {
+            ns = static_cast<int>(per_warp);
+            stage_area = static_cast<size_t>(W) * ns * stage;
+            if (stage_area < mb) stage_area = mb;
+            smem = stage_area + static_cast<size_t>(W) * ns * 8;
+        }
     }
     if (pp > (1ll << 30) || P > (1ll << 30))
         return fail(PA_ERR_INVALID_ARG, "%s", "partition count out of range");
@@ -161,7 +168,7 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
     pl->num_partitions = static_cast<int>(P);
     pl->partition_pages = static_cast<int>(pp);
     pl->stages = ns;
-    pl->warps_per_cta = pa::kWarps;
+    pl->warps_per_cta = W;
     pl->grid_ctas = units * P;
     pl->smem_bytes = smem;
     pl->workspace_bytes = ws;
@@ -188,11 +195,12 @@ template <int D, int B, bool FP8, int NH>
 cudaError_t launch_decode(const pa::DecodeParams& p, long long grid, size_t smem,
                           cudaStream_t st) {
     static std::atomic<int> done[kMaxDevices];
-    auto kern = pa::pa_decode_kernel<D, B, FP8, NH>;
+    constexpr int W = pa::decode_warps<D, B, FP8>();
+    auto kern = pa::pa_decode_kernel<D, B, FP8, NH, W>;
     if (smem > kMaxSmemPerCta) return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem(kern, done);
     if (e != cudaSuccess) return e;
-    kern<<<static_cast<unsigned>(grid), pa::kThreads, smem, st>>>(p);
+    kern<<<static_cast<unsigned>(grid), W * 32, smem, st>>>(p);
     return cudaGetLastError();
 }
 

@@ -68,14 +68,18 @@ struct DecodeParams {
     float scale_log2;  // scale * log2(e)
 };
 
-// Bytes of shared memory the merge step needs (overlaid on the page stages).
-template <int D, int NH>
-constexpr int merge_smem_bytes() {
-    return (kWarps * NH * 8 * (D + 4) + 2 * kWarps * 16) * 4;
+// Consumer warps per decode CTA.  Pages of 16 KiB stages (bf16, head size
+// 128, block size 32) get two warps so that three CTAs still fit on an SM;
+// smaller pages get four.
+constexpr int decode_warps(long long stage_bytes) { return stage_bytes >= 16384 ? 2 : 4; }
+
+template <int D, int B, bool FP8>
+constexpr int decode_warps() {
+    return decode_warps(2LL * D * B * (FP8 ? 1 : 2));
 }
 
-template <int D, int B, bool FP8, int NH>
-__global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodeParams p) {
+template <int D, int B, bool FP8, int NH, int W>
+__global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams p) {
     constexpr int ELEM = FP8 ? 1 : 2;
     constexpr int PAGE = D * B * ELEM;  // one K (or V) page of one kv head
     constexpr int STAGE = 2 * PAGE;
@@ -98,6 +102,51 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
     const int s = static_cast<int>((unit / p.Hk) % p.S);
     const int part = static_cast<int>(unit / ((long long)p.Hk * p.S));
 
+    const int j0 = part * p.PP;
+    const long long row0 = (long long)s * p.Hq + (long long)kvh * p.G;  // first q head row
+
+    // Loads that do not depend on the sequence length go out first, so their
+    // latencies overlap: the block-table window (every entry of the row up to
+    // the partition's end is readable), the raw query words and the scales.
+    // Block-table window: lane l holds the id of this warp's page (wbase + l).
+    const int32_t* btrow = p.bt + (long long)s * p.max_blocks;
+    const int jcap = min(j0 + p.PP, p.max_blocks);
+    auto load_win = [&](int base) -> int {
+        const int j = j0 + warp + W * (base + lane);
+        return j < jcap ? __ldg(btrow + j) : -1;
+    };
+    int win_a = load_win(0);
+    int win_b = load_win(32);
+    // Raw query words of head rows 8r + gq, in the order the fragments use.
+    uint32_t qraw[2][KT][2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int hl = 8 * r + gq;
+        const bool ok = (r < NH) && hl < p.G;
+        const uint16_t* qrow = p.q + (row0 + (ok ? hl : 0)) * D;
+#pragma unroll
+        for (int kt = 0; kt < KT; ++kt) {
+            uint32_t w0 = 0, w1 = 0;
+            if (ok) {
+                if constexpr (!FP8) {
+                    w0 = __ldg(reinterpret_cast<const unsigned int*>(qrow + 16 * kt + 2 * cq));
+                    w1 = __ldg(reinterpret_cast<const unsigned int*>(qrow + 16 * kt + 8 + 2 * cq));
+                } else {
+                    const uint2 w = __ldg(reinterpret_cast<const uint2*>(qrow + 16 * kt + 4 * cq));
+                    w0 = w.x;
+                    w1 = w.y;
+                }
+            }
+            qraw[r][kt][0] = w0;
+            qraw[r][kt][1] = w1;
+        }
+    }
+    float k_scale = 1.f, v_scale = 1.f;
+    if constexpr (FP8) {
+        k_scale = __ldg(p.k_scale);
+        v_scale = __ldg(p.v_scale);
+    }
+
     // ---- sequence length, with the device-side range checks
     int T = __ldg(p.seq_lens + s);
     uint32_t bad = 0;
@@ -109,14 +158,12 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
     if (nb > covered) { nb = covered; T = nb * B; bad = kDevSeqLen; }
     if (bad && part == 0 && kvh == 0 && threadIdx.x == 0) atomicOr(p.status, bad);
 
-    const int j0 = part * p.PP;
     const int j1 = min(nb, j0 + p.PP);
     const bool direct = (p.P == 1) || (nb <= p.PP);
-    const long long row0 = (long long)s * p.Hq + (long long)kvh * p.G;  // first q head row
 
     if (j0 >= j1) {
         if (part == 0) {  // empty sequence: defined as a zero output row
-            for (int i = threadIdx.x; i < p.G * D; i += kThreads)
+            for (int i = threadIdx.x; i < p.G * D; i += (W * 32))
                 p.out[row0 * D + i] = __float2bfloat16_rn(0.f);
         }
         return;
@@ -124,10 +171,10 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
 
     const int NS = p.stages;
     const int span = j1 - j0;
-    const int n_my = span > warp ? (span - warp + kWarps - 1) / kWarps : 0;
+    const int n_my = span > warp ? (span - warp + W - 1) / W : 0;
     const uint32_t sbase = smem_addr(smem);
     const uint32_t wstage0 = sbase + static_cast<uint32_t>(warp * NS * STAGE);
-    const uint32_t bar0 = sbase + static_cast<uint32_t>(kWarps * NS * STAGE + warp * NS * 8);
+    const uint32_t bar0 = sbase + static_cast<uint32_t>(W * NS * STAGE + warp * NS * 8);
 
     if (lane == 0) {
         for (int i = 0; i < NS; ++i) mbar_init(bar0 + 8 * i, 1);
@@ -135,14 +182,6 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
     }
     __syncwarp();
 
-    // Block-table window: lane l holds the id of this warp's page (wbase + l).
-    const int32_t* btrow = p.bt + (long long)s * p.max_blocks + j0 + warp;
-    auto load_win = [&](int base) -> int {
-        const int i = base + lane;
-        return i < n_my ? __ldg(btrow + (long long)kWarps * i) : -1;
-    };
-    int win_a = load_win(0);
-    int win_b = load_win(32);
     int wbase = 0;
     uint32_t valid_mask = 0;  // bit per stage: the page in it had a legal block id
 
@@ -188,45 +227,26 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
     float out_mul = 1.f;
     if constexpr (!FP8) {
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const int hl = 8 * r + gq;
-            const bool ok = (r < NH) && hl < p.G;
-            const uint16_t* qrow = p.q + (row0 + hl) * D;
+        for (int r = 0; r < 2; ++r)
 #pragma unroll
             for (int kt = 0; kt < KT; ++kt) {
-                uint32_t lo = 0, hi = 0;
-                if (ok) {
-                    lo = __ldg(reinterpret_cast<const unsigned int*>(qrow + 16 * kt + 2 * cq));
-                    hi = __ldg(reinterpret_cast<const unsigned int*>(qrow + 16 * kt + 8 + 2 * cq));
-                }
-                qa[kt][r] = lo;
-                qa[kt][r + 2] = hi;
+                qa[kt][r] = qraw[r][kt][0];
+                qa[kt][r + 2] = qraw[r][kt][1];
             }
-        }
     } else {
         // f16 operands: q is scaled by 2^-e so that max|q| < 2^15 (f16 range);
         // 2^e goes back into the logit multiplier.  Within each 16-wide chunk the
         // k order is permuted to match the e4m3 byte order delivered by ldmatrix:
         // k = 2c,2c+1 <-> d = 4c,4c+1 and k = 2c+8,2c+9 <-> d = 4c+2,4c+3.
-        float qf[2][KT][4];
         float amax = 0.f;
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const int hl = 8 * r + gq;
-            const bool ok = (r < NH) && hl < p.G;
-            const uint16_t* qrow = p.q + (row0 + hl) * D;
+        for (int r = 0; r < 2; ++r)
 #pragma unroll
             for (int kt = 0; kt < KT; ++kt) {
-                uint2 w = make_uint2(0u, 0u);
-                if (ok) w = __ldg(reinterpret_cast<const uint2*>(qrow + 16 * kt + 4 * cq));
-                qf[r][kt][0] = bf16_lo(w.x);
-                qf[r][kt][1] = bf16_hi(w.x);
-                qf[r][kt][2] = bf16_lo(w.y);
-                qf[r][kt][3] = bf16_hi(w.y);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(qf[r][kt][e]));
+                const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
+                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(w0)), fabsf(bf16_hi(w0))),
+                                         fmaxf(fabsf(bf16_lo(w1)), fabsf(bf16_hi(w1)))));
             }
-        }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
         int ex = 0;
@@ -238,11 +258,12 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
         for (int r = 0; r < 2; ++r)
 #pragma unroll
             for (int kt = 0; kt < KT; ++kt) {
-                qa[kt][r] = pack_f16x2(qf[r][kt][0] * down, qf[r][kt][1] * down);
-                qa[kt][r + 2] = pack_f16x2(qf[r][kt][2] * down, qf[r][kt][3] * down);
+                const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
+                qa[kt][r] = pack_f16x2(bf16_lo(w0) * down, bf16_hi(w0) * down);
+                qa[kt][r + 2] = pack_f16x2(bf16_lo(w1) * down, bf16_hi(w1) * down);
             }
-        qk_mul = p.scale_log2 * __ldg(p.k_scale) * up;
-        out_mul = __ldg(p.v_scale);
+        qk_mul = p.scale_log2 * k_scale * up;
+        out_mul = v_scale;
     }
 
     float m_run[NH], l_run[NH];
@@ -449,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
             timed_out = true;
             break;
         }
-        const int jg = j0 + warp + kWarps * k;
+        const int jg = j0 + warp + W * k;
         const int valid = ((valid_mask >> stage) & 1u) ? min(B, T - jg * B) : 0;
         const uint32_t kbase = wstage0 + static_cast<uint32_t>(stage * STAGE);
         if (valid == B)
@@ -486,8 +507,8 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
     }
     __syncthreads();  // every warp is done with its stages
     float* s_acc = reinterpret_cast<float*>(smem);
-    float* s_m = s_acc + kWarps * NH * 8 * RS;
-    float* s_l = s_m + kWarps * 16;
+    float* s_m = s_acc + W * NH * 8 * RS;
+    float* s_l = s_m + W * 16;
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
@@ -509,16 +530,16 @@ __global__ void __launch_bounds__(kThreads, 1) pa_decode_kernel(const DecodePara
     }
     __syncthreads();
 
-    for (int idx = threadIdx.x; idx < p.G * D; idx += kThreads) {
+    for (int idx = threadIdx.x; idx < p.G * D; idx += (W * 32)) {
         const int h = idx / D;
         const int d = idx - h * D;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w)
+        for (int w = 0; w < W; ++w)
             if (s_l[w * 16 + h] > 0.f) M = fmaxf(M, s_m[w * 16 + h]);
         float L = 0.f, O = 0.f;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
+        for (int w = 0; w < W; ++w) {
             const float l = s_l[w * 16 + h];
             if (l > 0.f) {
                 const float wt = exp2f(s_m[w * 16 + h] - M);

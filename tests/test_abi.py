@@ -135,3 +135,16 @@ def test_forced_partitions():
 def test_two_ctas_per_sm_fit_for_the_bf16_b16_pages():
     p = _plan(2)
     assert 2 * (p["smem_bytes"] + 1024) <= 228 * 1024
+
+
+def test_every_plan_fits_shared_memory():
+    # Every supported shape and forced split stays inside the 227 KiB opt-in
+    # limit of one CTA (a plan above it would fail to launch).
+    for D in (64, 128):
+        for B in (16, 32):
+            for kv in ("bf16", "fp8_e4m3"):
+                for G in (1, 4, 8, 16):
+                    for T in (1, 15, 17, 100, 1000, 20000, 131072):
+                        for pp in (0, 1, 2, 3, 5, 16, 64):
+                            p = pa.plan(4, 2 * G, 2, D, B, T, kv, partition_pages=pp, num_sms=148)
+                            assert p["smem_bytes"] <= 227 * 1024, (D, B, kv, G, T, pp)
