@@ -73,6 +73,7 @@ typedef enum pa_kv_dtype {
 #define PA_DEV_SEQ_LEN_OUT_OF_RANGE 0x2u/* seq_len < 0, > max_blocks*block_size, or beyond
                                            max_seq_len's partitions: length clamped           */
 #define PA_DEV_WAIT_TIMEOUT 0x4u        /* a page copy did not land within ~2 s: output void  */
+#define PA_DEV_PREFIX_MISMATCH 0x8u     /* a declared shared prefix does not hold             */
 
 /* Bytes at the start of the workspace reserved for the status word. */
 #define PA_WORKSPACE_HEADER_BYTES 256
@@ -86,11 +87,23 @@ typedef enum pa_kv_dtype {
  *      (lets the host plan without a GPU, e.g. to size a workspace).
  *  stages: 0 lets the planner choose; 2..16 forces that many page buffers
  *      per warp (shared memory grows with it; more than fits is rejected).
+ *  shared_prefix_blocks: k > 0 declares that the first k logical blocks are
+ *      the same physical blocks in every row of block_tables and that every
+ *      seq_len is at least k * block_size -- the prompt sharing of
+ *      "vLLM 0.25.0 release-notes commentary", section 1 (several outputs
+ *      share one prompt's KV).  The prefix pages are then streamed once per
+ *      group of 16 query rows (all sequences' heads of a kv head packed
+ *      together) instead of once per sequence, and merged with each
+ *      sequence's own pages by the combine kernel ("cascade" decode).
+ *      Kernels verify the declaration and set PA_DEV_PREFIX_MISMATCH when a
+ *      row's prefix differs from row 0's or a sequence is shorter than the
+ *      prefix (results for that sequence are then undefined).  0 = off.
  */
 typedef struct pa_options {
     int partition_pages;
     int num_sms;
     int stages;
+    int shared_prefix_blocks;
 } pa_options;
 
 /* What pa_decode will launch for a given problem. */
@@ -99,9 +112,11 @@ typedef struct pa_plan {
     int partition_pages;    /* blocks per partition                                    */
     int stages;             /* page buffers per warp in shared memory                  */
     int warps_per_cta;      /* consumer warps per CTA                                   */
-    long long grid_ctas;    /* CTAs of the decode kernel: num_seqs*num_kv_heads*P       */
+    long long grid_ctas;    /* CTAs of the decode kernel                                */
     size_t smem_bytes;      /* dynamic shared memory per CTA                            */
     size_t workspace_bytes; /* bytes pa_decode needs in `workspace`                     */
+    int prefix_partitions;  /* partitions of a declared shared prefix (0 = none)        */
+    int prefix_groups;      /* 16-query-row groups per kv head streaming the prefix     */
 } pa_plan;
 
 /*

@@ -31,6 +31,7 @@ PA_KV_FP8_E4M3 = 1
 PA_DEV_BAD_BLOCK_ID = 0x1
 PA_DEV_SEQ_LEN_OUT_OF_RANGE = 0x2
 PA_DEV_WAIT_TIMEOUT = 0x4
+PA_DEV_PREFIX_MISMATCH = 0x8
 
 WORKSPACE_HEADER_BYTES = 256
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -47,14 +48,15 @@ class PagedAttentionError(RuntimeError):
 
 class Options(ctypes.Structure):
     _fields_ = [("partition_pages", ctypes.c_int), ("num_sms", ctypes.c_int),
-                ("stages", ctypes.c_int)]
+                ("stages", ctypes.c_int), ("shared_prefix_blocks", ctypes.c_int)]
 
 
 class Plan(ctypes.Structure):
     _fields_ = [("num_partitions", ctypes.c_int), ("partition_pages", ctypes.c_int),
                 ("stages", ctypes.c_int), ("warps_per_cta", ctypes.c_int),
                 ("grid_ctas", ctypes.c_longlong), ("smem_bytes", ctypes.c_size_t),
-                ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace_bytes", ctypes.c_size_t), ("prefix_partitions", ctypes.c_int),
+                ("prefix_groups", ctypes.c_int)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}
@@ -113,10 +115,11 @@ def _check(rc: int):
                                       f"{L.pa_last_error_detail().decode()}")
 
 
-def _opts(partition_pages=0, num_sms=0, stages=0):
-    if not partition_pages and not num_sms and not stages:
+def _opts(partition_pages=0, num_sms=0, stages=0, shared_prefix_blocks=0):
+    if not partition_pages and not num_sms and not stages and not shared_prefix_blocks:
         return None
-    return ctypes.byref(Options(int(partition_pages), int(num_sms), int(stages)))
+    return ctypes.byref(Options(int(partition_pages), int(num_sms), int(stages),
+                                int(shared_prefix_blocks)))
 
 
 def kv_dtype_code(kv_dtype) -> int:
@@ -127,19 +130,19 @@ def kv_dtype_code(kv_dtype) -> int:
 
 
 def plan(num_seqs, num_heads, num_kv_heads, head_size, block_size, max_seq_len, kv_dtype="bf16",
-         partition_pages=0, num_sms=0, stages=0) -> dict:
+         partition_pages=0, num_sms=0, stages=0, shared_prefix_blocks=0) -> dict:
     p = Plan()
     _check(lib().pa_plan_decode(ctypes.byref(p), num_seqs, num_heads, num_kv_heads, head_size,
                                 block_size, max_seq_len, kv_dtype_code(kv_dtype),
-                                _opts(partition_pages, num_sms, stages)))
+                                _opts(partition_pages, num_sms, stages, shared_prefix_blocks)))
     return p.as_dict()
 
 
 def workspace_size(num_seqs, num_heads, num_kv_heads, head_size, block_size, max_seq_len,
-                   kv_dtype="bf16", partition_pages=0, num_sms=0) -> int:
+                   kv_dtype="bf16", partition_pages=0, num_sms=0, shared_prefix_blocks=0) -> int:
     n = lib().pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_size, block_size,
                                        max_seq_len, kv_dtype_code(kv_dtype),
-                                       _opts(partition_pages, num_sms))
+                                       _opts(partition_pages, num_sms, 0, shared_prefix_blocks))
     if n == 0:
         raise PagedAttentionError(PA_ERR_INVALID_ARG, lib().pa_last_error_detail().decode())
     return n
@@ -179,7 +182,7 @@ def _ptr(t, name, dtypes=None, device=None):
 def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, block_tables,
            seq_lens, block_size: int, max_seq_len: int, kv_dtype="bf16", k_scale=None,
            v_scale=None, workspace_tensor=None, partition_pages: int = 0, stream=None,
-           stages: int = 0):
+           stages: int = 0, shared_prefix_blocks: int = 0):
     """Paged decode attention into ``out`` (bf16 [num_seqs, num_heads, head_size]).
 
     key_cache: [num_blocks, num_kv_heads, head_size/x, block_size, x];
@@ -216,7 +219,8 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
     if code == PA_KV_FP8_E4M3:
         ks = _ptr(k_scale, "k_scale", (torch.float32,), dev)
         vs = _ptr(v_scale, "v_scale", (torch.float32,), dev)
-    need = workspace_size(S, Hq, num_kv_heads, D, block_size, max_seq_len, code, partition_pages)
+    need = workspace_size(S, Hq, num_kv_heads, D, block_size, max_seq_len, code, partition_pages,
+                          shared_prefix_blocks=shared_prefix_blocks)
     if workspace_tensor is None:
         workspace_tensor = workspace(need, dev)
     ws = _ptr(workspace_tensor, "workspace", None, dev)
@@ -225,7 +229,8 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
                             block_tables.shape[1], sl, int(block_size), int(max_seq_len),
                             int(num_blocks), code, ks, vs, ws,
                             workspace_tensor.numel() * workspace_tensor.element_size(),
-                            st.cuda_stream, _opts(partition_pages, 0, stages))
+                            st.cuda_stream,
+                            _opts(partition_pages, 0, stages, shared_prefix_blocks))
     _check(rc)
     return out
 

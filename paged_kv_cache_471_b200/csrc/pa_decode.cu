@@ -96,12 +96,17 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         return fail(PA_ERR_INVALID_ARG, "%s", "opts->stages must be 0 or 2..16");
     // Two page buffers per warp: measured on B200, more resident CTAs beat
     // deeper per-warp rings for the same bytes in flight.
+    const int prefix = opts ? opts->shared_prefix_blocks : 0;
+    if (prefix < 0 || static_cast<long long>(prefix) * block_size > max_seq_len)
+        return fail(PA_ERR_INVALID_ARG, "%s",
+                    "opts->shared_prefix_blocks must be in [0, max_seq_len / block_size]");
+    const bool cascade = prefix > 0 && num_seqs > 0;
     const size_t stage = 2ull * head_size * block_size * elem_bytes(kv_dtype);
     const int W = pa::decode_warps(static_cast<long long>(stage));
     int ns = kDefaultStages;
     if (opts && opts->stages > 0) ns = opts->stages;
     size_t stage_area = static_cast<size_t>(W) * ns * stage;
-    const size_t mb = merge_bytes(head_size, num_heads / num_kv_heads, W);
+    const size_t mb = merge_bytes(head_size, cascade ? 16 : num_heads / num_kv_heads, W);
     if (stage_area < mb) stage_area = mb;
     size_t smem = stage_area + static_cast<size_t>(W) * ns * 8;
     if (smem > kMaxSmemPerCta)
@@ -144,6 +149,14 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         P = 1;
         pp = pages_max > 0 ? pages_max : 1;
     }
+    // Shared prefix: its pages are split like the rest; each sequence's own
+    // pages (after the prefix) get their own partitions.
+    long long p_pre = 0, groups = 0;
+    if (cascade) {
+        p_pre = (prefix + pp - 1) / pp;
+        P = (pages_max - prefix + pp - 1) / pp;
+        groups = (static_cast<long long>(num_seqs) * (num_heads / num_kv_heads) + 15) / 16;
+    }
     // Short partitions: give each warp a buffer for every page it will read
     // (up to 4), so all copies are in flight after one block-table read.
     if (!(opts && opts->stages > 0)) {
@@ -160,18 +173,20 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         return fail(PA_ERR_INVALID_ARG, "%s", "partition count out of range");
 
     size_t ws = PA_WORKSPACE_HEADER_BYTES;
-    if (P > 1) {
-        ws += static_cast<size_t>(num_seqs) * num_heads * P * (static_cast<size_t>(head_size) + 2) *
-              sizeof(float);
+    if (P > 1 || cascade) {
+        ws += static_cast<size_t>(num_seqs) * num_heads * (P + p_pre) *
+              (static_cast<size_t>(head_size) + 2) * sizeof(float);
         ws = (ws + 255) & ~static_cast<size_t>(255);
     }
     pl->num_partitions = static_cast<int>(P);
     pl->partition_pages = static_cast<int>(pp);
     pl->stages = ns;
     pl->warps_per_cta = W;
-    pl->grid_ctas = units * P;
+    pl->grid_ctas = units * P + num_kv_heads * groups * p_pre;
     pl->smem_bytes = smem;
     pl->workspace_bytes = ws;
+    pl->prefix_partitions = static_cast<int>(p_pre);
+    pl->prefix_groups = static_cast<int>(groups);
     return PA_OK;
 }
 
@@ -206,8 +221,9 @@ cudaError_t launch_decode(const pa::DecodeParams& p, long long grid, size_t smem
 
 template <int D, int B, bool FP8>
 cudaError_t launch_nh(const pa::DecodeParams& p, long long grid, size_t smem, cudaStream_t st) {
-    return p.G > 8 ? launch_decode<D, B, FP8, 2>(p, grid, smem, st)
-                   : launch_decode<D, B, FP8, 1>(p, grid, smem, st);
+    // Shared-prefix units pack 16 query rows, so they need the 16-row form.
+    return (p.G > 8 || p.prefix_pages > 0) ? launch_decode<D, B, FP8, 2>(p, grid, smem, st)
+                                           : launch_decode<D, B, FP8, 1>(p, grid, smem, st);
 }
 
 template <int D, int B>
@@ -346,7 +362,8 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
     p.v_scale = v_scale;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     p.status = reinterpret_cast<uint32_t*>(ws);
-    const size_t rows = static_cast<size_t>(num_seqs) * num_heads * pl.num_partitions;
+    const int p_total = pl.num_partitions + pl.prefix_partitions;
+    const size_t rows = static_cast<size_t>(num_seqs) * num_heads * p_total;
     float* part = reinterpret_cast<float*>(ws + PA_WORKSPACE_HEADER_BYTES);
     p.ws_o = part;
     p.ws_m = part + rows * head_size;
@@ -361,12 +378,17 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
     p.stages = pl.stages;
     p.num_blocks = num_blocks;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.prefix_pages = pl.prefix_partitions > 0 ? opts->shared_prefix_blocks : 0;
+    p.prefix_parts = pl.prefix_partitions;
+    p.prefix_groups = pl.prefix_groups;
+    p.prefix_units = static_cast<long long>(num_kv_heads) * pl.prefix_groups * pl.prefix_partitions;
+    p.P_total = p_total;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = launch_any(p, head_size, block_size, kv_dtype == PA_KV_FP8_E4M3, pl.grid_ctas,
                                pl.smem_bytes, s);
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
-    if (pl.num_partitions > 1) {
+    if (pl.num_partitions > 1 || p.prefix_pages > 0) {
         pa::CombineParams c;
         c.out = p.out;
         c.ws_o = p.ws_o;
@@ -379,6 +401,9 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
         c.PP = pl.partition_pages;
         c.max_blocks = max_blocks_per_seq;
         c.B = block_size;
+        c.prefix_pages = p.prefix_pages;
+        c.prefix_parts = p.prefix_parts;
+        c.P_total = p.P_total;
         e = launch_combine(c, head_size, s);
         if (e != cudaSuccess) return fail(PA_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
     }

@@ -45,6 +45,7 @@ constexpr uint32_t kFull = 0xffffffffu;
 constexpr uint32_t kDevBadBlock = 0x1u;
 constexpr uint32_t kDevSeqLen = 0x2u;
 constexpr uint32_t kDevTimeout = 0x4u;
+constexpr uint32_t kDevPrefix = 0x8u;
 
 struct DecodeParams {
     __nv_bfloat16* out;       // [S, Hq, D]
@@ -61,12 +62,27 @@ struct DecodeParams {
     uint32_t* status;         // sticky status word
     int S, Hq, Hk, G;
     int max_blocks;
-    int P;   // partitions per (seq, kv head)
+    int P;   // partitions per (seq, kv head) over its own pages
     int PP;  // pages per partition
     int stages;
     long long num_blocks;
     float scale_log2;  // scale * log2(e)
+    // Shared-prefix (cascade) decode: the first prefix_pages logical blocks are
+    // the same physical blocks in every row of the block table.  They are
+    // streamed once per group of 16 query rows (all sequences' heads of one kv
+    // head) by the first prefix_units CTAs; per-sequence CTAs start after them.
+    int prefix_pages;         // 0: no shared prefix
+    int prefix_parts;         // partitions of the prefix
+    int prefix_groups;        // 16-row groups of the S*G query rows of a kv head
+    long long prefix_units;   // Hk * prefix_groups * prefix_parts
+    int P_total;              // partial slots per (seq, q head): prefix_parts + P
 };
+
+// Bytes of shared memory the final merge needs (it overlays the page stages).
+template <int D, int NH, int W>
+constexpr int merge_smem_bytes() {
+    return (W * NH * 8 * (D + 4) + 2 * W * 16) * 4;
+}
 
 // Consumer warps per decode CTA.  Pages of 16 KiB stages (bf16, head size
 // 128, block size 32) get two warps so that three CTAs still fit on an SM;
@@ -98,32 +114,54 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
     const int cq = lane & 3;   // thread in quad
 
     const long long unit = blockIdx.x;
-    const int kvh = static_cast<int>(unit % p.Hk);
-    const int s = static_cast<int>((unit / p.Hk) % p.S);
-    const int part = static_cast<int>(unit / ((long long)p.Hk * p.S));
-
-    const int j0 = part * p.PP;
+    const bool pre = unit < p.prefix_units;  // a shared-prefix unit
+    int kvh, s, part, rg = 0;
+    if (pre) {
+        kvh = static_cast<int>(unit % p.Hk);
+        rg = static_cast<int>((unit / p.Hk) % p.prefix_groups);
+        part = static_cast<int>(unit / ((long long)p.Hk * p.prefix_groups));
+        s = 0;
+    } else {
+        const long long u = unit - p.prefix_units;
+        kvh = static_cast<int>(u % p.Hk);
+        s = static_cast<int>((u / p.Hk) % p.S);
+        part = static_cast<int>(u / ((long long)p.Hk * p.S));
+    }
+    const bool cascade = p.prefix_pages > 0;
+    const int pg0 = pre ? 0 : p.prefix_pages;  // first page of this unit's page range
+    const int j0 = pg0 + part * p.PP;
     const long long row0 = (long long)s * p.Hq + (long long)kvh * p.G;  // first q head row
+    const int rows_total = p.S * p.G;  // query rows of one kv head (prefix units)
+
+    // Query row (s*Hq + head) of local row lr = 8r + gq, or -1 when unused.
+    auto row_of = [&](int lr) -> long long {
+        if (pre) {
+            const int gi = rg * 16 + lr;
+            if (gi >= rows_total) return -1;
+            return (long long)(gi / p.G) * p.Hq + (long long)kvh * p.G + gi % p.G;
+        }
+        return lr < p.G ? row0 + lr : -1;
+    };
 
     // Loads that do not depend on the sequence length go out first, so their
     // latencies overlap: the block-table window (every entry of the row up to
     // the partition's end is readable), the raw query words and the scales.
     // Block-table window: lane l holds the id of this warp's page (wbase + l).
     const int32_t* btrow = p.bt + (long long)s * p.max_blocks;
-    const int jcap = min(j0 + p.PP, p.max_blocks);
+    const int jcap = min(j0 + p.PP, pre ? p.prefix_pages : p.max_blocks);
     auto load_win = [&](int base) -> int {
         const int j = j0 + warp + W * (base + lane);
         return j < jcap ? __ldg(btrow + j) : -1;
     };
     int win_a = load_win(0);
     int win_b = load_win(32);
-    // Raw query words of head rows 8r + gq, in the order the fragments use.
+    // Raw query words of rows 8r + gq, in the order the fragments use.
     uint32_t qraw[2][KT][2];
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-        const int hl = 8 * r + gq;
-        const bool ok = (r < NH) && hl < p.G;
-        const uint16_t* qrow = p.q + (row0 + (ok ? hl : 0)) * D;
+        const long long qr = (r < NH) ? row_of(8 * r + gq) : -1;
+        const bool ok = qr >= 0;
+        const uint16_t* qrow = p.q + (ok ? qr : 0) * D;
 #pragma unroll
         for (int kt = 0; kt < KT; ++kt) {
             uint32_t w0 = 0, w1 = 0;
@@ -148,21 +186,35 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
     }
 
     // ---- sequence length, with the device-side range checks
-    int T = __ldg(p.seq_lens + s);
-    uint32_t bad = 0;
-    const int t_cap = p.max_blocks * B;
-    if (T < 0) { T = 0; bad = kDevSeqLen; }
-    if (T > t_cap) { T = t_cap; bad = kDevSeqLen; }
-    int nb = (T + B - 1) / B;
-    const int covered = p.P * p.PP;
-    if (nb > covered) { nb = covered; T = nb * B; bad = kDevSeqLen; }
-    if (bad && part == 0 && kvh == 0 && threadIdx.x == 0) atomicOr(p.status, bad);
+    int T, nb;
+    if (pre) {
+        nb = p.prefix_pages;  // every prefix page is full
+        T = nb * B;
+    } else {
+        T = __ldg(p.seq_lens + s);
+        uint32_t bad = 0;
+        const int t_cap = p.max_blocks * B;
+        if (T < 0) { T = 0; bad = kDevSeqLen; }
+        if (T > t_cap) { T = t_cap; bad = kDevSeqLen; }
+        nb = (T + B - 1) / B;
+        const int covered = pg0 + p.P * p.PP;
+        if (nb > covered) { nb = covered; T = nb * B; bad = kDevSeqLen; }
+        if (cascade && T < p.prefix_pages * B) bad |= kDevPrefix;
+        if (bad && part == 0 && kvh == 0 && threadIdx.x == 0) atomicOr(p.status, bad);
+        if (cascade && part == 0 && kvh == 0 && warp == 0 && s > 0) {
+            // The declared prefix must be the same physical blocks as row 0's.
+            bool same = true;
+            for (int j = lane; j < p.prefix_pages; j += 32)
+                same &= __ldg(btrow + j) == __ldg(p.bt + j);
+            if (!__all_sync(kFull, same) && lane == 0) atomicOr(p.status, kDevPrefix);
+        }
+    }
 
     const int j1 = min(nb, j0 + p.PP);
-    const bool direct = (p.P == 1) || (nb <= p.PP);
+    const bool direct = !cascade && ((p.P == 1) || (nb <= p.PP));
 
     if (j0 >= j1) {
-        if (part == 0) {  // empty sequence: defined as a zero output row
+        if (!cascade && part == 0) {  // empty sequence: defined as a zero output row
             for (int i = threadIdx.x; i < p.G * D; i += (W * 32))
                 p.out[row0 * D + i] = __float2bfloat16_rn(0.f);
         }
@@ -174,7 +226,10 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
     const int n_my = span > warp ? (span - warp + W - 1) / W : 0;
     const uint32_t sbase = smem_addr(smem);
     const uint32_t wstage0 = sbase + static_cast<uint32_t>(warp * NS * STAGE);
-    const uint32_t bar0 = sbase + static_cast<uint32_t>(W * NS * STAGE + warp * NS * 8);
+    // mbarriers sit after the larger of the page stages and the merge buffer
+    // that later overlays them (the host sizes shared memory the same way).
+    const int stage_area = max(W * NS * STAGE, merge_smem_bytes<D, NH, W>());
+    const uint32_t bar0 = sbase + static_cast<uint32_t>(stage_area + warp * NS * 8);
 
     if (lane == 0) {
         for (int i = 0; i < NS; ++i) mbar_init(bar0 + 8 * i, 1);
@@ -530,7 +585,9 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
     }
     __syncthreads();
 
-    for (int idx = threadIdx.x; idx < p.G * D; idx += (W * 32)) {
+    const int rows_here = pre ? min(16, rows_total - rg * 16) : p.G;
+    const int slot = pre ? part : (cascade ? p.prefix_parts : 0) + part;
+    for (int idx = threadIdx.x; idx < rows_here * D; idx += (W * 32)) {
         const int h = idx / D;
         const int d = idx - h * D;
         float M = -INFINITY;
@@ -548,11 +605,11 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
             }
         }
         const float o = L > 0.f ? (O / L) * out_mul : 0.f;
-        const long long row = row0 + h;
+        const long long row = row_of(h);
         if (direct) {
             p.out[row * D + d] = __float2bfloat16_rn(o);
         } else {
-            const long long prow = row * p.P + part;
+            const long long prow = row * p.P_total + slot;
             p.ws_o[prow * D + d] = o;
             if (d == 0) {
                 p.ws_m[prow] = M;
@@ -569,12 +626,15 @@ struct CombineParams {
     const float* ws_l;
     const int32_t* seq_lens;
     int S, Hq, P, PP, max_blocks, B;
+    int prefix_pages, prefix_parts, P_total;
 };
 
 // Log-sum-exp merge of the split-KV partials of one (sequence, q head) per
 // warp:  M = max_p m_p;  w_p = l_p 2^(m_p - M);  out = sum_p w_p o_p / sum_p w_p.
-// Rows whose sequence fits in one partition were written by the decode kernel
-// and are skipped here, as are partitions with an empty sum.
+// Without a shared prefix, rows whose sequence fits in one partition were
+// written by the decode kernel and are skipped here.  With one, the slots are
+// the prefix partitions followed by the sequence's own partitions.
+// Partitions with an empty sum are skipped.
 template <int D>
 __global__ void __launch_bounds__(kThreads) pa_combine_kernel(const CombineParams p) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -583,10 +643,16 @@ __global__ void __launch_bounds__(kThreads) pa_combine_kernel(const CombineParam
     const int s = static_cast<int>(row / p.Hq);
     int T = __ldg(p.seq_lens + s);
     T = max(0, min(T, p.max_blocks * p.B));
-    int nb = (T + p.B - 1) / p.B;
-    const int nps = min(p.P, (nb + p.PP - 1) / p.PP);
-    if (nps <= 1) return;
-    const long long base = row * p.P;
+    const int nb = (T + p.B - 1) / p.B;
+    int nps;
+    if (p.prefix_pages > 0) {
+        const int own = nb > p.prefix_pages ? (nb - p.prefix_pages + p.PP - 1) / p.PP : 0;
+        nps = p.prefix_parts + min(p.P, own);
+    } else {
+        nps = min(p.P, (nb + p.PP - 1) / p.PP);
+        if (nps <= 1) return;
+    }
+    const long long base = row * p.P_total;
     float M = -INFINITY;
     for (int i = lane; i < nps; i += 32)
         if (p.ws_l[base + i] > 0.f) M = fmaxf(M, p.ws_m[base + i]);

@@ -163,3 +163,54 @@ def test_bad_block_id_and_length_flags():
     assert torch.isfinite(out[0].float()).all()
     assert torch.equal(out[0], good[0])
     assert pa.read_status(ws) == 0
+
+
+@pytest.mark.parametrize("kv", [W.BF16, W.FP8_E4M3])
+@pytest.mark.parametrize("B", [16, 32])
+def test_one_hot_probe_bit_exact_with_shared_prefix(kv, B):
+    """Cascade decode: the probe token sits in the shared prefix (a shared
+    block, so every sequence sees it) or in a sequence's own pages."""
+    pref = 5
+    lens = [pref * B + 3, pref * B, 9 * B + 1]
+    cfg = W.PagedConfig(f"probe prefix B={B} {kv}", num_seqs=3, num_heads=8, num_kv_heads=2,
+                        head_size=128, block_size=B,
+                        num_blocks=pref + sum(-(-t // B) - pref for t in lens) + 6,
+                        seq_len_lo=1, seq_len_hi=max(lens), kv_dtype=kv,
+                        k_scale=0.05 if kv == W.FP8_E4M3 else 1.0,
+                        v_scale=0.05 if kv == W.FP8_E4M3 else 1.0, shared_prefix_blocks=pref,
+                        seed=91)
+    wl = W.make_workload(cfg, DEV, seq_lens=lens)
+    kc = wl.key_cache
+    for s, T in enumerate(lens):
+        for t in range(T):
+            pb, o = _token_slot(wl, s, t)
+            kc[pb, :, 0, o, 0] = 0
+    q = torch.zeros_like(wl.query)
+    q[:, :, 0] = 4096.0
+    wl.query = q
+    one = 1.0 if kv == W.BF16 else 0x7E
+    ws = torch.zeros(pa.workspace_size(3, 8, 2, 128, B, max(lens), kv, 2,
+                                       shared_prefix_blocks=pref), dtype=torch.uint8, device=DEV)
+    out = torch.empty_like(wl.query)
+    for t_star, seqs in [(0, [0, 1, 2]), (pref * B - 1, [0, 1, 2]), (2 * B + 3, [0, 1, 2]),
+                         (pref * B + 2, [0]), (9 * B, [2])]:
+        marks = []
+        for s in seqs:
+            pb, o = _token_slot(wl, s, t_star)
+            marks.append((pb, o, kc[pb, :, 0, o, 0].clone()))
+            kc[pb, :, 0, o, 0] = one if kv == W.BF16 else torch.full_like(marks[-1][2], one)
+        pa.decode(out, wl.query, kc, wl.value_cache, 2, cfg.scale, wl.block_tables, wl.seq_lens,
+                  B, max(lens), kv, wl.k_scale, wl.v_scale, workspace_tensor=ws,
+                  partition_pages=2, shared_prefix_blocks=pref)
+        torch.cuda.synchronize()
+        assert pa.read_status(ws) == 0
+        for s in seqs:
+            pb, o = _token_slot(wl, s, t_star)
+            for h in range(8):
+                v = wl.value_cache[pb, h // 4, :, o]
+                want = v if kv == W.BF16 else \
+                    (v.view(torch.float8_e4m3fn).float() * cfg.v_scale).to(torch.bfloat16)
+                assert torch.equal(out[s, h].view(torch.int16), want.view(torch.int16)), \
+                    (s, t_star, h)
+        for pb, o, old in reversed(marks):  # shared slots appear once per sequence
+            kc[pb, :, 0, o, 0] = old

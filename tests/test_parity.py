@@ -81,3 +81,82 @@ def test_full_size_sampled(idx):
     assert pa.read_status(device=DEV) == 0
     del wl, out
     torch.cuda.empty_cache()
+
+
+# ----------------------------------------------------------------- shared prefix
+PREFIX_CASES = {
+    "b32_bf16_g4": W.reduced(5, num_seqs=3, seq_len_hi=5000, seq_len_lo=4100,
+                             shared_prefix_blocks=40),
+    "b16_bf16_g8": W.reduced(3, num_seqs=5, seq_len_hi=3000, seq_len_lo=1000).replace(
+        shared_prefix_blocks=50, num_blocks=50 + 5 * 188 + 16),
+    "b16_fp8_g4": W.reduced(4, num_seqs=6, seq_len_hi=2500, seq_len_lo=800).replace(
+        shared_prefix_blocks=33, num_blocks=33 + 6 * 157 + 16),
+    "b16_bf16_g16": W.PagedConfig("prefix G=16", num_seqs=3, num_heads=32, num_kv_heads=2,
+                                  head_size=64, block_size=16, num_blocks=20 + 3 * 40 + 8,
+                                  seq_len_lo=400, seq_len_hi=640, shared_prefix_blocks=20,
+                                  seed=31),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PREFIX_CASES))
+@pytest.mark.parametrize("partition_pages", [0, 7])
+def test_shared_prefix_cascade(name, partition_pages):
+    cfg = PREFIX_CASES[name]
+    wl = W.make_workload(cfg, DEV)
+    ws = torch.zeros(pa.workspace_size(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads,
+                                       cfg.head_size, cfg.block_size, cfg.max_seq_len,
+                                       cfg.kv_dtype, partition_pages,
+                                       shared_prefix_blocks=cfg.shared_prefix_blocks),
+                     dtype=torch.uint8, device=DEV)
+    out = torch.empty_like(wl.query)
+    pa.decode(out, wl.query, wl.key_cache, wl.value_cache, cfg.num_kv_heads, cfg.scale,
+              wl.block_tables, wl.seq_lens, cfg.block_size, cfg.max_seq_len, cfg.kv_dtype,
+              wl.k_scale, wl.v_scale, workspace_tensor=ws, partition_pages=partition_pages,
+              shared_prefix_blocks=cfg.shared_prefix_blocks)
+    torch.cuda.synchronize()
+    assert pa.read_status(ws) == 0
+    compare(out, run_oracle(wl), cfg.kv_dtype, f"prefix {name} pp={partition_pages}")
+
+
+def test_shared_prefix_full_size_sampled():
+    cfg = W.CONFIGS[5]
+    wl = W.make_workload(cfg, DEV)
+    ws = torch.zeros(pa.workspace_size(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads,
+                                       cfg.head_size, cfg.block_size, cfg.max_seq_len,
+                                       shared_prefix_blocks=cfg.shared_prefix_blocks),
+                     dtype=torch.uint8, device=DEV)
+    out = torch.empty_like(wl.query)
+    pa.decode(out, wl.query, wl.key_cache, wl.value_cache, cfg.num_kv_heads, cfg.scale,
+              wl.block_tables, wl.seq_lens, cfg.block_size, cfg.max_seq_len, cfg.kv_dtype,
+              workspace_tensor=ws, shared_prefix_blocks=cfg.shared_prefix_blocks)
+    torch.cuda.synchronize()
+    assert pa.read_status(ws) == 0
+    pairs = sample_pairs(cfg, 10, seed=55)
+    ref = run_oracle_sampled(wl, pairs)
+    compare(torch.stack([out[s, h] for s, h in pairs]), ref, cfg.kv_dtype, "full cfg5 cascade")
+    del wl, out
+    torch.cuda.empty_cache()
+
+
+def test_shared_prefix_mismatch_is_flagged():
+    cfg = PREFIX_CASES["b16_bf16_g8"]
+    wl = W.make_workload(cfg, DEV)
+    ws = torch.zeros(pa.workspace_size(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads,
+                                       cfg.head_size, cfg.block_size, cfg.max_seq_len,
+                                       shared_prefix_blocks=cfg.shared_prefix_blocks),
+                     dtype=torch.uint8, device=DEV)
+    out = torch.empty_like(wl.query)
+    bt = wl.block_tables
+    bt[2, 7] = bt[2, cfg.shared_prefix_blocks]  # row 2's prefix now differs from row 0's
+    pa.decode(out, wl.query, wl.key_cache, wl.value_cache, cfg.num_kv_heads, cfg.scale, bt,
+              wl.seq_lens, cfg.block_size, cfg.max_seq_len, workspace_tensor=ws,
+              shared_prefix_blocks=cfg.shared_prefix_blocks)
+    torch.cuda.synchronize()
+    assert pa.read_status(ws, clear=True) & pa.PA_DEV_PREFIX_MISMATCH
+    wl.seq_lens[1] = cfg.shared_prefix_blocks * cfg.block_size - 3  # shorter than the prefix
+    bt[2, 7] = bt[0, 7]
+    pa.decode(out, wl.query, wl.key_cache, wl.value_cache, cfg.num_kv_heads, cfg.scale, bt,
+              wl.seq_lens, cfg.block_size, cfg.max_seq_len, workspace_tensor=ws,
+              shared_prefix_blocks=cfg.shared_prefix_blocks)
+    torch.cuda.synchronize()
+    assert pa.read_status(ws) & pa.PA_DEV_PREFIX_MISMATCH
