@@ -198,7 +198,8 @@ def workload_config(idx: int, num_seqs: int = 0):
     return W.CONFIGS[idx]
 
 
-def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, num_seqs=0):
+def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, num_seqs=0,
+             cascade=True):
     import torch
 
     import paged_kv_cache_471_b200 as pa
@@ -207,8 +208,11 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
     cfg = workload_config(idx, num_seqs)
     wl = W.make_workload(cfg, device)
     out = torch.empty_like(wl.query)
+    # A workload whose sequences share a prompt prefix declares it, so the
+    # prefix pages are streamed once per group of query rows (cascade decode).
+    prefix = cfg.shared_prefix_blocks if cascade else 0
     plan = pa.plan(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_size, cfg.block_size,
-                   cfg.max_seq_len, cfg.kv_dtype)
+                   cfg.max_seq_len, cfg.kv_dtype, shared_prefix_blocks=prefix)
     ws = torch.zeros(plan["workspace_bytes"], dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
     alg_bytes = bytes_of(wl)
@@ -219,7 +223,8 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
     def step():
         pa.decode(out, wl.query, wl.key_cache, wl.value_cache, cfg.num_kv_heads, cfg.scale,
                   wl.block_tables, wl.seq_lens, cfg.block_size, cfg.max_seq_len, cfg.kv_dtype,
-                  wl.k_scale, wl.v_scale, workspace_tensor=ws, stream=stream)
+                  wl.k_scale, wl.v_scale, workspace_tensor=ws, stream=stream,
+                  shared_prefix_blocks=prefix)
 
     for _ in range(max(warmup, 3)):
         if flush:
@@ -263,7 +268,8 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
     res = dict(cfg=cfg, wl=wl, plan=plan, alg_bytes=alg_bytes, kern_ms=kern_ms,
                region_ms=region_ms, step_ms=step_ms, flush=flush, flush_ms=flush_ms,
                clocks=clk.summary(), status=status,
-               launches_per_step=1 + (plan["num_partitions"] > 1))
+               launches_per_step=1 + (plan["num_partitions"] > 1 or prefix > 0),
+               shared_prefix_blocks=prefix)
 
     if want_e2e:
         # End to end through the public call, as a serving loop runs it: every
@@ -305,7 +311,7 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
                 pa.decode(out_d[b], q_d[b], wl.key_cache, wl.value_cache, cfg.num_kv_heads,
                           cfg.scale, bt_d[b], sl_d[b], cfg.block_size, cfg.max_seq_len,
                           cfg.kv_dtype, wl.k_scale, wl.v_scale, workspace_tensor=ws,
-                          stream=stream)
+                          stream=stream, shared_prefix_blocks=prefix)
                 ev_used[b].record(stream)
                 with torch.cuda.stream(down):
                     down.wait_event(ev_used[b])
@@ -411,6 +417,7 @@ def result_line(idx, r, n_gpus, steps, warmup, cpu=None):
             "l2": ("flushed between steps (256 MiB write, excluded from step time)"
                    if r["flush"] else "inputs larger than L2, no flush"),
             "plan": r["plan"],
+            "shared_prefix_blocks_declared": r["shared_prefix_blocks"],
             "parallelism": f"weak x{n_gpus} (independent batches per GPU)" if n_gpus > 1
             else "1 GPU",
         },
@@ -490,6 +497,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cascade", action="store_true",
+                    help="do not declare a workload's shared prefix (plain per-sequence decode)")
     ap.add_argument("--num-seqs", type=int, default=0,
                     help="run the workload with fewer sequences (profiling captures only)")
     ap.add_argument("--ref-budget", type=float, default=20.0,
@@ -515,7 +524,7 @@ def main(argv=None):
     configs = [1, 2, 3, 4, 5] if args.config == "all" else [int(args.config)]
     for idx in configs:
         r = time_gpu(idx, args.steps, args.warmup, device, want_e2e=not args.no_e2e, rank=rank,
-                     num_seqs=args.num_seqs)
+                     num_seqs=args.num_seqs, cascade=not args.no_cascade)
         r["step_ms"] = reduce_max(r["step_ms"], device)
         if "e2e_ms" in r:
             r["e2e_ms"] = reduce_max(r["e2e_ms"], device)
