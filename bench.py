@@ -452,6 +452,46 @@ def result_line(idx, r, n_gpus, steps, warmup, cpu=None):
     return line
 
 
+def run_copy_blocks(args, device):
+    """Bandwidth of pa_copy_blocks (copy on write of whole blocks) on the
+    Llama-style MHA block geometry: 4096 random (src, dst) pairs per call,
+    256 KiB of K+V per pair, so each call reads and writes 1 GiB."""
+    import torch
+
+    import paged_kv_cache_471_b200 as pa
+    from paged_kv_cache_471_b200 import workloads as W
+    cfg = W.CONFIGS[2]
+    kc = torch.empty(cfg.key_cache_shape(), dtype=torch.bfloat16, device=device)
+    vc = torch.empty(cfg.value_cache_shape(), dtype=torch.bfloat16, device=device)
+    kc.view(torch.int16).fill_(1)
+    vc.view(torch.int16).fill_(2)
+    n = 4096
+    g = torch.Generator().manual_seed(17)
+    perm = torch.randperm(cfg.num_blocks, generator=g)
+    src, dst = perm[:n].to(device), perm[n:2 * n].to(device)
+    moved = 2 * 2 * n * cfg.page_bytes() * cfg.num_kv_heads  # (K+V) x (read+write)
+    for _ in range(args.warmup):
+        pa.copy_blocks(kc, vc, src, dst)
+    torch.cuda.synchronize(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        pa.copy_blocks(kc, vc, src, dst)
+    b.record()
+    torch.cuda.synchronize(device)
+    ms = a.elapsed_time(b) / args.steps
+    peak, kind = measured_hbm_peak()
+    gbs = moved / (ms * 1e-3) / 1e9
+    print(json.dumps({"metric": "block copy (copy on write) GB/s, read+write", "value": round(gbs, 2),
+                      "unit": "GB/s", "ms_per_step": round(ms, 5), "steps": args.steps,
+                      "config": {"workload": f"{n} random block pairs, {cfg.num_kv_heads} kv heads "
+                                             f"x 128 x 16 bf16 (K+V 256 KiB per pair)",
+                                 "bytes_per_step": moved},
+                      "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": peak,
+                                   "peak_kind": kind, "unit": "GB/s",
+                                   "frac": round(gbs / peak, 4)}}), flush=True)
+
+
 def run_reference(args):
     """The oracle as the reference arm: each step one bounded sample."""
     import torch
@@ -497,6 +537,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--extra", default="", choices=["", "copy_blocks"],
+                    help="measure a side kernel instead of decode")
     ap.add_argument("--no-cascade", action="store_true",
                     help="do not declare a workload's shared prefix (plain per-sequence decode)")
     ap.add_argument("--num-seqs", type=int, default=0,
@@ -521,6 +563,10 @@ def main(argv=None):
     import paged_kv_cache_471_b200 as pa
     pa.lib()
 
+    if args.extra == "copy_blocks":
+        if rank == 0:
+            run_copy_blocks(args, device)
+        return 0
     configs = [1, 2, 3, 4, 5] if args.config == "all" else [int(args.config)]
     for idx in configs:
         r = time_gpu(idx, args.steps, args.warmup, device, want_e2e=not args.no_e2e, rank=rank,

@@ -60,7 +60,8 @@ typedef enum pa_status {
     PA_ERR_INVALID_ARG = 1,        /* null / misaligned pointer, inconsistent sizes    */
     PA_ERR_UNSUPPORTED = 2,        /* head_size, block_size, group size, dtype          */
     PA_ERR_WORKSPACE_TOO_SMALL = 3,/* workspace_bytes < pa_decode_workspace_size(...)   */
-    PA_ERR_CUDA = 4                /* a CUDA runtime call or launch failed              */
+    PA_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed              */
+    PA_ERR_OUT_OF_BLOCKS = 5       /* block manager: no free block / block-table row full */
 } pa_status;
 
 typedef enum pa_kv_dtype {
@@ -222,6 +223,77 @@ const char* pa_last_error_detail(void);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 int pa_version(void);
+
+/* ------------------------------------------------------------------------
+ * Block manager: hands out physical blocks and keeps the block tables that
+ * pa_decode reads.  It follows the PagedAttention idea of "vLLM 0.25.0
+ * release-notes commentary", section 1 (a sequence is like a process, a KV
+ * block like a page, the block table like a page table): blocks are
+ * allocated only when a sequence grows into them, and several sequences
+ * (e.g. outputs sampled from one prompt) can share blocks, a shared block
+ * being copied before it is written ("copy on write").
+ *
+ * Host-only bookkeeping, thread-safe (one mutex per manager); it never
+ * touches device memory.  Block ids are handed out in increasing order from
+ * a LIFO free list, so the sequence of ids is deterministic.
+ * ------------------------------------------------------------------------ */
+typedef struct pa_block_manager pa_block_manager;
+
+/* A manager of blocks [0, num_blocks) of block_size tokens; a sequence may
+ * hold at most max_blocks_per_seq blocks (the block-table row width). */
+pa_status pa_bm_create(pa_block_manager** out, int64_t num_blocks, int block_size,
+                       int max_blocks_per_seq);
+void pa_bm_destroy(pa_block_manager* bm);
+
+/* A new, empty sequence; *seq_id indexes the manager's sequences (ids of
+ * freed sequences are reused). */
+pa_status pa_bm_add_sequence(pa_block_manager* bm, int* seq_id);
+
+/* A new sequence that shares every block of `parent` (their reference counts
+ * go up by one) and has the parent's length. */
+pa_status pa_bm_fork(pa_block_manager* bm, int parent, int* child_id);
+
+/* Drop a sequence; blocks no other sequence references return to the pool. */
+pa_status pa_bm_free_sequence(pa_block_manager* bm, int seq_id);
+
+/*
+ * Grow a sequence by num_tokens, allocating the blocks it grows into.  When
+ * the sequence's last block is partly filled and shared with another
+ * sequence, that block is first replaced by a private copy: the call then
+ * returns *num_copies = 1 with the (source, destination) block ids in
+ * *copy_src / *copy_dst, and the caller must copy the block's K/V (for
+ * instance with pa_copy_blocks) before writing the new tokens.  All or
+ * nothing: on PA_ERR_OUT_OF_BLOCKS nothing changes.
+ */
+pa_status pa_bm_append_tokens(pa_block_manager* bm, int seq_id, int num_tokens,
+                              int64_t* copy_src, int64_t* copy_dst, int* num_copies);
+
+pa_status pa_bm_seq_len(pa_block_manager* bm, int seq_id, int64_t* len);
+
+/*
+ * Write the block-table rows and lengths of n sequences, in the given order,
+ * into host arrays block_tables [n, max_blocks_per_seq] (unused entries -1)
+ * and seq_lens [n], ready to copy to the device for pa_decode.
+ */
+pa_status pa_bm_export(pa_block_manager* bm, const int* seq_ids, int n, int32_t* block_tables,
+                       int max_blocks_per_seq, int32_t* seq_lens);
+
+int64_t pa_bm_num_free_blocks(pa_block_manager* bm);          /* -1 on NULL            */
+int pa_bm_refcount(pa_block_manager* bm, int64_t block);       /* -1 on a bad argument  */
+const char* pa_bm_last_error_detail(void);                     /* this thread's last    */
+
+/*
+ * Copy whole blocks (every kv head, K and V) within the caches:
+ * block dst[i] <- block src[i] for i < num_pairs.  src and dst are device
+ * arrays of int64 block ids.  A dst id must not appear twice, nor as a src,
+ * in one call.  Pairs with an id outside [0, num_blocks) are skipped and set
+ * PA_DEV_BAD_BLOCK_ID in *status (a device word; may be NULL).  Enqueued on
+ * `stream`; caches 16-byte aligned.
+ */
+pa_status pa_copy_blocks(void* key_cache, void* value_cache, int num_kv_heads, int head_size,
+                         int block_size, int64_t num_blocks, pa_kv_dtype kv_dtype,
+                         const int64_t* src, const int64_t* dst, int num_pairs,
+                         uint32_t* status, void* stream);
 
 #ifdef __cplusplus
 }

@@ -24,6 +24,7 @@ PA_ERR_INVALID_ARG = 1
 PA_ERR_UNSUPPORTED = 2
 PA_ERR_WORKSPACE_TOO_SMALL = 3
 PA_ERR_CUDA = 4
+PA_ERR_OUT_OF_BLOCKS = 5
 
 PA_KV_BF16 = 0
 PA_KV_FP8_E4M3 = 1
@@ -91,6 +92,32 @@ def _bind(lib):
     lib.pa_last_error_detail.restype = ctypes.c_char_p
     lib.pa_version.argtypes = []
     lib.pa_version.restype = _I
+    I64 = ctypes.c_int64
+    lib.pa_bm_create.argtypes = [ctypes.POINTER(_P), I64, _I, _I]
+    lib.pa_bm_create.restype = _I
+    lib.pa_bm_destroy.argtypes = [_P]
+    lib.pa_bm_destroy.restype = None
+    lib.pa_bm_add_sequence.argtypes = [_P, ctypes.POINTER(_I)]
+    lib.pa_bm_add_sequence.restype = _I
+    lib.pa_bm_fork.argtypes = [_P, _I, ctypes.POINTER(_I)]
+    lib.pa_bm_fork.restype = _I
+    lib.pa_bm_free_sequence.argtypes = [_P, _I]
+    lib.pa_bm_free_sequence.restype = _I
+    lib.pa_bm_append_tokens.argtypes = [_P, _I, _I, ctypes.POINTER(I64), ctypes.POINTER(I64),
+                                        ctypes.POINTER(_I)]
+    lib.pa_bm_append_tokens.restype = _I
+    lib.pa_bm_seq_len.argtypes = [_P, _I, ctypes.POINTER(I64)]
+    lib.pa_bm_seq_len.restype = _I
+    lib.pa_bm_export.argtypes = [_P, _P, _I, _P, _I, _P]
+    lib.pa_bm_export.restype = _I
+    lib.pa_bm_num_free_blocks.argtypes = [_P]
+    lib.pa_bm_num_free_blocks.restype = I64
+    lib.pa_bm_refcount.argtypes = [_P, I64]
+    lib.pa_bm_refcount.restype = _I
+    lib.pa_bm_last_error_detail.argtypes = []
+    lib.pa_bm_last_error_detail.restype = ctypes.c_char_p
+    lib.pa_copy_blocks.argtypes = [_P, _P, _I, _I, _I, I64, _I, _P, _P, _I, _P, _P]
+    lib.pa_copy_blocks.restype = _I
     return lib
 
 
@@ -279,3 +306,95 @@ def read_status(workspace_tensor=None, device=None, clear=False, stream=None) ->
 
 def version() -> int:
     return int(lib().pa_version())
+
+
+# --------------------------------------------------------------- block manager
+def _bm_check(rc: int):
+    if rc != PA_OK:
+        L = lib()
+        raise PagedAttentionError(rc, f"{L.pa_status_string(rc).decode()}: "
+                                      f"{L.pa_bm_last_error_detail().decode()}")
+
+
+class BlockManager:
+    """Host block allocator of libpagedattn (``pa_bm_*``): blocks on demand,
+    forked sequences sharing blocks, copy on write of a shared partial block."""
+
+    def __init__(self, num_blocks: int, block_size: int, max_blocks_per_seq: int):
+        self._h = ctypes.c_void_p()
+        _bm_check(lib().pa_bm_create(ctypes.byref(self._h), int(num_blocks), int(block_size),
+                                     int(max_blocks_per_seq)))
+        self.num_blocks, self.block_size = int(num_blocks), int(block_size)
+        self.max_blocks_per_seq = int(max_blocks_per_seq)
+
+    def close(self):
+        if self._h:
+            lib().pa_bm_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def add_sequence(self) -> int:
+        i = ctypes.c_int()
+        _bm_check(lib().pa_bm_add_sequence(self._h, ctypes.byref(i)))
+        return i.value
+
+    def fork(self, parent: int) -> int:
+        i = ctypes.c_int()
+        _bm_check(lib().pa_bm_fork(self._h, int(parent), ctypes.byref(i)))
+        return i.value
+
+    def free(self, seq: int):
+        _bm_check(lib().pa_bm_free_sequence(self._h, int(seq)))
+
+    def append(self, seq: int, num_tokens: int):
+        """Grow a sequence; returns (src, dst) when a copy on write is needed."""
+        a, b, n = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int()
+        _bm_check(lib().pa_bm_append_tokens(self._h, int(seq), int(num_tokens), ctypes.byref(a),
+                                            ctypes.byref(b), ctypes.byref(n)))
+        return (a.value, b.value) if n.value else None
+
+    def seq_len(self, seq: int) -> int:
+        n = ctypes.c_int64()
+        _bm_check(lib().pa_bm_seq_len(self._h, int(seq), ctypes.byref(n)))
+        return n.value
+
+    def export(self, seqs):
+        """(block_tables int32 [n, max_blocks_per_seq], seq_lens int32 [n]) on the host."""
+        import numpy as np
+        ids = np.ascontiguousarray(np.asarray(seqs, dtype=np.int32))
+        bt = np.empty((len(ids), self.max_blocks_per_seq), dtype=np.int32)
+        sl = np.empty((len(ids),), dtype=np.int32)
+        _bm_check(lib().pa_bm_export(self._h, ids.ctypes.data, len(ids), bt.ctypes.data,
+                                     self.max_blocks_per_seq, sl.ctypes.data))
+        return bt, sl
+
+    def num_free_blocks(self) -> int:
+        return int(lib().pa_bm_num_free_blocks(self._h))
+
+    def refcount(self, block: int) -> int:
+        return int(lib().pa_bm_refcount(self._h, int(block)))
+
+
+def copy_blocks(key_cache, value_cache, src, dst, kv_dtype="bf16", status=None, stream=None):
+    """Copy whole blocks (all kv heads, K and V): block dst[i] <- block src[i].
+    src / dst: int64 CUDA tensors of block ids."""
+    import torch
+    code = kv_dtype_code(kv_dtype)
+    dev = key_cache.device
+    kv_types = (torch.bfloat16,) if code == PA_KV_BF16 else (torch.uint8, torch.float8_e4m3fn)
+    n = int(src.numel())
+    if int(dst.numel()) != n:
+        raise ValueError("src and dst must have the same length")
+    Hk, D = value_cache.shape[1], value_cache.shape[2]
+    st = stream if stream is not None else torch.cuda.current_stream(dev)
+    rc = lib().pa_copy_blocks(
+        _ptr(key_cache, "key_cache", kv_types, dev), _ptr(value_cache, "value_cache", kv_types, dev),
+        int(Hk), int(D), int(value_cache.shape[3]), int(key_cache.shape[0]), code,
+        _ptr(src, "src", (torch.int64,), dev), _ptr(dst, "dst", (torch.int64,), dev), n,
+        None if status is None else _ptr(status, "status", None, dev), st.cuda_stream)
+    _bm_check(rc)

@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpagedattn.so")
-SOURCES = [os.path.join(CSRC, "pa_decode.cu")]
+SOURCES = [os.path.join(CSRC, "pa_decode.cu"), os.path.join(CSRC, "pa_blocks.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + [
     os.path.join(INCLUDE, "pagedattn.h")]
 

@@ -471,6 +471,7 @@ const char* pa_status_string(pa_status status) {
         case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED: unsupported shape or dtype";
         case PA_ERR_WORKSPACE_TOO_SMALL: return "PA_ERR_WORKSPACE_TOO_SMALL: workspace too small";
         case PA_ERR_CUDA: return "PA_ERR_CUDA: CUDA runtime error";
+        case PA_ERR_OUT_OF_BLOCKS: return "PA_ERR_OUT_OF_BLOCKS: no free block or row full";
     }
     return "unknown pa_status";
 }
