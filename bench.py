@@ -199,7 +199,7 @@ def workload_config(idx: int, num_seqs: int = 0):
 
 
 def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, num_seqs=0,
-             cascade=True):
+             cascade=True, alibi=False):
     import torch
 
     import paged_kv_cache_471_b200 as pa
@@ -210,7 +210,11 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
     out = torch.empty_like(wl.query)
     # A workload whose sequences share a prompt prefix declares it, so the
     # prefix pages are streamed once per group of query rows (cascade decode).
-    prefix = cfg.shared_prefix_blocks if cascade else 0
+    prefix = cfg.shared_prefix_blocks if (cascade and not alibi) else 0
+    slopes = None
+    if alibi:  # geometric ALiBi slopes 2^(-8 i / H)
+        slopes = torch.tensor([2.0 ** (-8.0 * (i + 1) / cfg.num_heads)
+                               for i in range(cfg.num_heads)], dtype=torch.float32, device=device)
     plan = pa.plan(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_size, cfg.block_size,
                    cfg.max_seq_len, cfg.kv_dtype, shared_prefix_blocks=prefix)
     ws = torch.zeros(plan["workspace_bytes"], dtype=torch.uint8, device=device)
@@ -224,7 +228,7 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
         pa.decode(out, wl.query, wl.key_cache, wl.value_cache, cfg.num_kv_heads, cfg.scale,
                   wl.block_tables, wl.seq_lens, cfg.block_size, cfg.max_seq_len, cfg.kv_dtype,
                   wl.k_scale, wl.v_scale, workspace_tensor=ws, stream=stream,
-                  shared_prefix_blocks=prefix)
+                  shared_prefix_blocks=prefix, alibi_slopes=slopes)
 
     for _ in range(max(warmup, 3)):
         if flush:
@@ -269,7 +273,7 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
                region_ms=region_ms, step_ms=step_ms, flush=flush, flush_ms=flush_ms,
                clocks=clk.summary(), status=status,
                launches_per_step=1 + (plan["num_partitions"] > 1 or prefix > 0),
-               shared_prefix_blocks=prefix)
+               shared_prefix_blocks=prefix, alibi=alibi)
 
     if want_e2e:
         # End to end through the public call, as a serving loop runs it: every
@@ -311,7 +315,7 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
                 pa.decode(out_d[b], q_d[b], wl.key_cache, wl.value_cache, cfg.num_kv_heads,
                           cfg.scale, bt_d[b], sl_d[b], cfg.block_size, cfg.max_seq_len,
                           cfg.kv_dtype, wl.k_scale, wl.v_scale, workspace_tensor=ws,
-                          stream=stream, shared_prefix_blocks=prefix)
+                          stream=stream, shared_prefix_blocks=prefix, alibi_slopes=slopes)
                 ev_used[b].record(stream)
                 with torch.cuda.stream(down):
                     down.wait_event(ev_used[b])
@@ -418,6 +422,7 @@ def result_line(idx, r, n_gpus, steps, warmup, cpu=None):
                    if r["flush"] else "inputs larger than L2, no flush"),
             "plan": r["plan"],
             "shared_prefix_blocks_declared": r["shared_prefix_blocks"],
+            "alibi": r["alibi"],
             "parallelism": f"weak x{n_gpus} (independent batches per GPU)" if n_gpus > 1
             else "1 GPU",
         },
@@ -539,6 +544,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--extra", default="", choices=["", "copy_blocks"],
                     help="measure a side kernel instead of decode")
+    ap.add_argument("--alibi", action="store_true", help="decode with ALiBi slopes")
     ap.add_argument("--no-cascade", action="store_true",
                     help="do not declare a workload's shared prefix (plain per-sequence decode)")
     ap.add_argument("--num-seqs", type=int, default=0,
@@ -570,7 +576,7 @@ def main(argv=None):
     configs = [1, 2, 3, 4, 5] if args.config == "all" else [int(args.config)]
     for idx in configs:
         r = time_gpu(idx, args.steps, args.warmup, device, want_e2e=not args.no_e2e, rank=rank,
-                     num_seqs=args.num_seqs, cascade=not args.no_cascade)
+                     num_seqs=args.num_seqs, cascade=not args.no_cascade, alibi=args.alibi)
         r["step_ms"] = reduce_max(r["step_ms"], device)
         if "e2e_ms" in r:
             r["e2e_ms"] = reduce_max(r["e2e_ms"], device)

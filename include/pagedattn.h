@@ -99,12 +99,19 @@ typedef enum pa_kv_dtype {
  *      Kernels verify the declaration and set PA_DEV_PREFIX_MISMATCH when a
  *      row's prefix differs from row 0's or a sequence is shorter than the
  *      prefix (results for that sequence are then undefined).  0 = off.
+ *  alibi_slopes: NULL, or a device array of num_heads fp32 slopes.  The call
+ *      on "PR #47361 report: Delete PagedAttention" (benchmark snippet) passes
+ *      alibi_slopes; the bias itself is not printed there, and is read as the
+ *      usual linear bias: the logit of token t (of T) of query head h gains
+ *      slope[h] * (t - (T - 1)).  Not combined with shared_prefix_blocks
+ *      (PA_ERR_UNSUPPORTED).
  */
 typedef struct pa_options {
     int partition_pages;
     int num_sms;
     int stages;
     int shared_prefix_blocks;
+    const float* alibi_slopes;
 } pa_options;
 
 /* What pa_decode will launch for a given problem. */

@@ -12,7 +12,9 @@ Every function here only marshals arguments; the arithmetic is in
 Parity status of each oracle function (what pins it is in tests/test_oracle.py):
   * oracle_pa_decode   -- pinned: dense SDPA equivalence, block-permutation
     invariance, uniform-logit mean, seq_len = 1, brute force at T <= 4,
-    a hand-derived golden case, planted-mistake sensitivity.
+    a hand-derived golden case, planted-mistake sensitivity; with ALiBi
+    slopes: SDPA with the additive bias as its mask, brute force, and zero
+    slopes reproducing the unbiased result bit for bit.
   * e4m3 / bf16 decode -- pinned: all 256 / 65536 codes against torch's
     float8_e4m3fn / bfloat16 conversions, and spot values of the format.
 """
@@ -57,7 +59,7 @@ def _bind(lib):
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
         ctypes.c_double, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_double,
-        ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_int]
+        ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
     lib.oracle_bf16_to_double.restype = ctypes.c_double
     lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
     lib.oracle_e4m3_to_double.restype = ctypes.c_double
@@ -96,7 +98,7 @@ def _np(t, dtype):
 def pa_decode(query, key_cache, value_cache, num_kv_heads: int, scale: float, block_tables,
               seq_lens, block_size: int, kv_dtype: int = KV_BF16, k_scale: float = 1.0,
               v_scale: float = 1.0, x: int | None = None, pairs=None, threads: int = 0,
-              lib=None) -> np.ndarray:
+              lib=None, alibi_slopes=None) -> np.ndarray:
     """fp64 attention output.
 
     query bf16 [S, Hq, D]; caches in the paged layouts (bf16 or e4m3 codes);
@@ -122,11 +124,16 @@ def pa_decode(query, key_cache, value_cache, num_kv_heads: int, scale: float, bl
         n_rows = S * Hq
         pr_ptr = None
     out = np.zeros((n_rows, D), dtype=np.float64)
+    slopes = None if alibi_slopes is None else np.ascontiguousarray(
+        _np(alibi_slopes, np.float32), dtype=np.float32)
+    if slopes is not None and slopes.shape != (Hq,):
+        raise ValueError("alibi_slopes must have one entry per query head")
     rc = lib.oracle_pa_decode(out.ctypes.data, q.ctypes.data, kc.ctypes.data, vc.ctypes.data,
                               int(kv_dtype), S, Hq, int(num_kv_heads), D, int(block_size),
                               int(x), float(scale), bt.ctypes.data, bt.shape[1], sl.ctypes.data,
                               float(k_scale), float(v_scale), n_rows if pr is not None else 0,
-                              pr_ptr, int(threads))
+                              pr_ptr, int(threads),
+                              None if slopes is None else slopes.ctypes.data)
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     return out if pairs is not None else out.reshape(S, Hq, D)

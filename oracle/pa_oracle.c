@@ -35,6 +35,12 @@
  *  - e4m3 is the OCP "fn" variant: bias 7, no infinities, S.1111.111 = NaN;
  *  - dequantised values are code * scale, formed exactly in fp64;
  *  - seq_len = 0 gives a zero output row; no causal mask (decode reads all T).
+ *
+ * Optional ALiBi bias: the call on "PR #47361 report: Delete PagedAttention"
+ * (benchmark snippet) carries an alibi_slopes argument but the pages do not
+ * print the bias.  Reading: the usual linear bias, per query head,
+ *     l_t += slope[h] * (t - (T - 1))
+ * i.e. the key position minus the decoding query's position T - 1.
  */
 #include <math.h>
 #include <stdint.h>
@@ -80,7 +86,7 @@ static double load_elem(const void* base, int64_t idx, int kv_dtype, double scl)
 static void one_row(double* out_row, const uint16_t* q_row, const void* key_cache,
                     const void* value_cache, int kv_dtype, int Hk, int D, int B, int x,
                     double scale, const int32_t* bt_row, int T, int g, double k_scale,
-                    double v_scale, double* logit) {
+                    double v_scale, double slope, double* logit) {
     int d, t;
     double qd[512];
     for (d = 0; d < D; ++d) qd[d] = oracle_bf16_to_double(q_row[d]);
@@ -97,7 +103,7 @@ static void one_row(double* out_row, const uint16_t* q_row, const void* key_cach
             int64_t ki = ((((pb * Hk + g) * (D / x) + d / x) * B + o) * x) + d % x;
             acc += qd[d] * load_elem(key_cache, ki, kv_dtype, k_scale);
         }
-        logit[t] = scale * acc;
+        logit[t] = scale * acc + slope * (double)(t - (T - 1));
         if (logit[t] > mx) mx = logit[t];
     }
     /* softmax weights and the weighted sum of V */
@@ -116,6 +122,7 @@ static void one_row(double* out_row, const uint16_t* q_row, const void* key_cach
 }
 
 /*
+ * alibi_slopes: fp32 [Hq] or NULL (no bias).
  * out:        fp64 [n_rows][D]; rows are (s, h) in row-major order when
  *             pairs == NULL (n_rows = S * Hq), else pairs[2i], pairs[2i+1].
  * query:      bf16 bits [S][Hq][D]
@@ -127,7 +134,7 @@ int oracle_pa_decode(double* out, const uint16_t* query, const void* key_cache,
                      const void* value_cache, int kv_dtype, int S, int Hq, int Hk, int D, int B,
                      int x, double scale, const int32_t* block_tables, int max_blocks_per_seq,
                      const int32_t* seq_lens, double k_scale, double v_scale, int n_pairs,
-                     const int32_t* pairs, int n_threads) {
+                     const int32_t* pairs, int n_threads, const float* alibi_slopes) {
     if (S < 0 || Hq <= 0 || Hk <= 0 || Hq % Hk || D <= 0 || D > 512 || B <= 0 || x <= 0 ||
         D % x)
         return -1;
@@ -160,7 +167,7 @@ int oracle_pa_decode(double* out, const uint16_t* query, const void* key_cache,
             one_row(out + (int64_t)i * D, query + ((int64_t)s * Hq + h) * D, key_cache,
                     value_cache, kv_dtype, Hk, D, B, x, scale,
                     block_tables + (int64_t)s * max_blocks_per_seq, seq_lens[s], h / G, k_scale,
-                    v_scale, logit);
+                    v_scale, alibi_slopes ? (double)alibi_slopes[h] : 0.0, logit);
         }
         free(logit);
     }

@@ -49,7 +49,8 @@ class PagedAttentionError(RuntimeError):
 
 class Options(ctypes.Structure):
     _fields_ = [("partition_pages", ctypes.c_int), ("num_sms", ctypes.c_int),
-                ("stages", ctypes.c_int), ("shared_prefix_blocks", ctypes.c_int)]
+                ("stages", ctypes.c_int), ("shared_prefix_blocks", ctypes.c_int),
+                ("alibi_slopes", ctypes.c_void_p)]
 
 
 class Plan(ctypes.Structure):
@@ -142,11 +143,12 @@ def _check(rc: int):
                                       f"{L.pa_last_error_detail().decode()}")
 
 
-def _opts(partition_pages=0, num_sms=0, stages=0, shared_prefix_blocks=0):
-    if not partition_pages and not num_sms and not stages and not shared_prefix_blocks:
+def _opts(partition_pages=0, num_sms=0, stages=0, shared_prefix_blocks=0, alibi_ptr=None):
+    if not partition_pages and not num_sms and not stages and not shared_prefix_blocks \
+            and not alibi_ptr:
         return None
     return ctypes.byref(Options(int(partition_pages), int(num_sms), int(stages),
-                                int(shared_prefix_blocks)))
+                                int(shared_prefix_blocks), alibi_ptr))
 
 
 def kv_dtype_code(kv_dtype) -> int:
@@ -209,7 +211,7 @@ def _ptr(t, name, dtypes=None, device=None):
 def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, block_tables,
            seq_lens, block_size: int, max_seq_len: int, kv_dtype="bf16", k_scale=None,
            v_scale=None, workspace_tensor=None, partition_pages: int = 0, stream=None,
-           stages: int = 0, shared_prefix_blocks: int = 0):
+           stages: int = 0, shared_prefix_blocks: int = 0, alibi_slopes=None):
     """Paged decode attention into ``out`` (bf16 [num_seqs, num_heads, head_size]).
 
     key_cache: [num_blocks, num_kv_heads, head_size/x, block_size, x];
@@ -251,13 +253,18 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
     if workspace_tensor is None:
         workspace_tensor = workspace(need, dev)
     ws = _ptr(workspace_tensor, "workspace", None, dev)
+    alibi = None
+    if alibi_slopes is not None:
+        if alibi_slopes.shape != (Hq,):
+            raise ValueError("alibi_slopes must be [num_heads]")
+        alibi = _ptr(alibi_slopes, "alibi_slopes", (torch.float32,), dev)
     st = stream if stream is not None else torch.cuda.current_stream(dev)
     rc = lib().pa_decode_ex(*args_ptrs, S, Hq, int(num_kv_heads), D, float(scale), bt,
                             block_tables.shape[1], sl, int(block_size), int(max_seq_len),
                             int(num_blocks), code, ks, vs, ws,
                             workspace_tensor.numel() * workspace_tensor.element_size(),
                             st.cuda_stream,
-                            _opts(partition_pages, 0, stages, shared_prefix_blocks))
+                            _opts(partition_pages, 0, stages, shared_prefix_blocks, alibi))
     _check(rc)
     return out
 

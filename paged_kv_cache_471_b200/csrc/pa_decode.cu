@@ -101,6 +101,8 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         return fail(PA_ERR_INVALID_ARG, "%s",
                     "opts->shared_prefix_blocks must be in [0, max_seq_len / block_size]");
     const bool cascade = prefix > 0 && num_seqs > 0;
+    if (cascade && opts->alibi_slopes)
+        return fail(PA_ERR_UNSUPPORTED, "%s", "ALiBi slopes with a shared prefix");
     const size_t stage = 2ull * head_size * block_size * elem_bytes(kv_dtype);
     const int W = pa::decode_warps(static_cast<long long>(stage));
     int ns = kDefaultStages;
@@ -336,6 +338,8 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
         if (!q.p) return fail(PA_ERR_INVALID_ARG, "%s is NULL", q.name);
         if (!aligned(q.p, q.a)) return fail(PA_ERR_INVALID_ARG, "%s is misaligned", q.name);
     }
+    if (opts && opts->alibi_slopes && !aligned(opts->alibi_slopes, 4))
+        return fail(PA_ERR_INVALID_ARG, "%s", "alibi_slopes is misaligned");
     if (kv_dtype == PA_KV_FP8_E4M3) {
         if (!k_scale || !v_scale)
             return fail(PA_ERR_INVALID_ARG, "%s", "k_scale and v_scale are required for FP8");
@@ -383,6 +387,7 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
     p.prefix_groups = pl.prefix_groups;
     p.prefix_units = static_cast<long long>(num_kv_heads) * pl.prefix_groups * pl.prefix_partitions;
     p.P_total = p_total;
+    p.alibi = opts ? opts->alibi_slopes : nullptr;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = launch_any(p, head_size, block_size, kv_dtype == PA_KV_FP8_E4M3, pl.grid_ctas,

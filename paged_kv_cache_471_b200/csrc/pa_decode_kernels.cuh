@@ -76,6 +76,7 @@ struct DecodeParams {
     int prefix_groups;        // 16-row groups of the S*G query rows of a kv head
     long long prefix_units;   // Hk * prefix_groups * prefix_parts
     int P_total;              // partial slots per (seq, q head): prefix_parts + P
+    const float* alibi;       // [Hq] ALiBi slopes, or nullptr
 };
 
 // Bytes of shared memory the final merge needs (it overlays the page stages).
@@ -183,6 +184,14 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
     if constexpr (FP8) {
         k_scale = __ldg(p.k_scale);
         v_scale = __ldg(p.v_scale);
+    }
+    // ALiBi: logit of token t gains slope * (t - (T - 1)); kept in log2 units.
+    const bool has_alibi = p.alibi != nullptr;
+    float slope2[NH];
+#pragma unroll
+    for (int r = 0; r < NH; ++r) {
+        const long long qr = row_of(8 * r + gq);
+        slope2[r] = (has_alibi && qr >= 0) ? __ldg(p.alibi + qr % p.Hq) * 1.4426950408889634f : 0.f;
     }
 
     // ---- sequence length, with the device-side range checks
@@ -342,7 +351,7 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
 
     // One landed page: S = Q K^T, online softmax, O^T += V^T P^T.  FULL pages
     // (every slot a token) skip all masking.
-    auto page = [&](auto full_tag, const uint32_t kbase, const int valid) {
+    auto page = [&](auto full_tag, const uint32_t kbase, const int valid, const int pos0) {
         constexpr bool FULL = decltype(full_tag)::value;
         const uint32_t vbase = kbase + PAGE;
 
@@ -397,6 +406,8 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     float x = sc[nt][2 * r + e] * qk_mul;
+                    if (has_alibi)
+                        x = fmaf(slope2[r], static_cast<float>(pos0 + 8 * nt + 2 * cq + e), x);
                     if constexpr (!FULL) {
                         if (8 * nt + 2 * cq + e >= valid) x = -INFINITY;
                     }
@@ -528,10 +539,11 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
         const int jg = j0 + warp + W * k;
         const int valid = ((valid_mask >> stage) & 1u) ? min(B, T - jg * B) : 0;
         const uint32_t kbase = wstage0 + static_cast<uint32_t>(stage * STAGE);
+        const int pos0 = jg * B - (T - 1);  // ALiBi position of the page's first slot
         if (valid == B)
-            page(std::true_type{}, kbase, valid);
+            page(std::true_type{}, kbase, valid, pos0);
         else
-            page(std::false_type{}, kbase, valid);
+            page(std::false_type{}, kbase, valid, pos0);
         __syncwarp();
         if (k + NS < n_my) issue(k + NS);
         if (++stage == NS) {

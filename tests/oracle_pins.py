@@ -118,8 +118,9 @@ class Case:
                                 np.asarray(self.seq_lens, np.int32), self.B, self.kv,
                                 self.k_scale, self.v_scale, x=self.x, lib=lib, **kw)
 
-    def dense(self):
-        """fp64 SDPA on the contiguous K/V (library routine)."""
+    def dense(self, alibi_slopes=None):
+        """fp64 SDPA on the contiguous K/V (library routine); an ALiBi bias
+        enters as SDPA's additive float mask."""
         G = self.Hq // self.Hk
         out = torch.zeros((self.S, self.Hq, self.D), dtype=torch.float64)
         for s, T in enumerate(self.seq_lens):
@@ -130,7 +131,12 @@ class Case:
             K = K.repeat_interleave(G, dim=0)  # [Hq, T, D]
             V = V.repeat_interleave(G, dim=0)
             q = self.q[s].to(torch.float64).unsqueeze(1)  # [Hq, 1, D]
-            o = F.scaled_dot_product_attention(q, K, V, scale=self.scale)
+            mask = None
+            if alibi_slopes is not None:
+                pos = torch.arange(T, dtype=torch.float64) - (T - 1)
+                mask = (torch.as_tensor(alibi_slopes, dtype=torch.float32).to(torch.float64)
+                        [:, None, None] * pos[None, None, :])
+            o = F.scaled_dot_product_attention(q, K, V, attn_mask=mask, scale=self.scale)
             out[s] = o[:, 0, :]
         return out.numpy()
 
@@ -318,5 +324,49 @@ def pin_bf16_table(lib):
             assert v == r, f"bf16 {b:#x}"
 
 
+def _slopes(Hq, seed):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.rand(Hq, generator=g) * 0.5).to(torch.float32)
+
+
+def pin_alibi_dense(lib):
+    for kw in (DENSE_CASES[0], DENSE_CASES[2], DENSE_CASES[3]):
+        c = Case(**kw)
+        sl = _slopes(c.Hq, 21)
+        got = c.run(lib, alibi_slopes=sl)
+        ref = c.dense(alibi_slopes=sl)
+        err = np.max(np.abs(got - ref))
+        assert err < 1e-12, f"alibi dense {kw}: {err}"
+
+
+def pin_alibi_brute_force(lib):
+    c = Case(seed=14, S=2, Hq=4, Hk=2, D=8, B=2, seq_lens=[4, 3])
+    sl = _slopes(4, 22).tolist()
+    got = c.run(lib, alibi_slopes=torch.tensor(sl, dtype=torch.float32))
+    G = 2
+    for s, T in enumerate(c.seq_lens):
+        K = decode_codes(c.Kd[s], c.kv).tolist()
+        V = decode_codes(c.Vd[s], c.kv).tolist()
+        qs = c.q[s].to(torch.float64).tolist()
+        for h in range(4):
+            g = h // G
+            lg = [c.scale * math.fsum(qs[h][d] * K[g][t][d] for d in range(8))
+                  + float(torch.tensor(sl[h], dtype=torch.float32)) * (t - (T - 1))
+                  for t in range(T)]
+            m = max(lg)
+            w = [math.exp(x - m) for x in lg]
+            den = math.fsum(w)
+            want = [math.fsum(w[t] * V[g][t][d] for t in range(T)) / den for d in range(8)]
+            assert np.max(np.abs(got[s, h] - np.array(want))) < 1e-13, (s, h)
+
+
+def pin_alibi_zero_slopes_is_plain(lib):
+    c = Case(**DENSE_CASES[1])
+    a = c.run(lib)
+    b = c.run(lib, alibi_slopes=torch.zeros(c.Hq, dtype=torch.float32))
+    assert np.array_equal(a, b), "zero ALiBi slopes must leave the output unchanged"
+
+
 ALL_PINS = [pin_golden, pin_dense_equivalence, pin_permutation_invariance, pin_uniform_logits,
-            pin_seq_len_one, pin_brute_force, pin_e4m3_table, pin_bf16_table]
+            pin_seq_len_one, pin_brute_force, pin_e4m3_table, pin_bf16_table, pin_alibi_dense,
+            pin_alibi_brute_force, pin_alibi_zero_slopes_is_plain]

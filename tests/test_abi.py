@@ -61,7 +61,7 @@ def _decode(L, **over):
                 num_heads=8, num_kv_heads=2, head_size=128, scale=0.088, block_tables=0x50000,
                 max_blocks_per_seq=4, seq_lens=0x60000, block_size=16, max_seq_len=64,
                 num_blocks=64, kv_dtype=0, k_scale=None, v_scale=None, workspace=0x70000,
-                workspace_bytes=1 << 20, stream=None, opts=ctypes.byref(pa.Options(0, 148, 0, 0)))
+                workspace_bytes=1 << 20, stream=None, opts=ctypes.byref(pa.Options(0, 148, 0, 0, None)))
     args.update(over)
     return L.pa_decode_ex(*args.values())
 
@@ -148,3 +148,11 @@ def test_every_plan_fits_shared_memory():
                         for pp in (0, 1, 2, 3, 5, 16, 64):
                             p = pa.plan(4, 2 * G, 2, D, B, T, kv, partition_pages=pp, num_sms=148)
                             assert p["smem_bytes"] <= 227 * 1024, (D, B, kv, G, T, pp)
+
+
+def test_alibi_with_shared_prefix_is_refused(L):
+    slopes = ctypes.c_void_p(0x80000)
+    rc = _decode(L, opts=ctypes.byref(pa.Options(0, 148, 0, 2, slopes)))
+    assert rc == pa.PA_ERR_UNSUPPORTED
+    rc = _decode(L, opts=ctypes.byref(pa.Options(0, 148, 0, 0, ctypes.c_void_p(0x80002))))
+    assert rc == pa.PA_ERR_INVALID_ARG  # misaligned slopes

@@ -36,7 +36,7 @@ def test_oracle_uses_threads(lib):
 
 MUTANTS = {
     "gqa head map h % Hk": ("h / G, k_scale", "h % Hk, k_scale"),
-    "scale dropped": ("logit[t] = scale * acc;", "logit[t] = acc;"),
+    "scale dropped": ("logit[t] = scale * acc + slope", "logit[t] = acc + slope"),
     "x-lane reversed": (") * x) + d % x;", ") * x) + (x - 1 - d % x);"),
     "V slot reversed": ("+ d) * B + o;", "+ d) * B + (B - 1 - o);"),
     "identity block map": ("int64_t pb = (int64_t)bt_row[t / B];\n        int o = t % B;\n        double acc",
@@ -46,6 +46,8 @@ MUTANTS = {
     "normalised by T": ("out_row[d] /= denom;", "out_row[d] /= (double)T;"),
     "k_scale on V": ("load_elem(value_cache, vi, kv_dtype, v_scale)",
                      "load_elem(value_cache, vi, kv_dtype, k_scale)"),
+    "ALiBi bias sign": ("slope * (double)(t - (T - 1));", "slope * (double)((T - 1) - t);"),
+    "ALiBi slope of the kv head": ("(double)alibi_slopes[h]", "(double)alibi_slopes[h / G]"),
     "last token dropped": ("for (t = 0; t < T; ++t) {\n        int64_t pb = (int64_t)bt_row[t / B];\n        int o = t % B;\n        double p",
                            "for (t = 0; t < T - (T > 1); ++t) {\n        int64_t pb = (int64_t)bt_row[t / B];\n        int o = t % B;\n        double p"),
 }

@@ -160,3 +160,34 @@ def test_shared_prefix_mismatch_is_flagged():
               shared_prefix_blocks=cfg.shared_prefix_blocks)
     torch.cuda.synchronize()
     assert pa.read_status(ws) & pa.PA_DEV_PREFIX_MISMATCH
+
+
+# ----------------------------------------------------------------------- ALiBi
+def alibi_slopes(n):
+    """Geometric slopes 2^(-8 i / n), i = 1..n (the usual ALiBi choice)."""
+    return torch.tensor([2.0 ** (-8.0 * (i + 1) / n) for i in range(n)], dtype=torch.float32)
+
+
+@pytest.mark.parametrize("idx", [1, 3, 4])
+@pytest.mark.parametrize("partition_pages", [0, 5])
+def test_alibi(idx, partition_pages):
+    cfg = REDUCED[idx]
+    wl = W.make_workload(cfg, DEV)
+    sl = alibi_slopes(cfg.num_heads)
+    out = torch.empty_like(wl.query)
+    pa.decode(out, wl.query, wl.key_cache, wl.value_cache, cfg.num_kv_heads, cfg.scale,
+              wl.block_tables, wl.seq_lens, cfg.block_size, cfg.max_seq_len, cfg.kv_dtype,
+              wl.k_scale, wl.v_scale, partition_pages=partition_pages,
+              alibi_slopes=sl.to(DEV))
+    torch.cuda.synchronize()
+    c = wl.cfg
+    from parity_helpers import kv_code
+    import oracle
+    ref = oracle.pa_decode(wl.query.cpu(), wl.key_cache.cpu(), wl.value_cache.cpu(),
+                           c.num_kv_heads, c.scale, wl.block_tables.cpu(), wl.seq_lens.cpu(),
+                           c.block_size, kv_code(c), c.k_scale, c.v_scale, alibi_slopes=sl)
+    compare(out, ref, cfg.kv_dtype, f"alibi cfg{idx} pp={partition_pages}")
+    # the bias matters: the plain result is far from the biased one
+    plain = run_gpu(wl)
+    torch.cuda.synchronize()
+    assert (plain.float() - out.float()).abs().max().item() > 0.05
