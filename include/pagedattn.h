@@ -90,9 +90,10 @@ typedef enum pa_kv_dtype {
  *      per warp (shared memory grows with it; more than fits is rejected).
  *  shared_prefix_blocks: k > 0 declares that the first k logical blocks are
  *      the same physical blocks in every row of block_tables and that every
- *      seq_len is at least k * block_size -- the prompt sharing of
- *      "vLLM 0.25.0 release-notes commentary", section 1 (several outputs
- *      share one prompt's KV).  The prefix pages are then streamed once per
+ *      seq_len is at least k * block_size -- the prompt reuse that
+ *      "vLLM 0.25.0 release-notes commentary", section 1, lists among the gains
+ *      of paging (outputs of one prompt read its KV blocks).  The prefix pages
+ *      are then streamed once per
  *      group of 16 query rows (all sequences' heads of a kv head packed
  *      together) instead of once per sequence, and merged with each
  *      sequence's own pages by the combine kernel ("cascade" decode).
