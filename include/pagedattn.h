@@ -106,6 +106,14 @@ typedef enum pa_kv_dtype {
  *      usual linear bias: the logit of token t (of T) of query head h gains
  *      slope[h] * (t - (T - 1)).  Not combined with shared_prefix_blocks
  *      (PA_ERR_UNSUPPORTED).
+ *  fp8_compute: with an e4m3 cache, non-zero runs q.K^T and P.V as e4m3 x e4m3
+ *      tensor-core products with fp32 accumulation -- the FP8 compute that
+ *      "Why PagedAttention was retired", section 4, names as the successor of
+ *      dequantise-on-load -- instead of converting K/V to f16.  K/V codes go
+ *      into the products unchanged; the query (scaled by a power of two) and
+ *      the softmax weights (x 256) are each carried as a hi + lo pair of e4m3
+ *      codes, about 2^-8 relative together, so accuracy stays near the f16
+ *      path's.  Requires kv_dtype = PA_KV_FP8_E4M3.
  */
 typedef struct pa_options {
     int partition_pages;
@@ -113,6 +121,7 @@ typedef struct pa_options {
     int stages;
     int shared_prefix_blocks;
     const float* alibi_slopes;
+    int fp8_compute;
 } pa_options;
 
 /* What pa_decode will launch for a given problem. */

@@ -50,7 +50,7 @@ class PagedAttentionError(RuntimeError):
 class Options(ctypes.Structure):
     _fields_ = [("partition_pages", ctypes.c_int), ("num_sms", ctypes.c_int),
                 ("stages", ctypes.c_int), ("shared_prefix_blocks", ctypes.c_int),
-                ("alibi_slopes", ctypes.c_void_p)]
+                ("alibi_slopes", ctypes.c_void_p), ("fp8_compute", ctypes.c_int)]
 
 
 class Plan(ctypes.Structure):
@@ -143,12 +143,13 @@ def _check(rc: int):
                                       f"{L.pa_last_error_detail().decode()}")
 
 
-def _opts(partition_pages=0, num_sms=0, stages=0, shared_prefix_blocks=0, alibi_ptr=None):
+def _opts(partition_pages=0, num_sms=0, stages=0, shared_prefix_blocks=0, alibi_ptr=None,
+          fp8_compute=False):
     if not partition_pages and not num_sms and not stages and not shared_prefix_blocks \
-            and not alibi_ptr:
+            and not alibi_ptr and not fp8_compute:
         return None
     return ctypes.byref(Options(int(partition_pages), int(num_sms), int(stages),
-                                int(shared_prefix_blocks), alibi_ptr))
+                                int(shared_prefix_blocks), alibi_ptr, int(bool(fp8_compute))))
 
 
 def kv_dtype_code(kv_dtype) -> int:
@@ -211,7 +212,8 @@ def _ptr(t, name, dtypes=None, device=None):
 def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, block_tables,
            seq_lens, block_size: int, max_seq_len: int, kv_dtype="bf16", k_scale=None,
            v_scale=None, workspace_tensor=None, partition_pages: int = 0, stream=None,
-           stages: int = 0, shared_prefix_blocks: int = 0, alibi_slopes=None):
+           stages: int = 0, shared_prefix_blocks: int = 0, alibi_slopes=None,
+           fp8_compute: bool = False):
     """Paged decode attention into ``out`` (bf16 [num_seqs, num_heads, head_size]).
 
     key_cache: [num_blocks, num_kv_heads, head_size/x, block_size, x];
@@ -264,7 +266,8 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
                             int(num_blocks), code, ks, vs, ws,
                             workspace_tensor.numel() * workspace_tensor.element_size(),
                             st.cuda_stream,
-                            _opts(partition_pages, 0, stages, shared_prefix_blocks, alibi))
+                            _opts(partition_pages, 0, stages, shared_prefix_blocks, alibi,
+                                  fp8_compute))
     _check(rc)
     return out
 

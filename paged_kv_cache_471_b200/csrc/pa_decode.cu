@@ -208,12 +208,12 @@ cudaError_t ensure_smem(K kernel, std::atomic<int>* done) {
     return e;
 }
 
-template <int D, int B, bool FP8, int NH>
+template <int D, int B, bool FP8, int NH, bool F8MMA>
 cudaError_t launch_decode(const pa::DecodeParams& p, long long grid, size_t smem,
                           cudaStream_t st) {
     static std::atomic<int> done[kMaxDevices];
     constexpr int W = pa::decode_warps<D, B, FP8>();
-    auto kern = pa::pa_decode_kernel<D, B, FP8, NH, W>;
+    auto kern = pa::pa_decode_kernel<D, B, FP8, NH, W, F8MMA>;
     if (smem > kMaxSmemPerCta) return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem(kern, done);
     if (e != cudaSuccess) return e;
@@ -221,25 +221,28 @@ cudaError_t launch_decode(const pa::DecodeParams& p, long long grid, size_t smem
     return cudaGetLastError();
 }
 
-template <int D, int B, bool FP8>
+template <int D, int B, bool FP8, bool F8MMA>
 cudaError_t launch_nh(const pa::DecodeParams& p, long long grid, size_t smem, cudaStream_t st) {
     // Shared-prefix units pack 16 query rows, so they need the 16-row form.
-    return (p.G > 8 || p.prefix_pages > 0) ? launch_decode<D, B, FP8, 2>(p, grid, smem, st)
-                                           : launch_decode<D, B, FP8, 1>(p, grid, smem, st);
+    return (p.G > 8 || p.prefix_pages > 0)
+               ? launch_decode<D, B, FP8, 2, F8MMA>(p, grid, smem, st)
+               : launch_decode<D, B, FP8, 1, F8MMA>(p, grid, smem, st);
 }
 
 template <int D, int B>
-cudaError_t launch_dtype(const pa::DecodeParams& p, bool fp8, long long grid, size_t smem,
-                         cudaStream_t st) {
-    return fp8 ? launch_nh<D, B, true>(p, grid, smem, st) : launch_nh<D, B, false>(p, grid, smem, st);
+cudaError_t launch_dtype(const pa::DecodeParams& p, bool fp8, bool f8mma, long long grid,
+                         size_t smem, cudaStream_t st) {
+    if (!fp8) return launch_nh<D, B, false, false>(p, grid, smem, st);
+    return f8mma ? launch_nh<D, B, true, true>(p, grid, smem, st)
+                 : launch_nh<D, B, true, false>(p, grid, smem, st);
 }
 
-cudaError_t launch_any(const pa::DecodeParams& p, int D, int B, bool fp8, long long grid,
-                       size_t smem, cudaStream_t st) {
-    if (D == 64) return B == 16 ? launch_dtype<64, 16>(p, fp8, grid, smem, st)
-                                : launch_dtype<64, 32>(p, fp8, grid, smem, st);
-    return B == 16 ? launch_dtype<128, 16>(p, fp8, grid, smem, st)
-                   : launch_dtype<128, 32>(p, fp8, grid, smem, st);
+cudaError_t launch_any(const pa::DecodeParams& p, int D, int B, bool fp8, bool f8mma,
+                       long long grid, size_t smem, cudaStream_t st) {
+    if (D == 64) return B == 16 ? launch_dtype<64, 16>(p, fp8, f8mma, grid, smem, st)
+                                : launch_dtype<64, 32>(p, fp8, f8mma, grid, smem, st);
+    return B == 16 ? launch_dtype<128, 16>(p, fp8, f8mma, grid, smem, st)
+                   : launch_dtype<128, 32>(p, fp8, f8mma, grid, smem, st);
 }
 
 cudaError_t launch_combine(const pa::CombineParams& c, int D, cudaStream_t st) {
@@ -338,6 +341,8 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
         if (!q.p) return fail(PA_ERR_INVALID_ARG, "%s is NULL", q.name);
         if (!aligned(q.p, q.a)) return fail(PA_ERR_INVALID_ARG, "%s is misaligned", q.name);
     }
+    if (opts && opts->fp8_compute && kv_dtype != PA_KV_FP8_E4M3)
+        return fail(PA_ERR_INVALID_ARG, "%s", "fp8_compute needs an e4m3 KV cache");
     if (opts && opts->alibi_slopes && !aligned(opts->alibi_slopes, 4))
         return fail(PA_ERR_INVALID_ARG, "%s", "alibi_slopes is misaligned");
     if (kv_dtype == PA_KV_FP8_E4M3) {
@@ -390,8 +395,9 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
     p.alibi = opts ? opts->alibi_slopes : nullptr;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_any(p, head_size, block_size, kv_dtype == PA_KV_FP8_E4M3, pl.grid_ctas,
-                               pl.smem_bytes, s);
+    const bool f8mma = opts && opts->fp8_compute && kv_dtype == PA_KV_FP8_E4M3;
+    cudaError_t e = launch_any(p, head_size, block_size, kv_dtype == PA_KV_FP8_E4M3, f8mma,
+                               pl.grid_ctas, pl.smem_bytes, s);
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
     if (pl.num_partitions > 1 || p.prefix_pages > 0) {
         pa::CombineParams c;

@@ -95,9 +95,11 @@ constexpr int decode_warps() {
     return decode_warps(2LL * D * B * (FP8 ? 1 : 2));
 }
 
-template <int D, int B, bool FP8, int NH, int W>
+template <int D, int B, bool FP8, int NH, int W, bool F8MMA>
 __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams p) {
+    static_assert(!F8MMA || FP8, "e4m3 MMAs need e4m3 pages");
     constexpr int ELEM = FP8 ? 1 : 2;
+    constexpr int K32 = D / 32;  // 32-wide k-steps over the head dim (e4m3 MMA)
     constexpr int PAGE = D * B * ELEM;  // one K (or V) page of one kv head
     constexpr int STAGE = 2 * PAGE;
     constexpr int NT = B / 8;   // 8-token n-tiles per page (QK)
@@ -286,10 +288,52 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
     for (int i = 0; i < n_pro; ++i) issue(i);
 
     // ---- Q fragments (A operand of S = Q K^T; rows = heads 8r + gq)
-    uint32_t qa[KT][4];
+    uint32_t qa[F8MMA ? 1 : KT][4];
+    uint32_t qa8[F8MMA ? K32 : 1][2][4];  // e4m3 MMAs: [k-step][hi, lo][regs]
     float qk_mul = p.scale_log2;
     float out_mul = 1.f;
-    if constexpr (!FP8) {
+    if constexpr (F8MMA) {
+        // e4m3 operands: q is scaled by 2^e so that max|q| 2^e < 256, then
+        // split into hi + lo e4m3 codes (about 2^-8 relative together); both
+        // halves multiply the same K bytes, so one accumulator takes both.
+        // Natural d order: register i holds d = 32 jp + 16 (i >> 1) + 4 cq + 0..3.
+        float amax = 0.f;
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int kt = 0; kt < KT; ++kt) {
+                const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
+                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(w0)), fabsf(bf16_hi(w0))),
+                                         fmaxf(fabsf(bf16_lo(w1)), fabsf(bf16_hi(w1)))));
+            }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+        int e = 0;
+        if (amax > 0.f && amax < INFINITY)
+            e = 7 - (static_cast<int>((__float_as_uint(amax) >> 23) & 0xff) - 127);
+        e = max(-100, min(100, e));
+        const float up = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+        const float down = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+#pragma unroll
+        for (int jp = 0; jp < K32; ++jp)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = i & 1, kt = 2 * jp + (i >> 1);
+                if (r >= NH) {  // rows 8..15 unused: zero codes
+                    qa8[jp][0][i] = 0u;
+                    qa8[jp][1][i] = 0u;
+                    continue;
+                }
+                const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
+                float unused;
+                const uint32_t a = split_e4m3x2(bf16_lo(w0) * up, bf16_hi(w0) * up, &unused);
+                const uint32_t b = split_e4m3x2(bf16_lo(w1) * up, bf16_hi(w1) * up, &unused);
+                qa8[jp][0][i] = __byte_perm(a, b, 0x5410);  // hi codes of d .. d+3
+                qa8[jp][1][i] = __byte_perm(a, b, 0x7632);  // lo codes
+            }
+        qk_mul = p.scale_log2 * k_scale * down;
+        out_mul = v_scale;
+    } else if constexpr (!FP8) {
 #pragma unroll
         for (int r = 0; r < 2; ++r)
 #pragma unroll
@@ -375,6 +419,22 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
                         mma_bf16_16816(sc[2 * np], qa[kt], b0, b1);
                         mma_bf16_16816(sc[2 * np + 1], qa[kt], b2, b3);
                     }
+            } else if constexpr (F8MMA) {
+                // K bytes go into the MMA as they are: register = 4 e4m3 codes of
+                // d = 4 cq..4 cq+3 of a 16-d chunk of one token.
+#pragma unroll
+                for (int jp = 0; jp < K32; ++jp)
+#pragma unroll
+                    for (int np = 0; np < NT / 2; ++np) {
+                        const int tok = 8 * (2 * np + (mi & 1)) + r8;
+                        const int chunk = 2 * jp + (mi >> 1);
+                        uint32_t w0, w1, w2, w3;
+                        ldsm_x4(kbase + chunk * CHUNK + tok * 16, w0, w1, w2, w3);
+                        mma_e4m3_16832(sc[2 * np], qa8[jp][0], w0, w2);
+                        mma_e4m3_16832(sc[2 * np], qa8[jp][1], w0, w2);
+                        mma_e4m3_16832(sc[2 * np + 1], qa8[jp][0], w1, w3);
+                        mma_e4m3_16832(sc[2 * np + 1], qa8[jp][1], w1, w3);
+                    }
             } else {
 #pragma unroll
                 for (int jp = 0; jp < KT / 2; ++jp)
@@ -427,7 +487,14 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
                 const float p0 = fast_exp2(v[nt][0] - m_use);
                 const float p1 = fast_exp2(v[nt][1] - m_use);
                 uint32_t w;
-                if constexpr (!FP8) {
+                if constexpr (F8MMA) {
+                    // weights x 256 as hi + lo e4m3 codes (hi pair | lo pair << 16);
+                    // the running sum uses the represented values, in the same x 256
+                    // units as the accumulator.
+                    float sum2;
+                    w = split_e4m3x2(p0 * 256.f, p1 * 256.f, &sum2);
+                    ls += sum2;
+                } else if constexpr (!FP8) {
                     w = pack_bf16x2(p0, p1);
                     ls += bf16_lo(w) + bf16_hi(w);
                 } else {
@@ -456,6 +523,60 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
             }
         }
 
+        if constexpr (F8MMA) {
+            // O^T += V^T P^T with one 32-token e4m3 k-step per page: tokens
+            // 16 kk + 4 cq .. +3 of each k-tile come from the same quad shuffles
+            // as below; V bytes go into the MMA as they are.  Block size 16
+            // leaves the upper 16 tokens of the step empty (zeros).
+            uint32_t bh[NH][2], bl[NH][2];
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+                for (int r = 0; r < NH; ++r) {
+                    if (kk < KK) {
+                        const uint32_t x0 = __shfl_sync(kFull, pp[r][2 * kk], src0);
+                        const uint32_t y0 = __shfl_sync(kFull, pp[r][2 * kk + 1], src0);
+                        const uint32_t x1 = __shfl_sync(kFull, pp[r][2 * kk], src1);
+                        const uint32_t y1 = __shfl_sync(kFull, pp[r][2 * kk + 1], src1);
+                        const uint32_t u0 = hi_half ? y0 : x0;  // tokens 4cq, 4cq+1
+                        const uint32_t u1 = hi_half ? y1 : x1;  // tokens 4cq+2, 4cq+3
+                        bh[r][kk] = __byte_perm(u0, u1, 0x5410);
+                        bl[r][kk] = __byte_perm(u0, u1, 0x7632);
+                    } else {
+                        bh[r][kk] = 0u;
+                        bl[r][kk] = 0u;
+                    }
+                }
+            uint32_t vmask[2] = {kFull, kFull};
+            if constexpr (!FULL) {
+#pragma unroll
+                for (int kk = 0; kk < KK; ++kk) {
+                    const int t0 = 16 * kk + 4 * cq;
+                    vmask[kk] = (t0 < valid ? 0x000000ffu : 0u) | (t0 + 1 < valid ? 0x0000ff00u : 0u) |
+                                (t0 + 2 < valid ? 0x00ff0000u : 0u) | (t0 + 3 < valid ? 0xff000000u : 0u);
+                }
+            }
+#pragma unroll
+            for (int mp = 0; mp < MT / 2; ++mp) {
+                uint32_t w[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
+#pragma unroll
+                for (int kk = 0; kk < KK; ++kk) {
+                    ldsm_x4(vbase + (32 * mp + lane) * B + kk * 16, w[kk][0], w[kk][1], w[kk][2],
+                            w[kk][3]);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) w[kk][i] &= vmask[kk];
+                }
+                const uint32_t a0[4] = {w[0][0], w[0][1], w[1][0], w[1][1]};
+                const uint32_t a1[4] = {w[0][2], w[0][3], w[1][2], w[1][3]};
+#pragma unroll
+                for (int r = 0; r < NH; ++r) {
+                    mma_e4m3_16832(acc[2 * mp][r], a0, bh[r][0], bh[r][1]);
+                    mma_e4m3_16832(acc[2 * mp][r], a0, bl[r][0], bl[r][1]);
+                    mma_e4m3_16832(acc[2 * mp + 1][r], a1, bh[r][0], bh[r][1]);
+                    mma_e4m3_16832(acc[2 * mp + 1][r], a1, bl[r][0], bl[r][1]);
+                }
+            }
+        } else {
         // ---------------- O^T += V^T P^T  (rows: head dim, cols: heads, k: tokens)
         // Per 16-token k-tile, thread cq holds V for tokens 4cq..4cq+3 (one
         // contiguous 4-token group per row), so k = 2cq,2cq+1 <-> tokens
@@ -524,6 +645,7 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
                 }
             }
         }
+        }  // e4m3 MMAs or f16/bf16 MMAs
     };
 
     bool timed_out = false;

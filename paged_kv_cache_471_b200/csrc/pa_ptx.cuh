@@ -110,6 +110,17 @@ __device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D = A(16x32, row) * B(32x8, col) + D on e4m3 operands, fp32 accumulate.
+// Each A/B register holds four consecutive k elements, lowest k in the low byte.
+__device__ __forceinline__ void mma_e4m3_16832(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // 2^x on the special-function unit (PTX ex2.approx, flush-to-zero; 2^-inf = 0).
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;
@@ -129,6 +140,31 @@ __device__ __forceinline__ uint32_t e4m3_lo_pair(uint32_t w) {
 }
 __device__ __forceinline__ uint32_t e4m3_hi_pair(uint32_t w) {
     return e4m3x2_to_f16x2(static_cast<uint16_t>(w >> 16));
+}
+
+// Two floats to two e4m3 codes (round to nearest even, saturating to +-448);
+// `lo` lands in the low byte.
+__device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// x split into two e4m3 codes whose values add up to x to about 2^-8
+// relative: hi = e4m3(x), lo = e4m3(x - hi).  Returns hi | lo << 8 for each
+// of two inputs packed as (hi0, hi1) in the low half-word and (lo0, lo1) in
+// the high one, plus the represented values' sum in *sum.
+__device__ __forceinline__ uint32_t split_e4m3x2(float x0, float x1, float* sum) {
+    const uint16_t h = f32x2_to_e4m3x2(x0, x1);
+    const uint32_t hf = e4m3x2_to_f16x2(h);
+    const float h0 = __half2float(__ushort_as_half(static_cast<unsigned short>(hf & 0xffffu)));
+    const float h1 = __half2float(__ushort_as_half(static_cast<unsigned short>(hf >> 16)));
+    const uint16_t l = f32x2_to_e4m3x2(x0 - h0, x1 - h1);
+    const uint32_t lf = e4m3x2_to_f16x2(l);
+    const float l0 = __half2float(__ushort_as_half(static_cast<unsigned short>(lf & 0xffffu)));
+    const float l1 = __half2float(__ushort_as_half(static_cast<unsigned short>(lf >> 16)));
+    *sum = (h0 + l0) + (h1 + l1);
+    return static_cast<uint32_t>(h) | (static_cast<uint32_t>(l) << 16);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

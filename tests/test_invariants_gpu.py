@@ -36,10 +36,13 @@ def _token_slot(wl, s, t):
     return int(wl.block_tables[s, t // B]), t % B
 
 
-@pytest.mark.parametrize("kv", [W.BF16, W.FP8_E4M3])
+@pytest.mark.parametrize("kv", [W.BF16, W.FP8_E4M3, "fp8_compute"])
 @pytest.mark.parametrize("D,B", [(128, 16), (64, 32), (128, 32)])
 @pytest.mark.parametrize("pp", [0, 2])
 def test_one_hot_probe_bit_exact(kv, D, B, pp):
+    f8c = kv == "fp8_compute"
+    if f8c:
+        kv = W.FP8_E4M3
     lens = (3 * B + 5, B, 1, 7 * B - 1)
     cfg = _cfg(D=D, B=B, G=4, kv=kv, lens=lens)
     wl = W.make_workload(cfg, DEV, seq_lens=list(lens))
@@ -59,7 +62,13 @@ def test_one_hot_probe_bit_exact(kv, D, B, pp):
             pb, o = _token_slot(wl, s, t_star)
             old = kc[pb, :, 0, o, 0].clone()
             kc[pb, :, 0, o, 0] = one if kv == W.BF16 else torch.full_like(old, one)
-            out = run_gpu(wl, partition_pages=pp)
+            if f8c:
+                out = torch.empty_like(wl.query)
+                pa.decode(out, wl.query, kc, wl.value_cache, cfg.num_kv_heads, cfg.scale,
+                          wl.block_tables, wl.seq_lens, B, cfg.max_seq_len, kv, wl.k_scale,
+                          wl.v_scale, partition_pages=pp, fp8_compute=True)
+            else:
+                out = run_gpu(wl, partition_pages=pp)
             torch.cuda.synchronize()
             for g in range(cfg.num_kv_heads):
                 v = wl.value_cache[pb, g, :, o]

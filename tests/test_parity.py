@@ -191,3 +191,54 @@ def test_alibi(idx, partition_pages):
     plain = run_gpu(wl)
     torch.cuda.synchronize()
     assert (plain.float() - out.float()).abs().max().item() > 0.05
+
+
+# ---------------------------------------------------------- FP8 tensor-core compute
+def _decode_fp8_compute(wl, partition_pages=0):
+    c = wl.cfg
+    out = torch.empty_like(wl.query)
+    pa.decode(out, wl.query, wl.key_cache, wl.value_cache, c.num_kv_heads, c.scale,
+              wl.block_tables, wl.seq_lens, c.block_size, c.max_seq_len, c.kv_dtype,
+              wl.k_scale, wl.v_scale, partition_pages=partition_pages, fp8_compute=True)
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("D,B,G", list(itertools.product([64, 128], [16, 32], [1, 4, 8, 16])),
+                         ids=lambda v: str(v))
+def test_fp8_compute_shapes(D, B, G):
+    Hk = 2
+    lens = [1, B - 1, B, B + 1, 3 * B + 5, 17 * B - 1, 40 * B + 3]
+    cfg = W.PagedConfig(f"fp8 compute D={D} B={B} G={G}", num_seqs=len(lens), num_heads=Hk * G,
+                        num_kv_heads=Hk, head_size=D, block_size=B,
+                        num_blocks=sum(-(-t // B) for t in lens) + 9, seq_len_lo=1,
+                        seq_len_hi=max(lens), kv_dtype=W.FP8_E4M3, k_scale=0.05, v_scale=0.04,
+                        seed=777 + D + B + G)
+    wl = W.make_workload(cfg, DEV, seq_lens=lens)
+    ref = run_oracle(wl)
+    for pp in (0, 4):
+        compare(_decode_fp8_compute(wl, pp), ref, W.FP8_E4M3, f"{cfg.name} pp={pp}")
+
+
+def test_fp8_compute_reduced_and_full_size():
+    cfg = REDUCED[4]
+    wl = W.make_workload(cfg, DEV)
+    compare(_decode_fp8_compute(wl), run_oracle(wl), cfg.kv_dtype, "fp8 compute reduced cfg4")
+    cfg = W.CONFIGS[4]
+    wl = W.make_workload(cfg, DEV)
+    out = _decode_fp8_compute(wl)
+    assert torch.isfinite(out.float()).all()
+    pairs = sample_pairs(cfg, 24, seed=44)
+    ref = run_oracle_sampled(wl, pairs)
+    compare(torch.stack([out[s, h] for s, h in pairs]), ref, cfg.kv_dtype, "fp8 compute full cfg4")
+    del wl, out
+    torch.cuda.empty_cache()
+
+
+def test_fp8_compute_needs_fp8_cache():
+    cfg = REDUCED[1]
+    wl = W.make_workload(cfg, DEV)
+    with pytest.raises(pa.PagedAttentionError):
+        pa.decode(torch.empty_like(wl.query), wl.query, wl.key_cache, wl.value_cache,
+                  cfg.num_kv_heads, cfg.scale, wl.block_tables, wl.seq_lens, cfg.block_size,
+                  cfg.max_seq_len, fp8_compute=True)
