@@ -114,6 +114,13 @@ typedef enum pa_kv_dtype {
  *      the softmax weights (x 256) are each carried as a hi + lo pair of e4m3
  *      codes, about 2^-8 relative together, so accuracy stays near the f16
  *      path's.  Requires kv_dtype = PA_KV_FP8_E4M3.
+ *  test_stall_copies: for testing the failure path only.  Non-zero makes every
+ *      page's completion barrier wait for 16 bytes that no copy delivers and
+ *      cuts each wait to ~20 ms, so the kernel takes its give-up path: it lets
+ *      the copies it issued land, sets PA_DEV_WAIT_TIMEOUT and returns, with
+ *      the output undefined and the context usable.  Every real copy still
+ *      completes; nothing faults or hangs.  Use on small problems (each warp
+ *      spends ~20 ms per stage).
  */
 typedef struct pa_options {
     int partition_pages;
@@ -122,6 +129,7 @@ typedef struct pa_options {
     int shared_prefix_blocks;
     const float* alibi_slopes;
     int fp8_compute;
+    int test_stall_copies;
 } pa_options;
 
 /* What pa_decode will launch for a given problem. */

@@ -50,7 +50,8 @@ class PagedAttentionError(RuntimeError):
 class Options(ctypes.Structure):
     _fields_ = [("partition_pages", ctypes.c_int), ("num_sms", ctypes.c_int),
                 ("stages", ctypes.c_int), ("shared_prefix_blocks", ctypes.c_int),
-                ("alibi_slopes", ctypes.c_void_p), ("fp8_compute", ctypes.c_int)]
+                ("alibi_slopes", ctypes.c_void_p), ("fp8_compute", ctypes.c_int),
+                ("test_stall_copies", ctypes.c_int)]
 
 
 class Plan(ctypes.Structure):
@@ -144,12 +145,13 @@ def _check(rc: int):
 
 
 def _opts(partition_pages=0, num_sms=0, stages=0, shared_prefix_blocks=0, alibi_ptr=None,
-          fp8_compute=False):
+          fp8_compute=False, test_stall_copies=False):
     if not partition_pages and not num_sms and not stages and not shared_prefix_blocks \
-            and not alibi_ptr and not fp8_compute:
+            and not alibi_ptr and not fp8_compute and not test_stall_copies:
         return None
     return ctypes.byref(Options(int(partition_pages), int(num_sms), int(stages),
-                                int(shared_prefix_blocks), alibi_ptr, int(bool(fp8_compute))))
+                                int(shared_prefix_blocks), alibi_ptr, int(bool(fp8_compute)),
+                                int(bool(test_stall_copies))))
 
 
 def kv_dtype_code(kv_dtype) -> int:
@@ -213,7 +215,7 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
            seq_lens, block_size: int, max_seq_len: int, kv_dtype="bf16", k_scale=None,
            v_scale=None, workspace_tensor=None, partition_pages: int = 0, stream=None,
            stages: int = 0, shared_prefix_blocks: int = 0, alibi_slopes=None,
-           fp8_compute: bool = False):
+           fp8_compute: bool = False, test_stall_copies: bool = False):
     """Paged decode attention into ``out`` (bf16 [num_seqs, num_heads, head_size]).
 
     key_cache: [num_blocks, num_kv_heads, head_size/x, block_size, x];
@@ -267,7 +269,7 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
                             workspace_tensor.numel() * workspace_tensor.element_size(),
                             st.cuda_stream,
                             _opts(partition_pages, 0, stages, shared_prefix_blocks, alibi,
-                                  fp8_compute))
+                                  fp8_compute, test_stall_copies))
     _check(rc)
     return out
 

@@ -18,6 +18,8 @@ constexpr size_t kSmemPerSm = 228 * 1024;
 constexpr size_t kSmemReservedPerCta = 1024;
 constexpr size_t kMaxSmemPerCta = 227 * 1024;  // opt-in limit of sm_100
 constexpr int kMinPartitionPages = 16;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // a page copy's wait bound
+constexpr unsigned long long kTestWaitLimitNs = 20000000ull;  // with test_stall_copies
 constexpr long long kLongPartitionPages = 256;
 constexpr int kDefaultStages = 2;
 constexpr int kMaxShortStages = 4;
@@ -393,6 +395,12 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
     p.prefix_units = static_cast<long long>(num_kv_heads) * pl.prefix_groups * pl.prefix_partitions;
     p.P_total = p_total;
     p.alibi = opts ? opts->alibi_slopes : nullptr;
+    p.stall_tx_bytes = 0;
+    p.wait_limit_ns = kWaitLimitNs;
+    if (opts && opts->test_stall_copies) {
+        p.stall_tx_bytes = 16;
+        p.wait_limit_ns = kTestWaitLimitNs;
+    }
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool f8mma = opts && opts->fp8_compute && kv_dtype == PA_KV_FP8_E4M3;

@@ -77,6 +77,10 @@ struct DecodeParams {
     long long prefix_units;   // Hk * prefix_groups * prefix_parts
     int P_total;              // partial slots per (seq, q head): prefix_parts + P
     const float* alibi;       // [Hq] ALiBi slopes, or nullptr
+    // Failure-path test hook: each page's mbarrier expects stall_tx_bytes more
+    // than its copies deliver, so every wait runs out after wait_limit_ns.
+    int stall_tx_bytes;
+    unsigned long long wait_limit_ns;
 };
 
 // Bytes of shared memory the final merge needs (it overlays the page stages).
@@ -273,7 +277,7 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
             if (ok) {
                 const size_t off = static_cast<size_t>(pb) * block_stride + head_off;
                 const uint32_t dst = wstage0 + static_cast<uint32_t>(stage * STAGE);
-                mbar_arrive_expect_tx(bar, STAGE);
+                mbar_arrive_expect_tx(bar, STAGE + p.stall_tx_bytes);
                 bulk_copy_g2s(dst, p.kc + off, PAGE, bar);
                 bulk_copy_g2s(dst + PAGE, p.vc + off, PAGE, bar);
             } else {
@@ -653,7 +657,7 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
     int stage = 0;
     uint32_t phase = 0;
     for (; k < n_my; ++k) {
-        const bool landed = mbar_wait_bounded(bar0 + 8 * stage, phase);
+        const bool landed = mbar_wait_bounded(bar0 + 8 * stage, phase, p.wait_limit_ns);
         if (!__all_sync(kFull, landed)) {
             timed_out = true;
             break;
@@ -679,7 +683,7 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
         // shared memory can be handed to anyone else, then report.
         const int last = min(n_my, k + NS);
         for (int i = k; i < last; ++i) {
-            (void)mbar_wait_bounded(bar0 + 8 * stage, phase);
+            (void)mbar_wait_bounded(bar0 + 8 * stage, phase, p.wait_limit_ns);
             if (++stage == NS) {
                 stage = 0;
                 phase ^= 1u;

@@ -51,14 +51,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait for the phase with the given parity, giving up after ~2 s of device
-// time or 2^26 polls, whichever comes first.  Returns false on give-up.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+// Wait for the phase with the given parity, giving up after limit_ns of
+// device time or 2^26 polls, whichever comes first.  Returns false on give-up.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  uint64_t limit_ns = 2000000000ull) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 0; it < (1u << 26); ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 63u && global_timer_ns() - t0 > 2000000000ull) return false;
+        if ((it & 63u) == 63u && global_timer_ns() - t0 > limit_ns) return false;
     }
     return false;
 }

@@ -61,7 +61,7 @@ def _decode(L, **over):
                 num_heads=8, num_kv_heads=2, head_size=128, scale=0.088, block_tables=0x50000,
                 max_blocks_per_seq=4, seq_lens=0x60000, block_size=16, max_seq_len=64,
                 num_blocks=64, kv_dtype=0, k_scale=None, v_scale=None, workspace=0x70000,
-                workspace_bytes=1 << 20, stream=None, opts=ctypes.byref(pa.Options(0, 148, 0, 0, None, 0)))
+                workspace_bytes=1 << 20, stream=None, opts=ctypes.byref(pa.Options(0, 148, 0, 0, None, 0, 0)))
     args.update(over)
     return L.pa_decode_ex(*args.values())
 

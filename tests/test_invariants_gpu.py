@@ -223,3 +223,24 @@ def test_one_hot_probe_bit_exact_with_shared_prefix(kv, B):
                     (s, t_star, h)
         for pb, o, old in reversed(marks):  # shared slots appear once per sequence
             kc[pb, :, 0, o, 0] = old
+
+
+def test_wait_give_up_path_sets_status_and_leaves_context_usable():
+    """With test_stall_copies every page barrier waits for bytes no copy sends
+    (the copies themselves all land) and each wait gives up after ~20 ms: the
+    kernel must drain, flag PA_DEV_WAIT_TIMEOUT and return; afterwards a normal
+    decode on the same context is correct."""
+    lens = [80]
+    cfg = _cfg(lens=lens, G=4, Hk=1)
+    wl = W.make_workload(cfg, DEV, seq_lens=lens)
+    ws = torch.zeros(pa.workspace_size(1, 4, 1, 128, 16, 80), dtype=torch.uint8, device=DEV)
+    out = torch.empty_like(wl.query)
+    pa.decode(out, wl.query, wl.key_cache, wl.value_cache, 1, cfg.scale, wl.block_tables,
+              wl.seq_lens, 16, 80, workspace_tensor=ws, test_stall_copies=True)
+    torch.cuda.synchronize()
+    assert pa.read_status(ws, clear=True) & pa.PA_DEV_WAIT_TIMEOUT
+    assert torch.isfinite(out.float()).all()
+    good = run_gpu(wl, ws=ws)
+    torch.cuda.synchronize()
+    assert pa.read_status(ws) == 0
+    compare(good, run_oracle(wl), cfg.kv_dtype, "after a give-up")
