@@ -17,6 +17,7 @@ constexpr int kVersion = 10000;  // 1.0.0
 constexpr size_t kSmemPerSm = 228 * 1024;
 constexpr size_t kSmemReservedPerCta = 1024;
 constexpr size_t kMaxSmemPerCta = 227 * 1024;  // opt-in limit of sm_100
+constexpr size_t kStaticSmemReserve = 256;      // the kernel's own __shared__ variables
 constexpr int kMinPartitionPages = 16;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // a page copy's wait bound
 constexpr unsigned long long kTestWaitLimitNs = 20000000ull;  // with test_stall_copies
@@ -113,7 +114,7 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
     const size_t mb = merge_bytes(head_size, cascade ? 16 : num_heads / num_kv_heads, W);
     if (stage_area < mb) stage_area = mb;
     size_t smem = stage_area + static_cast<size_t>(W) * ns * 8;
-    if (smem > kMaxSmemPerCta)
+    if (smem > kMaxSmemPerCta - kStaticSmemReserve)
         return fail(PA_ERR_INVALID_ARG, "%s", "too many stages for shared memory");
     long long per_sm = static_cast<long long>(kSmemPerSm / (smem + kSmemReservedPerCta));
     if (per_sm < 1) per_sm = 1;
@@ -204,9 +205,17 @@ cudaError_t ensure_smem(K kernel, std::atomic<int>* done) {
     if (e != cudaSuccess) return e;
     const bool cached = dev >= 0 && dev < kMaxDevices;
     if (cached && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kMaxSmemPerCta));
-    if (e == cudaSuccess && cached) done[dev].store(1, std::memory_order_release);
+    // The opt-in limit covers static and dynamic shared memory together.
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kernel);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kMaxSmemPerCta - fa.sharedSizeBytes));
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();  // do not leave the error for an unrelated later call
+        return e;
+    }
+    if (cached) done[dev].store(1, std::memory_order_release);
     return e;
 }
 
@@ -216,7 +225,7 @@ cudaError_t launch_decode(const pa::DecodeParams& p, long long grid, size_t smem
     static std::atomic<int> done[kMaxDevices];
     constexpr int W = pa::decode_warps<D, B, FP8>();
     auto kern = pa::pa_decode_kernel<D, B, FP8, NH, W, F8MMA>;
-    if (smem > kMaxSmemPerCta) return cudaErrorInvalidValue;
+    if (smem > kMaxSmemPerCta - kStaticSmemReserve) return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem(kern, done);
     if (e != cudaSuccess) return e;
     kern<<<static_cast<unsigned>(grid), W * 32, smem, st>>>(p);

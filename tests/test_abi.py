@@ -147,7 +147,7 @@ def test_every_plan_fits_shared_memory():
                     for T in (1, 15, 17, 100, 1000, 20000, 131072):
                         for pp in (0, 1, 2, 3, 5, 16, 64):
                             p = pa.plan(4, 2 * G, 2, D, B, T, kv, partition_pages=pp, num_sms=148)
-                            assert p["smem_bytes"] <= 227 * 1024, (D, B, kv, G, T, pp)
+                            assert p["smem_bytes"] <= 227 * 1024 - 256, (D, B, kv, G, T, pp)
 
 
 def test_alibi_with_shared_prefix_is_refused(L):
