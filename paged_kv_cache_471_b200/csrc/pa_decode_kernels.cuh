@@ -399,8 +399,10 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
 
     // One landed page: S = Q K^T, online softmax, O^T += V^T P^T.  FULL pages
     // (every slot a token) skip all masking.
-    auto page = [&](auto full_tag, const uint32_t kbase, const int valid, const int pos0) {
+    auto page = [&](auto full_tag, auto alibi_tag, const uint32_t kbase, const int valid,
+                    const int pos0) {
         constexpr bool FULL = decltype(full_tag)::value;
+        constexpr bool ALIBI = decltype(alibi_tag)::value;
         const uint32_t vbase = kbase + PAGE;
 
         // ---------------- S = Q K^T  (rows: heads, cols: tokens)
@@ -470,7 +472,7 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     float x = sc[nt][2 * r + e] * qk_mul;
-                    if (has_alibi)
+                    if constexpr (ALIBI)
                         x = fmaf(slope2[r], static_cast<float>(pos0 + 8 * nt + 2 * cq + e), x);
                     if constexpr (!FULL) {
                         if (8 * nt + 2 * cq + e >= valid) x = -INFINITY;
@@ -666,10 +668,17 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
         const int valid = ((valid_mask >> stage) & 1u) ? min(B, T - jg * B) : 0;
         const uint32_t kbase = wstage0 + static_cast<uint32_t>(stage * STAGE);
         const int pos0 = jg * B - (T - 1);  // ALiBi position of the page's first slot
-        if (valid == B)
-            page(std::true_type{}, kbase, valid, pos0);
-        else
-            page(std::false_type{}, kbase, valid, pos0);
+        if (!has_alibi) {
+            if (valid == B)
+                page(std::true_type{}, std::false_type{}, kbase, valid, pos0);
+            else
+                page(std::false_type{}, std::false_type{}, kbase, valid, pos0);
+        } else {
+            if (valid == B)
+                page(std::true_type{}, std::true_type{}, kbase, valid, pos0);
+            else
+                page(std::false_type{}, std::true_type{}, kbase, valid, pos0);
+        }
         __syncwarp();
         if (k + NS < n_my) issue(k + NS);
         if (++stage == NS) {
