@@ -19,6 +19,7 @@ constexpr size_t kSmemReservedPerCta = 1024;
 constexpr size_t kMaxSmemPerCta = 227 * 1024;  // opt-in limit of sm_100
 constexpr size_t kStaticSmemReserve = 256;      // the kernel's own __shared__ variables
 constexpr int kMinPartitionPages = 16;
+constexpr int kMaxRankedSeqs = 256;  // batches ranked by length on the device
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // a page copy's wait bound
 constexpr unsigned long long kTestWaitLimitNs = 20000000ull;  // with test_stall_copies
 constexpr long long kLongPartitionPages = 256;
@@ -128,6 +129,11 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         pp = opts->partition_pages;
     } else if (pages_max == 0 || units == 0) {
         pp = 1;
+    } else if (units >= slots && num_seqs <= kMaxRankedSeqs) {
+        // Enough (sequence, kv head) units to fill every CTA slot: no split.
+        // CTAs take sequences longest first (ranked on the device), which
+        // bounds the last wave's tail without partitions (measured on B200).
+        pp = pages_max;
     } else {
         // Split count:
         //  * enough partitions to balance uneven lengths: about four partitions
@@ -404,6 +410,7 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
     p.prefix_units = static_cast<long long>(num_kv_heads) * pl.prefix_groups * pl.prefix_partitions;
     p.P_total = p_total;
     p.alibi = opts ? opts->alibi_slopes : nullptr;
+    p.longest_first = (num_seqs > 1 && num_seqs <= kMaxRankedSeqs) ? 1 : 0;
     p.stall_tx_bytes = 0;
     p.wait_limit_ns = kWaitLimitNs;
     if (opts && opts->test_stall_copies) {

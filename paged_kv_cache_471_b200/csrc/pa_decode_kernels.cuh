@@ -81,6 +81,9 @@ struct DecodeParams {
     // than its copies deliver, so every wait runs out after wait_limit_ns.
     int stall_tx_bytes;
     unsigned long long wait_limit_ns;
+    // Longest first: per-sequence CTAs take sequences in order of decreasing
+    // length (ties by index), ranked by every CTA from seq_lens (num_seqs <= 256).
+    int longest_first;
 };
 
 // Bytes of shared memory the final merge needs (it overlays the page stages).
@@ -133,6 +136,37 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
         kvh = static_cast<int>(u % p.Hk);
         s = static_cast<int>((u / p.Hk) % p.S);
         part = static_cast<int>(u / ((long long)p.Hk * p.S));
+        if (p.longest_first) {
+            // The unit's sequence index is a rank: find the sequence with that
+            // rank among all lengths, longest first, so that the longest work
+            // starts first and the last wave of CTAs is short.  Uses the start
+            // of shared memory, which holds no page yet.
+            int* lens = reinterpret_cast<int*>(smem);
+            const int cap = p.max_blocks * B;
+            const int len0 = max(0, min(__ldg(p.seq_lens), cap));
+            int differs = 0;
+            for (int i = threadIdx.x; i < p.S; i += W * 32) {
+                lens[i] = max(0, min(__ldg(p.seq_lens + i), cap));
+                differs |= lens[i] != len0;
+            }
+            // Equal lengths (a block-wide vote): index order is already longest
+            // first.  Otherwise every sequence's rank is counted and the one
+            // whose rank is the unit's index is picked.
+            if (__syncthreads_or(differs)) {
+                for (int i = threadIdx.x; i < p.S; i += W * 32) {
+                    const int v = lens[i];
+                    int rank = 0;
+                    for (int j = 0; j < p.S; ++j) {
+                        const int w2 = lens[j];
+                        rank += (w2 > v) | ((w2 == v) & (j < i));
+                    }
+                    if (rank == s) lens[p.S] = i;
+                }
+                __syncthreads();
+                s = lens[p.S];
+            }
+            __syncthreads();  // the scratch is page memory from here on
+        }
     }
     const bool cascade = p.prefix_pages > 0;
     const int pg0 = pre ? 0 : p.prefix_pages;  // first page of this unit's page range

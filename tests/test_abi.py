@@ -112,7 +112,7 @@ def test_planner_on_the_five_workloads():
     p1, p2, p3, p4, p5 = (_plan(i) for i in range(1, 6))
     assert p1["num_partitions"] == 1 and p1["partition_pages"] == 16
     assert p2["num_partitions"] == 1 and p2["grid_ctas"] == 64 * 32
-    assert p3["num_partitions"] >= 2  # variable lengths: bound the last wave's tail
+    assert p3["num_partitions"] == 1  # enough units to fill the GPU; longest-first order
     assert p4["num_partitions"] == 1 and p4["grid_ctas"] == 256 * 8
     assert p5["num_partitions"] >= 4  # 64 (seq, kv head) units cannot fill 148 SMs
     for p in (p1, p2, p3, p4, p5):
