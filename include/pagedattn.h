@@ -113,7 +113,10 @@ typedef enum pa_kv_dtype {
  *      into the products unchanged; the query (scaled by a power of two) and
  *      the softmax weights (x 256) are each carried as a hi + lo pair of e4m3
  *      codes, about 2^-8 relative together, so accuracy stays near the f16
- *      path's.  Requires kv_dtype = PA_KV_FP8_E4M3.
+ *      path's.  The query's power of two is shared by the rows one warp
+ *      handles: components more than about 2^9 below their largest |q| keep
+ *      only an absolute error of about 2^-17 max|q| (the e4m3 subnormal
+ *      floor).  Requires kv_dtype = PA_KV_FP8_E4M3.
  *  test_stall_copies: for testing the failure path only.  Non-zero makes every
  *      page's completion barrier wait for 16 bytes that no copy delivers and
  *      cuts each wait to ~20 ms, so the kernel takes its give-up path: it lets
