@@ -129,10 +129,13 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         pp = opts->partition_pages;
     } else if (pages_max == 0 || units == 0) {
         pp = 1;
-    } else if (units >= slots && num_seqs <= kMaxRankedSeqs) {
-        // Enough (sequence, kv head) units to fill every CTA slot: no split.
-        // CTAs take sequences longest first (ranked on the device), which
-        // bounds the last wave's tail without partitions (measured on B200).
+    } else if (units >= 2 * slots && num_seqs <= kMaxRankedSeqs) {
+        // At least two waves of (sequence, kv head) units: no split.  CTAs
+        // take sequences longest first (ranked on the device), which keeps
+        // the last wave short for mixed lengths.  Between one and two waves,
+        // equal lengths would leave a last wave of a few full-length units
+        // running alone, so those batches are split (measured on B200: 64
+        // sequences x 8 kv heads x 16384 tokens ran 12% slower unsplit).
         pp = pages_max;
     } else {
         // Split count:

@@ -112,7 +112,7 @@ def test_planner_on_the_five_workloads():
     p1, p2, p3, p4, p5 = (_plan(i) for i in range(1, 6))
     assert p1["num_partitions"] == 1 and p1["partition_pages"] == 16
     assert p2["num_partitions"] == 1 and p2["grid_ctas"] == 64 * 32
-    assert p3["num_partitions"] == 1  # enough units to fill the GPU; longest-first order
+    assert p3["num_partitions"] == 1  # two waves of units; longest-first order
     assert p4["num_partitions"] == 1 and p4["grid_ctas"] == 256 * 8
     assert p5["num_partitions"] >= 4  # 64 (seq, kv head) units cannot fill 148 SMs
     for p in (p1, p2, p3, p4, p5):
@@ -123,6 +123,16 @@ def test_planner_on_the_five_workloads():
     ws = pa.workspace_size(c5.num_seqs, c5.num_heads, c5.num_kv_heads, 128, 32, c5.max_seq_len,
                            num_sms=148)
     assert ws >= 256 + 8 * 32 * p5["num_partitions"] * 130 * 4
+
+
+def test_planner_splits_between_one_and_two_waves():
+    # 64 sequences x 8 kv heads = 512 units for 148 x 3 CTA slots: unsplit, a
+    # last wave of 68 full-length units would run alone.
+    p = pa.plan(64, 32, 8, 128, 16, 16384, "bf16", num_sms=148)
+    assert p["num_partitions"] >= 2
+    # 1024 units (more than two waves) are not split.
+    p = pa.plan(128, 32, 8, 128, 16, 16384, "bf16", num_sms=148)
+    assert p["num_partitions"] == 1
 
 
 def test_forced_partitions():
