@@ -193,9 +193,9 @@ def workload_config(idx: int, num_seqs: int = 0):
     """The named workload, or the same shape with fewer sequences and a pool
     sized to them (used for small profiler captures)."""
     from paged_kv_cache_471_b200 import workloads as W
-    if num_seqs and num_seqs < W.CONFIGS[idx].num_seqs:
+    if num_seqs and num_seqs < W.WORKLOADS[idx].num_seqs:
         return W.reduced(idx, num_seqs=num_seqs)
-    return W.CONFIGS[idx]
+    return W.WORKLOADS[idx]
 
 
 def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, num_seqs=0,
@@ -515,7 +515,7 @@ def run_copy_blocks(args, device):
 
     import paged_kv_cache_471_b200 as pa
     from paged_kv_cache_471_b200 import workloads as W
-    cfg = W.CONFIGS[2]
+    cfg = W.WORKLOADS[2]
     kc = torch.empty(cfg.key_cache_shape(), dtype=torch.bfloat16, device=device)
     vc = torch.empty(cfg.value_cache_shape(), dtype=torch.bfloat16, device=device)
     kc.view(torch.int16).fill_(1)
@@ -555,7 +555,7 @@ def run_reference(args):
         return 0
     from paged_kv_cache_471_b200 import workloads as W
     idx = int(args.config) if args.config not in ("all",) else 2
-    cfg = W.CONFIGS[idx]
+    cfg = W.WORKLOADS[idx]
     dev = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
     wl = W.make_workload(cfg, dev) if dev.type == "cuda" else W.make_workload(
         W.reduced(idx, num_seqs=2), dev)
@@ -623,15 +623,15 @@ def main(argv=None):
         if rank == 0:
             run_copy_blocks(args, device)
         return 0
-    configs = [1, 2, 3, 4, 5] if args.config == "all" else [int(args.config)]
-    for idx in configs:
+    cfg_ids = [1, 2, 3, 4, 5] if args.config == "all" else [int(args.config)]
+    for idx in cfg_ids:
         r = time_gpu(idx, args.steps, args.warmup, device, want_e2e=not args.no_e2e, rank=rank,
                      num_seqs=args.num_seqs, cascade=not args.no_cascade, alibi=args.alibi)
         r["step_ms"] = reduce_max(r["step_ms"], device)
         if "e2e_ms" in r:
             r["e2e_ms"] = reduce_max(r["e2e_ms"], device)
         cpu = None
-        if rank == 0 and ws == 1 and not args.no_cpu and idx == configs[0]:
+        if rank == 0 and ws == 1 and not args.no_cpu and idx == cfg_ids[0]:
             cpu = cpu_sample(idx, r["wl"])
         if rank == 0:
             print(json.dumps(result_line(idx, r, ws, args.steps, args.warmup, cpu)), flush=True)

@@ -99,7 +99,7 @@ class PagedConfig:
 
 
 # The five workloads of the decode benchmark (sizes as stated for each).
-CONFIGS = {
+WORKLOADS = {
     1: PagedConfig("tiny MHA decode: 4 seqs, 8/8 heads, D=64, B=16, T~U[1,256], bf16",
                    num_seqs=4, num_heads=8, num_kv_heads=8, head_size=64, block_size=16,
                    num_blocks=128, seq_len_lo=1, seq_len_hi=256, seed=1001),
@@ -125,8 +125,8 @@ def reduced(idx: int, num_seqs: Optional[int] = None, seq_len_hi: Optional[int] 
             seq_len_lo: Optional[int] = None, num_blocks: Optional[int] = None,
             shared_prefix_blocks: Optional[int] = None) -> PagedConfig:
     """A smaller batch with the same heads, head size, block size, dtype and
-    length mix as CONFIGS[idx], small enough for the oracle to finish in seconds."""
-    c = CONFIGS[idx]
+    length mix as WORKLOADS[idx], small enough for the oracle to finish in seconds."""
+    c = WORKLOADS[idx]
     hi = seq_len_hi if seq_len_hi is not None else c.seq_len_hi
     lo = seq_len_lo if seq_len_lo is not None else min(c.seq_len_lo, hi)
     S = num_seqs if num_seqs is not None else c.num_seqs

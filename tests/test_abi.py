@@ -103,7 +103,7 @@ def test_workspace_size_header_only_without_split():
 
 
 def _plan(idx, **kw):
-    c = W.CONFIGS[idx]
+    c = W.WORKLOADS[idx]
     return pa.plan(c.num_seqs, c.num_heads, c.num_kv_heads, c.head_size, c.block_size,
                    c.max_seq_len, c.kv_dtype, num_sms=148, **kw)
 
@@ -118,7 +118,7 @@ def test_planner_on_the_five_workloads():
     for p in (p1, p2, p3, p4, p5):
         assert p["smem_bytes"] <= 227 * 1024 and 2 <= p["stages"] <= 8
         P, PP = p["num_partitions"], p["partition_pages"]
-    c5 = W.CONFIGS[5]
+    c5 = W.WORKLOADS[5]
     assert p5["num_partitions"] * p5["partition_pages"] >= c5.max_blocks_per_seq
     ws = pa.workspace_size(c5.num_seqs, c5.num_heads, c5.num_kv_heads, 128, 32, c5.max_seq_len,
                            num_sms=148)

@@ -23,7 +23,7 @@ def _lib():
 # dtype and length mix; sizes the oracle finishes in seconds, still many
 # pages per (sequence, kv head) and ragged last blocks.
 REDUCED = {
-    1: W.CONFIGS[1],  # already tiny
+    1: W.WORKLOADS[1],  # already tiny
     2: W.reduced(2, num_seqs=3, seq_len_hi=1000, seq_len_lo=700),
     3: W.reduced(3, num_seqs=6, seq_len_hi=2100, seq_len_lo=100),
     4: W.reduced(4, num_seqs=4, seq_len_hi=1500, seq_len_lo=900),
@@ -68,7 +68,7 @@ def test_shapes(D, B, G, kv):
 def test_full_size_sampled(idx):
     """Full workload in the launch configuration the bench times; sampled rows
     against the oracle, plus whole-output sanity (finite, no poison)."""
-    cfg = W.CONFIGS[idx]
+    cfg = W.WORKLOADS[idx]
     wl = W.make_workload(cfg, DEV)
     out = run_gpu(wl)
     torch.cuda.synchronize()
@@ -119,7 +119,7 @@ def test_shared_prefix_cascade(name, partition_pages):
 
 
 def test_shared_prefix_full_size_sampled():
-    cfg = W.CONFIGS[5]
+    cfg = W.WORKLOADS[5]
     wl = W.make_workload(cfg, DEV)
     ws = torch.zeros(pa.workspace_size(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads,
                                        cfg.head_size, cfg.block_size, cfg.max_seq_len,
@@ -224,7 +224,7 @@ def test_fp8_compute_reduced_and_full_size():
     cfg = REDUCED[4]
     wl = W.make_workload(cfg, DEV)
     compare(_decode_fp8_compute(wl), run_oracle(wl), cfg.kv_dtype, "fp8 compute reduced cfg4")
-    cfg = W.CONFIGS[4]
+    cfg = W.WORKLOADS[4]
     wl = W.make_workload(cfg, DEV)
     out = _decode_fp8_compute(wl)
     assert torch.isfinite(out.float()).all()

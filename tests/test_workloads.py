@@ -6,7 +6,7 @@ from paged_kv_cache_471_b200 import workloads as W
 
 
 def test_configs_match_stated_sizes():
-    c = W.CONFIGS
+    c = W.WORKLOADS
     assert (c[1].num_seqs, c[1].num_heads, c[1].num_kv_heads, c[1].head_size,
             c[1].block_size, c[1].num_blocks) == (4, 8, 8, 64, 16, 128)
     assert (c[2].num_seqs, c[2].num_heads, c[2].head_size, c[2].seq_len_hi) == (64, 32, 128, 4096)
@@ -18,7 +18,7 @@ def test_configs_match_stated_sizes():
 
 def test_tables_deterministic_and_distinct():
     for idx in (1, 3):
-        cfg = W.CONFIGS[idx]
+        cfg = W.WORKLOADS[idx]
         a = W.draw_tables(cfg)
         b = W.draw_tables(cfg)
         assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
@@ -32,14 +32,14 @@ def test_tables_deterministic_and_distinct():
 
 
 def test_full_pool_permutation_config4():
-    cfg = W.CONFIGS[4]
+    cfg = W.WORKLOADS[4]
     sl, bt = W.draw_tables(cfg)
     assert bt.shape == (256, 1024)
     assert torch.equal(bt.flatten().sort().values, torch.arange(262144, dtype=torch.int32))
 
 
 def test_shared_prefix_config5():
-    cfg = W.CONFIGS[5]
+    cfg = W.WORKLOADS[5]
     sl, bt = W.draw_tables(cfg)
     assert (bt[:, :1024] == bt[0:1, :1024]).all()
     rest = bt[:, 1024:]
