@@ -486,6 +486,9 @@ def result_line(idx, r, n_gpus, steps, warmup, cpu=None):
             "traffic": traffic_per_launch(idx),
             "kernel": KERNEL_NAME + (" + pa_combine_kernel" if r["launches_per_step"] > 1 else ""),
             "bytes_per_launch": r["alg_bytes"],
+            "launch_ms": {"mean": round(kern_avg, 5),
+                          "median": round(statistics.median(r["kern_ms"]), 5),
+                          "min": round(min(r["kern_ms"]), 5)},
         },
         "gpu_launches": steps * r["launches_per_step"],
         "clocks": r["clocks"],
