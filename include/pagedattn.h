@@ -27,6 +27,10 @@
  *  - Ownership: the caller allocates and owns every buffer.  pa_decode
  *    allocates nothing, never synchronises, and only enqueues work on the
  *    given stream (a cudaStream_t passed as void*; NULL = legacy default).
+ *    Kernels are launched with programmatic stream serialization and wait
+ *    for every grid ahead of them before touching memory, so stream order
+ *    holds for all they read and write; only their launch overlaps the
+ *    previous kernel's end.
  *  - Argument errors are returned synchronously, before any launch, and
  *    before any CUDA call.  pa_last_error_detail() then names the argument.
  *  - Launch failures return PA_ERR_CUDA.

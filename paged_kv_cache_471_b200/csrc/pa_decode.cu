@@ -228,6 +228,28 @@ cudaError_t ensure_smem(K kernel, std::atomic<int>* done) {
     return e;
 }
 
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the kernel ahead of it in the stream drains, which hides the launch
+// gap between back-to-back calls and between decode and combine.  Both
+// kernels wait (griddepcontrol.wait) before touching memory, so stream order
+// is kept for everything they read and write.
+template <typename Params>
+cudaError_t launch_pdl(void (*kern)(Params), unsigned grid, unsigned block, size_t smem,
+                       cudaStream_t st, const Params& p) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 template <int D, int B, bool FP8, int NH, bool F8MMA>
 cudaError_t launch_decode(const pa::DecodeParams& p, long long grid, size_t smem,
                           cudaStream_t st) {
@@ -237,8 +259,7 @@ cudaError_t launch_decode(const pa::DecodeParams& p, long long grid, size_t smem
     if (smem > kMaxSmemPerCta - kStaticSmemReserve) return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem(kern, done);
     if (e != cudaSuccess) return e;
-    kern<<<static_cast<unsigned>(grid), W * 32, smem, st>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(kern, static_cast<unsigned>(grid), W * 32, smem, st, p);
 }
 
 template <int D, int B, bool FP8, bool F8MMA>
@@ -268,11 +289,8 @@ cudaError_t launch_any(const pa::DecodeParams& p, int D, int B, bool fp8, bool f
 cudaError_t launch_combine(const pa::CombineParams& c, int D, cudaStream_t st) {
     const long long rows = static_cast<long long>(c.S) * c.Hq;
     const unsigned grid = static_cast<unsigned>((rows + pa::kWarps - 1) / pa::kWarps);
-    if (D == 64)
-        pa::pa_combine_kernel<64><<<grid, pa::kThreads, 0, st>>>(c);
-    else
-        pa::pa_combine_kernel<128><<<grid, pa::kThreads, 0, st>>>(c);
-    return cudaGetLastError();
+    return D == 64 ? launch_pdl(pa::pa_combine_kernel<64>, grid, pa::kThreads, 0, st, c)
+                   : launch_pdl(pa::pa_combine_kernel<128>, grid, pa::kThreads, 0, st, c);
 }
 
 // Scratch of pa_decode_noalloc: one fixed array per device, in the

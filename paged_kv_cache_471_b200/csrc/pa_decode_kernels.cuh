@@ -118,6 +118,13 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
 
     extern __shared__ __align__(128) uint8_t smem[];
 
+    // Launched with programmatic stream serialization: wait for the kernel
+    // ahead in the stream (which may write the inputs) before any access, and
+    // let the next kernel (the combine, or the next call) be scheduled now;
+    // it waits for this grid to complete in turn.
+    grid_dep_wait();
+    grid_dep_launch_dependents();
+
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int gq = lane >> 2;  // fragment row group
@@ -818,6 +825,8 @@ struct CombineParams {
 // Partitions with an empty sum are skipped.
 template <int D>
 __global__ void __launch_bounds__(kThreads) pa_combine_kernel(const CombineParams p) {
+    grid_dep_wait();  // the decode grid's partials are complete and visible
+    grid_dep_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long row = (long long)blockIdx.x * kWarps + warp;
     if (row >= (long long)p.S * p.Hq) return;

@@ -1,7 +1,7 @@
 // Thin inline-PTX wrappers for sm_100a used by the paged decode kernels:
-// mbarrier + 1-D bulk async copies (TMA engine, no tensor map, never
-// multicast), ldmatrix, warp-level bf16/f16 MMA with fp32 accumulation, and
-// e4m3 -> f16 conversion.
+// grid dependency control, mbarrier + 1-D bulk async copies (TMA engine, no
+// tensor map, never multicast), ldmatrix, warp-level bf16/f16 MMA with fp32
+// accumulation, and e4m3 -> f16 conversion.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -18,6 +18,22 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
+}
+
+// ---------------------------------------------------------------- launch order
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may be scheduled before the kernel ahead of it in the stream
+// has finished.  grid_dep_wait() returns once every grid this one depends on
+// has completed and its memory operations are visible (at once when there is
+// none), so nothing may be read or written before it.  After
+// grid_dep_launch_dependents() has run in every CTA (or the CTA has exited),
+// the next such kernel in the stream may be scheduled.
+__device__ __forceinline__ void grid_dep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_dep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- mbarrier

@@ -146,6 +146,67 @@ def test_non_default_stream():
     compare(out, run_oracle(wl), cfg.kv_dtype, "side stream")
 
 
+def _split_pair():
+    """Two batches of the same shape and different data, decoded with forced
+    partitions so that every call runs the decode and the combine kernel."""
+    lens = [1000, 37, 700, 2000]
+    wa = W.make_workload(_cfg(lens=lens, G=4, seed=301), DEV, seq_lens=lens)
+    wb = W.make_workload(_cfg(lens=lens, G=4, seed=302), DEV, seq_lens=lens)
+    return wa, wb
+
+
+def test_back_to_back_calls_sharing_a_workspace():
+    """Calls queued back to back on one stream with one workspace: each
+    kernel is launched while the one ahead of it drains (dependent launch) and
+    must still see the inputs and partials in stream order.  The outputs equal
+    those of calls separated by a device synchronisation, bit for bit."""
+    wa, wb = _split_pair()
+    c = wa.cfg
+    ws = torch.zeros(pa.workspace_size(c.num_seqs, c.num_heads, c.num_kv_heads, c.head_size,
+                                       c.block_size, c.max_seq_len, c.kv_dtype,
+                                       partition_pages=3), dtype=torch.uint8, device=DEV)
+    alone = []
+    for wl in (wa, wb):
+        alone.append(run_gpu(wl, partition_pages=3, ws=ws))
+        torch.cuda.synchronize()
+    outs = [torch.empty_like(wa.query) for _ in range(6)]
+    for i, o in enumerate(outs):
+        run_gpu((wa, wb)[i % 2], partition_pages=3, ws=ws, out=o)
+    torch.cuda.synchronize()
+    for i, o in enumerate(outs):
+        assert torch.equal(o, alone[i % 2]), f"call {i}"
+    compare(alone[1], run_oracle(wb), c.kv_dtype, "second batch")
+
+
+def test_calls_captured_in_a_cuda_graph():
+    """The same sequence of calls captured in a CUDA graph (the dependent
+    launches become graph edges) and replayed: bit-identical outputs."""
+    wa, wb = _split_pair()
+    c = wa.cfg
+    ws = torch.zeros(pa.workspace_size(c.num_seqs, c.num_heads, c.num_kv_heads, c.head_size,
+                                       c.block_size, c.max_seq_len, c.kv_dtype,
+                                       partition_pages=3), dtype=torch.uint8, device=DEV)
+    alone = [run_gpu(wl, partition_pages=3, ws=ws) for wl in (wa, wb)]
+    torch.cuda.synchronize()
+    outs = [torch.zeros_like(wa.query) for _ in range(4)]
+    st = torch.cuda.Stream(DEV)
+    st.wait_stream(torch.cuda.current_stream(DEV))
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(st):
+        with torch.cuda.graph(graph, stream=st):
+            for i, o in enumerate(outs):
+                run_gpu((wa, wb)[i % 2], partition_pages=3, ws=ws, out=o, stream=st)
+    torch.cuda.current_stream(DEV).wait_stream(st)
+    for _ in range(2):
+        for o in outs:
+            o.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        for i, o in enumerate(outs):
+            assert torch.equal(o, alone[i % 2]), f"graph call {i}"
+    del graph
+
+
 def test_bad_block_id_and_length_flags():
     lens = [100, 64]
     cfg = _cfg(lens=lens)
