@@ -252,24 +252,27 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
     if code == PA_KV_FP8_E4M3:
         ks = _ptr(k_scale, "k_scale", (torch.float32,), dev)
         vs = _ptr(v_scale, "v_scale", (torch.float32,), dev)
-    need = workspace_size(S, Hq, num_kv_heads, D, block_size, max_seq_len, code, partition_pages,
-                          shared_prefix_blocks=shared_prefix_blocks)
-    if workspace_tensor is None:
-        workspace_tensor = workspace(need, dev)
-    ws = _ptr(workspace_tensor, "workspace", None, dev)
     alibi = None
     if alibi_slopes is not None:
         if alibi_slopes.shape != (Hq,):
             raise ValueError("alibi_slopes must be [num_heads]")
         alibi = _ptr(alibi_slopes, "alibi_slopes", (torch.float32,), dev)
     st = stream if stream is not None else torch.cuda.current_stream(dev)
-    rc = lib().pa_decode_ex(*args_ptrs, S, Hq, int(num_kv_heads), D, float(scale), bt,
-                            block_tables.shape[1], sl, int(block_size), int(max_seq_len),
-                            int(num_blocks), code, ks, vs, ws,
-                            workspace_tensor.numel() * workspace_tensor.element_size(),
-                            st.cuda_stream,
-                            _opts(partition_pages, 0, stages, shared_prefix_blocks, alibi,
-                                  fp8_compute, test_stall_copies))
+    # The library plans for, and launches on, the current device: make it the
+    # tensors' device for the call.
+    with torch.cuda.device(dev):
+        need = workspace_size(S, Hq, num_kv_heads, D, block_size, max_seq_len, code,
+                              partition_pages, shared_prefix_blocks=shared_prefix_blocks)
+        if workspace_tensor is None:
+            workspace_tensor = workspace(need, dev)
+        ws = _ptr(workspace_tensor, "workspace", None, dev)
+        rc = lib().pa_decode_ex(*args_ptrs, S, Hq, int(num_kv_heads), D, float(scale), bt,
+                                block_tables.shape[1], sl, int(block_size), int(max_seq_len),
+                                int(num_blocks), code, ks, vs, ws,
+                                workspace_tensor.numel() * workspace_tensor.element_size(),
+                                st.cuda_stream,
+                                _opts(partition_pages, 0, stages, shared_prefix_blocks, alibi,
+                                      fp8_compute, test_stall_copies))
     _check(rc)
     return out
 
@@ -292,13 +295,15 @@ def decode_noalloc(out, query, key_cache, value_cache, num_kv_heads: int, scale:
         ks = _ptr(k_scale, "k_scale", (torch.float32,), dev)
         vs = _ptr(v_scale, "v_scale", (torch.float32,), dev)
     st = stream if stream is not None else torch.cuda.current_stream(dev)
-    rc = lib().pa_decode_noalloc(
-        _ptr(out, "out", (torch.bfloat16,), dev), _ptr(query, "query", (torch.bfloat16,), dev),
-        _ptr(key_cache, "key_cache", kv_types, dev), _ptr(value_cache, "value_cache", kv_types, dev),
-        S, Hq, int(num_kv_heads), D, float(scale),
-        _ptr(block_tables, "block_tables", (torch.int32,), dev), block_tables.shape[1],
-        _ptr(seq_lens, "seq_lens", (torch.int32,), dev), int(block_size), int(max_seq_len),
-        int(key_cache.shape[0]), code, ks, vs, st.cuda_stream)
+    ptrs = (_ptr(out, "out", (torch.bfloat16,), dev), _ptr(query, "query", (torch.bfloat16,), dev),
+            _ptr(key_cache, "key_cache", kv_types, dev),
+            _ptr(value_cache, "value_cache", kv_types, dev))
+    bt = _ptr(block_tables, "block_tables", (torch.int32,), dev)
+    sl = _ptr(seq_lens, "seq_lens", (torch.int32,), dev)
+    with torch.cuda.device(dev):  # the scratch array of the tensors' device
+        rc = lib().pa_decode_noalloc(*ptrs, S, Hq, int(num_kv_heads), D, float(scale), bt,
+                                     block_tables.shape[1], sl, int(block_size), int(max_seq_len),
+                                     int(key_cache.shape[0]), code, ks, vs, st.cuda_stream)
     _check(rc)
     return out
 
@@ -311,8 +316,10 @@ def read_status(workspace_tensor=None, device=None, clear=False, stream=None) ->
         workspace_tensor = workspace(WORKSPACE_HEADER_BYTES, dev)
     st = stream if stream is not None else torch.cuda.current_stream(workspace_tensor.device)
     flags = ctypes.c_uint32(0)
-    _check(lib().pa_read_device_status(ctypes.c_void_p(workspace_tensor.data_ptr()),
-                                       ctypes.byref(flags), int(bool(clear)), st.cuda_stream))
+    with torch.cuda.device(workspace_tensor.device):
+        rc = lib().pa_read_device_status(ctypes.c_void_p(workspace_tensor.data_ptr()),
+                                         ctypes.byref(flags), int(bool(clear)), st.cuda_stream)
+    _check(rc)
     return int(flags.value)
 
 
@@ -404,9 +411,11 @@ def copy_blocks(key_cache, value_cache, src, dst, kv_dtype="bf16", status=None, 
         raise ValueError("src and dst must have the same length")
     Hk, D = value_cache.shape[1], value_cache.shape[2]
     st = stream if stream is not None else torch.cuda.current_stream(dev)
-    rc = lib().pa_copy_blocks(
-        _ptr(key_cache, "key_cache", kv_types, dev), _ptr(value_cache, "value_cache", kv_types, dev),
-        int(Hk), int(D), int(value_cache.shape[3]), int(key_cache.shape[0]), code,
-        _ptr(src, "src", (torch.int64,), dev), _ptr(dst, "dst", (torch.int64,), dev), n,
-        None if status is None else _ptr(status, "status", None, dev), st.cuda_stream)
+    args = (_ptr(key_cache, "key_cache", kv_types, dev),
+            _ptr(value_cache, "value_cache", kv_types, dev),
+            int(Hk), int(D), int(value_cache.shape[3]), int(key_cache.shape[0]), code,
+            _ptr(src, "src", (torch.int64,), dev), _ptr(dst, "dst", (torch.int64,), dev), n,
+            None if status is None else _ptr(status, "status", None, dev), st.cuda_stream)
+    with torch.cuda.device(dev):
+        rc = lib().pa_copy_blocks(*args)
     _bm_check(rc)
