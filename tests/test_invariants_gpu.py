@@ -207,6 +207,43 @@ def test_calls_captured_in_a_cuda_graph():
     del graph
 
 
+@pytest.mark.parametrize("case", ["direct", "split", "cascade", "fp8_split"])
+def test_writes_stay_inside_out_and_workspace(case):
+    """Guard bands on both sides of `out` and of the workspace keep their
+    sentinel values through a call that writes outputs (and, split or
+    cascade, partials): no kernel writes outside the buffers it was given."""
+    lens = [300, 37, 1000, 520]
+    kv = W.FP8_E4M3 if case == "fp8_split" else W.BF16
+    pref = 2 if case == "cascade" else 0
+    cfg = _cfg(lens=lens, G=4, kv=kv, seed=411)
+    if pref:
+        cfg = cfg.replace(shared_prefix_blocks=pref)
+    wl = W.make_workload(cfg, DEV, seq_lens=lens)
+    pp = 0 if case in ("direct", "cascade") else 3
+    c = wl.cfg
+    need = pa.workspace_size(c.num_seqs, c.num_heads, c.num_kv_heads, c.head_size, c.block_size,
+                             c.max_seq_len, c.kv_dtype, partition_pages=pp,
+                             shared_prefix_blocks=pref)
+    G_WS = 256
+    wbuf = torch.full((need + 2 * G_WS,), 0xA5, dtype=torch.uint8, device=DEV)
+    wbuf[G_WS:G_WS + need].zero_()
+    ws = wbuf[G_WS:G_WS + need]
+    G_OUT = 64
+    n = wl.query.numel()
+    sentinel = -12288.0  # exact in bf16
+    obuf = torch.full((n + 2 * G_OUT,), sentinel, dtype=torch.bfloat16, device=DEV)
+    out = obuf[G_OUT:G_OUT + n].view(wl.query.shape)
+    pa.decode(out, wl.query, wl.key_cache, wl.value_cache, c.num_kv_heads, c.scale,
+              wl.block_tables, wl.seq_lens, c.block_size, c.max_seq_len, c.kv_dtype,
+              wl.k_scale, wl.v_scale, workspace_tensor=ws, partition_pages=pp,
+              shared_prefix_blocks=pref)
+    torch.cuda.synchronize()
+    assert (obuf[:G_OUT] == sentinel).all() and (obuf[-G_OUT:] == sentinel).all()
+    assert (wbuf[:G_WS] == 0xA5).all() and (wbuf[-G_WS:] == 0xA5).all()
+    assert pa.read_status(ws) == 0
+    compare(out, run_oracle(wl), c.kv_dtype, case)
+
+
 def test_bad_block_id_and_length_flags():
     lens = [100, 64]
     cfg = _cfg(lens=lens)
