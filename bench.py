@@ -199,7 +199,7 @@ def workload_config(idx: int, num_seqs: int = 0):
 
 
 def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, num_seqs=0,
-             cascade=True, alibi=False):
+             cascade=True, alibi=False, schedule="auto"):
     import torch
 
     import paged_kv_cache_471_b200 as pa
@@ -215,8 +215,10 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
     if alibi:  # geometric ALiBi slopes 2^(-8 i / H)
         slopes = torch.tensor([2.0 ** (-8.0 * (i + 1) / cfg.num_heads)
                                for i in range(cfg.num_heads)], dtype=torch.float32, device=device)
+    if prefix and schedule == "balanced":
+        schedule = "auto"  # balanced ranges do not take a shared prefix
     plan = pa.plan(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_size, cfg.block_size,
-                   cfg.max_seq_len, cfg.kv_dtype, shared_prefix_blocks=prefix)
+                   cfg.max_seq_len, cfg.kv_dtype, shared_prefix_blocks=prefix, schedule=schedule)
     ws = torch.zeros(plan["workspace_bytes"], dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
     alg_bytes = bytes_of(wl)
@@ -228,7 +230,7 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
         pa.decode(out, wl.query, wl.key_cache, wl.value_cache, cfg.num_kv_heads, cfg.scale,
                   wl.block_tables, wl.seq_lens, cfg.block_size, cfg.max_seq_len, cfg.kv_dtype,
                   wl.k_scale, wl.v_scale, workspace_tensor=ws, stream=stream,
-                  shared_prefix_blocks=prefix, alibi_slopes=slopes)
+                  shared_prefix_blocks=prefix, alibi_slopes=slopes, schedule=schedule)
 
     for _ in range(max(warmup, 3)):
         if flush:
@@ -308,7 +310,7 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
                                            cfg.num_kv_heads, cfg.scale, wl.block_tables,
                                            wl.seq_lens, cfg.block_size, cfg.max_seq_len,
                                            cfg.kv_dtype, wl.k_scale, wl.v_scale,
-                                           workspace_tensor=ws, stream=st)
+                                           workspace_tensor=ws, stream=st, schedule=schedule)
             step_on(gs)  # warm on the capture stream
             gs.synchronize()
             with torch.cuda.graph(graph, stream=gs):
@@ -330,7 +332,8 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
                region_ms=region_ms, step_ms=step_ms, local_step_ms=local_step_ms, flush=flush,
                flush_ms=flush_ms,
                clocks=clk.summary(), status=status,
-               launches_per_step=1 + (plan["num_partitions"] > 1 or prefix > 0),
+               launches_per_step=1 + (plan["num_partitions"] > 1 or prefix > 0
+                                      or plan["balanced"] == 1),
                shared_prefix_blocks=prefix, alibi=alibi, extra=extra)
 
     if want_e2e:
@@ -373,7 +376,8 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
                 pa.decode(out_d[b], q_d[b], wl.key_cache, wl.value_cache, cfg.num_kv_heads,
                           cfg.scale, bt_d[b], sl_d[b], cfg.block_size, cfg.max_seq_len,
                           cfg.kv_dtype, wl.k_scale, wl.v_scale, workspace_tensor=ws,
-                          stream=stream, shared_prefix_blocks=prefix, alibi_slopes=slopes)
+                          stream=stream, shared_prefix_blocks=prefix, alibi_slopes=slopes,
+                          schedule=schedule)
                 ev_used[b].record(stream)
                 with torch.cuda.stream(down):
                     down.wait_event(ev_used[b])
@@ -621,6 +625,8 @@ def main(argv=None):
     ap.add_argument("--extra", default="", choices=["", "copy_blocks"],
                     help="measure a side kernel instead of decode")
     ap.add_argument("--alibi", action="store_true", help="decode with ALiBi slopes")
+    ap.add_argument("--schedule", default="auto", choices=["auto", "balanced", "partitioned"],
+                    help="how CTAs share the work (pa_options.schedule)")
     ap.add_argument("--no-cascade", action="store_true",
                     help="do not declare a workload's shared prefix (plain per-sequence decode)")
     ap.add_argument("--num-seqs", type=int, default=0,
@@ -652,7 +658,8 @@ def main(argv=None):
     cfg_ids = [1, 2, 3, 4, 5] if args.config == "all" else [int(args.config)]
     for idx in cfg_ids:
         r = time_gpu(idx, args.steps, args.warmup, device, want_e2e=not args.no_e2e, rank=rank,
-                     num_seqs=args.num_seqs, cascade=not args.no_cascade, alibi=args.alibi)
+                     num_seqs=args.num_seqs, cascade=not args.no_cascade, alibi=args.alibi,
+                     schedule=args.schedule)
         r["step_ms"] = reduce_max(r["step_ms"], device)
         if "e2e_ms" in r:
             r["e2e_ms"] = reduce_max(r["e2e_ms"], device)

@@ -121,6 +121,16 @@ typedef enum pa_kv_dtype {
  *      handles: components more than about 2^9 below their largest |q| keep
  *      only an absolute error of about 2^-17 max|q| (the e4m3 subnormal
  *      floor).  Requires kv_dtype = PA_KV_FP8_E4M3.
+ *  schedule: how CTAs share the work.  PA_SCHEDULE_AUTO (0) and
+ *      PA_SCHEDULE_PARTITIONED: one CTA per (sequence, kv head, partition), as
+ *      many waves as that takes; the hardware hands units to SMs as they free
+ *      up.  PA_SCHEDULE_BALANCED: one wave of CTAs (grid_ctas = resident CTA
+ *      slots), each taking an equal contiguous share of all (sequence, kv
+ *      head, page) work; units cut at a share's ends are merged by the
+ *      combine kernel, which then runs on every call.  That removes the last
+ *      partial wave, but every CTA then waits for the slowest SM; it pays
+ *      where SMs stream at even rates (measured on e4m3 pages, ~1%).  Needs
+ *      no shared prefix and no forced partition_pages (PA_ERR_UNSUPPORTED).
  *  test_stall_copies: for testing the failure path only.  Non-zero makes every
  *      page's completion barrier wait for 16 bytes that no copy delivers and
  *      cuts each wait to ~20 ms, so the kernel takes its give-up path: it lets
@@ -137,7 +147,13 @@ typedef struct pa_options {
     const float* alibi_slopes;
     int fp8_compute;
     int test_stall_copies;
+    int schedule;
 } pa_options;
+
+/* pa_options.schedule values. */
+#define PA_SCHEDULE_AUTO 0
+#define PA_SCHEDULE_BALANCED 1
+#define PA_SCHEDULE_PARTITIONED 2
 
 /* What pa_decode will launch for a given problem. */
 typedef struct pa_plan {
@@ -150,6 +166,8 @@ typedef struct pa_plan {
     size_t workspace_bytes; /* bytes pa_decode needs in `workspace`                     */
     int prefix_partitions;  /* partitions of a declared shared prefix (0 = none)        */
     int prefix_groups;      /* 16-query-row groups per kv head streaming the prefix     */
+    int balanced;           /* 1: balanced page ranges (num_partitions and
+                               partition_pages are then 0), 0: fixed partitions        */
 } pa_plan;
 
 /*

@@ -51,7 +51,7 @@ class Options(ctypes.Structure):
     _fields_ = [("partition_pages", ctypes.c_int), ("num_sms", ctypes.c_int),
                 ("stages", ctypes.c_int), ("shared_prefix_blocks", ctypes.c_int),
                 ("alibi_slopes", ctypes.c_void_p), ("fp8_compute", ctypes.c_int),
-                ("test_stall_copies", ctypes.c_int)]
+                ("test_stall_copies", ctypes.c_int), ("schedule", ctypes.c_int)]
 
 
 class Plan(ctypes.Structure):
@@ -59,7 +59,7 @@ class Plan(ctypes.Structure):
                 ("stages", ctypes.c_int), ("warps_per_cta", ctypes.c_int),
                 ("grid_ctas", ctypes.c_longlong), ("smem_bytes", ctypes.c_size_t),
                 ("workspace_bytes", ctypes.c_size_t), ("prefix_partitions", ctypes.c_int),
-                ("prefix_groups", ctypes.c_int)]
+                ("prefix_groups", ctypes.c_int), ("balanced", ctypes.c_int)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}
@@ -144,14 +144,20 @@ def _check(rc: int):
                                       f"{L.pa_last_error_detail().decode()}")
 
 
+SCHEDULES = {"auto": 0, "balanced": 1, "partitioned": 2}
+
+
 def _opts(partition_pages=0, num_sms=0, stages=0, shared_prefix_blocks=0, alibi_ptr=None,
-          fp8_compute=False, test_stall_copies=False):
+          fp8_compute=False, test_stall_copies=False, schedule="auto"):
+    if schedule not in SCHEDULES:
+        raise ValueError(f"schedule must be one of {sorted(SCHEDULES)}")
     if not partition_pages and not num_sms and not stages and not shared_prefix_blocks \
-            and not alibi_ptr and not fp8_compute and not test_stall_copies:
+            and not alibi_ptr and not fp8_compute and not test_stall_copies \
+            and schedule == "auto":
         return None
     return ctypes.byref(Options(int(partition_pages), int(num_sms), int(stages),
                                 int(shared_prefix_blocks), alibi_ptr, int(bool(fp8_compute)),
-                                int(bool(test_stall_copies))))
+                                int(bool(test_stall_copies)), SCHEDULES[schedule]))
 
 
 def kv_dtype_code(kv_dtype) -> int:
@@ -162,19 +168,23 @@ def kv_dtype_code(kv_dtype) -> int:
 
 
 def plan(num_seqs, num_heads, num_kv_heads, head_size, block_size, max_seq_len, kv_dtype="bf16",
-         partition_pages=0, num_sms=0, stages=0, shared_prefix_blocks=0) -> dict:
+         partition_pages=0, num_sms=0, stages=0, shared_prefix_blocks=0, fp8_compute=False,
+         schedule="auto") -> dict:
     p = Plan()
     _check(lib().pa_plan_decode(ctypes.byref(p), num_seqs, num_heads, num_kv_heads, head_size,
                                 block_size, max_seq_len, kv_dtype_code(kv_dtype),
-                                _opts(partition_pages, num_sms, stages, shared_prefix_blocks)))
+                                _opts(partition_pages, num_sms, stages, shared_prefix_blocks,
+                                      None, fp8_compute, False, schedule)))
     return p.as_dict()
 
 
 def workspace_size(num_seqs, num_heads, num_kv_heads, head_size, block_size, max_seq_len,
-                   kv_dtype="bf16", partition_pages=0, num_sms=0, shared_prefix_blocks=0) -> int:
+                   kv_dtype="bf16", partition_pages=0, num_sms=0, shared_prefix_blocks=0,
+                   fp8_compute=False, schedule="auto", stages=0) -> int:
     n = lib().pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_size, block_size,
                                        max_seq_len, kv_dtype_code(kv_dtype),
-                                       _opts(partition_pages, num_sms, 0, shared_prefix_blocks))
+                                       _opts(partition_pages, num_sms, stages, shared_prefix_blocks,
+                                             None, fp8_compute, False, schedule))
     if n == 0:
         raise PagedAttentionError(PA_ERR_INVALID_ARG, lib().pa_last_error_detail().decode())
     return n
@@ -215,7 +225,7 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
            seq_lens, block_size: int, max_seq_len: int, kv_dtype="bf16", k_scale=None,
            v_scale=None, workspace_tensor=None, partition_pages: int = 0, stream=None,
            stages: int = 0, shared_prefix_blocks: int = 0, alibi_slopes=None,
-           fp8_compute: bool = False, test_stall_copies: bool = False):
+           fp8_compute: bool = False, test_stall_copies: bool = False, schedule: str = "auto"):
     """Paged decode attention into ``out`` (bf16 [num_seqs, num_heads, head_size]).
 
     key_cache: [num_blocks, num_kv_heads, head_size/x, block_size, x];
@@ -262,7 +272,9 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
     # tensors' device for the call.
     with torch.cuda.device(dev):
         need = workspace_size(S, Hq, num_kv_heads, D, block_size, max_seq_len, code,
-                              partition_pages, shared_prefix_blocks=shared_prefix_blocks)
+                              partition_pages, shared_prefix_blocks=shared_prefix_blocks,
+                              fp8_compute=fp8_compute and code == PA_KV_FP8_E4M3,
+                              schedule=schedule, stages=stages)
         if workspace_tensor is None:
             workspace_tensor = workspace(need, dev)
         ws = _ptr(workspace_tensor, "workspace", None, dev)
@@ -272,7 +284,7 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
                                 workspace_tensor.numel() * workspace_tensor.element_size(),
                                 st.cuda_stream,
                                 _opts(partition_pages, 0, stages, shared_prefix_blocks, alibi,
-                                      fp8_compute, test_stall_copies))
+                                      fp8_compute, test_stall_copies, schedule))
     _check(rc)
     return out
 

@@ -107,6 +107,11 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
     const bool cascade = prefix > 0 && num_seqs > 0;
     if (cascade && opts->alibi_slopes)
         return fail(PA_ERR_UNSUPPORTED, "%s", "ALiBi slopes with a shared prefix");
+    const int schedule = opts ? opts->schedule : PA_SCHEDULE_AUTO;
+    if (schedule != PA_SCHEDULE_AUTO && schedule != PA_SCHEDULE_BALANCED &&
+        schedule != PA_SCHEDULE_PARTITIONED)
+        return fail(PA_ERR_INVALID_ARG, "%s", "opts->schedule");
+    const bool f8mma = opts && opts->fp8_compute && kv_dtype == PA_KV_FP8_E4M3;
     const size_t stage = 2ull * head_size * block_size * elem_bytes(kv_dtype);
     const int W = pa::decode_warps(static_cast<long long>(stage));
     int ns = kDefaultStages;
@@ -120,10 +125,47 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
     long long per_sm = static_cast<long long>(kSmemPerSm / (smem + kSmemReservedPerCta));
     if (per_sm < 1) per_sm = 1;
     if (per_sm > kMaxCtasPerSm) per_sm = kMaxCtasPerSm;  // register limit
+    if (f8mma && per_sm > 2) per_sm = 2;                // e4m3-MMA forms: ~200+ registers
     const long long slots = static_cast<long long>(sms) * per_sm;
 
     const long long pages_max = (static_cast<long long>(max_seq_len) + block_size - 1) / block_size;
     const long long units = static_cast<long long>(num_seqs) * num_kv_heads;
+
+    // Balanced ranges (on request): one wave of CTAs, each an equal share of
+    // all pages (pa_decode_kernels.cuh).  Not the default: measured on B200,
+    // SMs stream bf16 pages at rates ~7% apart (std), so equal static shares
+    // wait for the slowest SMs, while one CTA per unit lets the hardware hand
+    // more units to faster SMs.  e4m3 pages stream at even rates across SMs,
+    // and there the balanced ranges gained ~1% (256 x 16384 tokens).  Needs no
+    // shared prefix, no forced partitions, the per-sequence page scan in the
+    // stage area, and page counts in int.
+    const bool forced_pp = opts && opts->partition_pages > 0;
+    const bool br_fits = !cascade && !forced_pp && num_seqs > 0 &&
+                         (static_cast<size_t>(num_seqs) + 1 + 32 * W) * 4 <= stage_area &&
+                         units * (pages_max + 1) < (1ll << 31);
+    if (schedule == PA_SCHEDULE_BALANCED && !br_fits)
+        return fail(PA_ERR_UNSUPPORTED, "%s",
+                    "balanced ranges need no shared prefix, no forced partitions and a batch "
+                    "whose lengths fit the stage memory");
+    const bool balanced = br_fits && schedule == PA_SCHEDULE_BALANCED;
+    if (balanced) {
+        const long long rows = 2 * slots * (num_heads / num_kv_heads);
+        size_t ws = PA_WORKSPACE_HEADER_BYTES;
+        ws += ((static_cast<size_t>(num_seqs) + 2) * sizeof(int) + 255) & ~static_cast<size_t>(255);
+        ws += static_cast<size_t>(rows) * (static_cast<size_t>(head_size) + 2) * sizeof(float);
+        ws = (ws + 255) & ~static_cast<size_t>(255);
+        pl->num_partitions = 0;
+        pl->partition_pages = 0;
+        pl->stages = ns;
+        pl->warps_per_cta = W;
+        pl->grid_ctas = slots;
+        pl->smem_bytes = smem;
+        pl->workspace_bytes = ws;
+        pl->prefix_partitions = 0;
+        pl->prefix_groups = 0;
+        pl->balanced = 1;
+        return PA_OK;
+    }
     long long pp;
     if (opts && opts->partition_pages > 0) {
         pp = opts->partition_pages;
@@ -201,6 +243,7 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
     pl->workspace_bytes = ws;
     pl->prefix_partitions = static_cast<int>(p_pre);
     pl->prefix_groups = static_cast<int>(groups);
+    pl->balanced = 0;
     return PA_OK;
 }
 
@@ -410,8 +453,16 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     p.status = reinterpret_cast<uint32_t*>(ws);
     const int p_total = pl.num_partitions + pl.prefix_partitions;
-    const size_t rows = static_cast<size_t>(num_seqs) * num_heads * p_total;
+    size_t rows = static_cast<size_t>(num_seqs) * num_heads * p_total;
     float* part = reinterpret_cast<float*>(ws + PA_WORKSPACE_HEADER_BYTES);
+    if (pl.balanced) {
+        // [header][per-sequence page scan, S + 2 ints][slots: 2 per CTA, G rows each]
+        p.br_scan = reinterpret_cast<int*>(ws + PA_WORKSPACE_HEADER_BYTES);
+        const size_t scan_bytes =
+            ((static_cast<size_t>(num_seqs) + 2) * sizeof(int) + 255) & ~static_cast<size_t>(255);
+        part = reinterpret_cast<float*>(ws + PA_WORKSPACE_HEADER_BYTES + scan_bytes);
+        rows = 2 * static_cast<size_t>(pl.grid_ctas) * (num_heads / num_kv_heads);
+    }
     p.ws_o = part;
     p.ws_m = part + rows * head_size;
     p.ws_l = p.ws_m + rows;
@@ -431,7 +482,8 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
     p.prefix_units = static_cast<long long>(num_kv_heads) * pl.prefix_groups * pl.prefix_partitions;
     p.P_total = p_total;
     p.alibi = opts ? opts->alibi_slopes : nullptr;
-    p.longest_first = (num_seqs > 1 && num_seqs <= kMaxRankedSeqs) ? 1 : 0;
+    p.longest_first = (!pl.balanced && num_seqs > 1 && num_seqs <= kMaxRankedSeqs) ? 1 : 0;
+    p.balanced = pl.balanced;
     p.stall_tx_bytes = 0;
     p.wait_limit_ns = kWaitLimitNs;
     if (opts && opts->test_stall_copies) {
@@ -444,7 +496,7 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
     cudaError_t e = launch_any(p, head_size, block_size, kv_dtype == PA_KV_FP8_E4M3, f8mma,
                                pl.grid_ctas, pl.smem_bytes, s);
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
-    if (pl.num_partitions > 1 || p.prefix_pages > 0) {
+    if (pl.balanced || pl.num_partitions > 1 || p.prefix_pages > 0) {
         pa::CombineParams c;
         c.out = p.out;
         c.ws_o = p.ws_o;
@@ -460,6 +512,10 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
         c.prefix_pages = p.prefix_pages;
         c.prefix_parts = p.prefix_parts;
         c.P_total = p.P_total;
+        c.balanced = pl.balanced;
+        c.Hk = num_kv_heads;
+        c.G = num_heads / num_kv_heads;
+        c.br_scan = p.br_scan;
         e = launch_combine(c, head_size, s);
         if (e != cudaSuccess) return fail(PA_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
     }

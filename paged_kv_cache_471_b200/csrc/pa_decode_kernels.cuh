@@ -1,8 +1,11 @@
 // Paged decode attention kernels for sm_100a.
 //
-// pa_decode_kernel: one CTA per (sequence, kv head, partition); four warps,
-// each an independent producer/consumer pipeline over its share of the
-// partition's pages (pages w, w+4, w+8, ... of the partition).
+// pa_decode_kernel: by default one CTA per (sequence, kv head, partition);
+// with balanced ranges, one wave of CTAs that each walk an equal contiguous
+// share of all (sequence, kv head, page) work, one unit segment at a time
+// (see DecodeParams::balanced).  Within a segment, four warps (two for 16 KiB
+// pages), each an independent producer/consumer pipeline over its share of
+// the segment's pages (pages w, w+4, w+8, ... of the segment).
 //   * Lane 0 of a warp reads the block table (the page table of
 //     "Why PagedAttention was retired", section 1), widens the physical id to
 //     64 bits, and moves the whole (block, kv head) K page and V page --
@@ -18,11 +21,12 @@
 //   * FP8 e4m3 pages are converted in registers (exact e4m3 -> f16) right
 //     before the MMA; k_scale folds into the logit scale and v_scale into the
 //     output, so the conversion needs no multiply (section 4 of the page).
-//   * The four warps' (max, sum, acc) are merged in shared memory; the CTA
-//     writes bf16 out directly, or, when the sequence is split over several
-//     partitions, an fp32 partial plus its (max, sum) for pa_combine_kernel
-//     (the exp_sums / max_logits / tmp_output roles of the partitioned
-//     variant in the PR #47361 benchmark snippet).
+//   * The warps' (max, sum, acc) are merged in shared memory; the CTA
+//     writes bf16 out directly, or, when the unit is split over several
+//     partitions (or cut at a balanced range's end), an fp32 partial plus its
+//     (max, sum) for pa_combine_kernel (the exp_sums / max_logits /
+//     tmp_output roles of the partitioned variant in the PR #47361 benchmark
+//     snippet).
 //
 // Every mbarrier wait is bounded (~2 s); on give-up the warp drains its copies
 // in flight (bounded too), ORs PA_DEV_WAIT_TIMEOUT into the status word and
@@ -84,6 +88,15 @@ struct DecodeParams {
     // Longest first: per-sequence CTAs take sequences in order of decreasing
     // length (ties by index), ranked by every CTA from seq_lens (num_seqs <= 256).
     int longest_first;
+    // Balanced ranges (no shared prefix): the grid's CTAs take equal contiguous
+    // shares of all pages in (sequence, kv head, page) order, and each walks
+    // its share one unit segment at a time.  A segment that is a whole unit
+    // writes `out`; a cut one writes slot 2 c + k of CTA c (k = 0: the first
+    // segment of its range, 1: the last), rows of G query heads, for
+    // pa_combine_kernel.  CTA 0 leaves the per-sequence page prefix and the
+    // pages per CTA in br_scan[0 .. S + 1] for the combine.
+    int balanced;
+    int* br_scan;
 };
 
 // Bytes of shared memory the final merge needs (it overlays the page stages).
@@ -130,54 +143,152 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
     const int gq = lane >> 2;  // fragment row group
     const int cq = lane & 3;   // thread in quad
 
-    const long long unit = blockIdx.x;
-    const bool pre = unit < p.prefix_units;  // a shared-prefix unit
-    int kvh, s, part, rg = 0;
-    if (pre) {
-        kvh = static_cast<int>(unit % p.Hk);
-        rg = static_cast<int>((unit / p.Hk) % p.prefix_groups);
-        part = static_cast<int>(unit / ((long long)p.Hk * p.prefix_groups));
-        s = 0;
+    // ---------------- this CTA's work: one unit, or a balanced page range
+    bool pre = false;  // a shared-prefix unit
+    int kvh = 0, s = 0, part = 0, rg = 0;
+    long long bx = 0, bx_first = 0, bx_end = 0;  // balanced: pages [bx, bx_end) still to do
+    int bj = 0, bn = 0;                          // balanced: page in the unit, pages of the unit
+    const int t_cap = p.max_blocks * B;
+    auto pages_of = [&](int seq) {
+        const int t = max(0, min(__ldg(p.seq_lens + seq), t_cap));
+        return (t + B - 1) / B;
+    };
+    if (p.balanced) {
+        // Pages of every sequence and their exclusive prefix sum, at the start
+        // of shared memory (no page is in flight yet): scan[i] for i < S, the
+        // total at scan[S], then one partial sum per thread.
+        int* scan = reinterpret_cast<int*>(smem);
+        int* tsum = scan + p.S + 1;
+        constexpr int NT = W * 32;
+        const int chunk = (p.S + NT - 1) / NT;
+        const int i0 = min(p.S, static_cast<int>(threadIdx.x) * chunk);
+        const int i1 = min(p.S, i0 + chunk);
+        int local = 0;
+        bool bad_len = false;
+        for (int i = i0; i < i1; ++i) {
+            const int t = __ldg(p.seq_lens + i);
+            bad_len |= t < 0 || t > t_cap;
+            const int n = pages_of(i);
+            scan[i] = n;
+            local += n;
+        }
+        if (bad_len && blockIdx.x == 0) atomicOr(p.status, kDevSeqLen);
+        tsum[threadIdx.x] = local;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int run = 0;
+            for (int t = 0; t < NT; ++t) {
+                const int v = tsum[t];
+                tsum[t] = run;
+                run += v;
+            }
+            scan[p.S] = run;
+        }
+        __syncthreads();
+        int run = tsum[threadIdx.x];
+        for (int i = i0; i < i1; ++i) {
+            const int v = scan[i];
+            scan[i] = run;
+            run += v;
+        }
+        __syncthreads();
+        const long long total = static_cast<long long>(p.Hk) * scan[p.S];
+        const long long per = max(1LL, (total + gridDim.x - 1) / gridDim.x);
+        bx = static_cast<long long>(blockIdx.x) * per;
+        bx_first = bx;
+        bx_end = min(total, bx + per);
+        if (blockIdx.x == 0) {
+            for (int i = threadIdx.x; i <= p.S; i += NT) p.br_scan[i] = scan[i];
+            if (threadIdx.x == 0) p.br_scan[p.S + 1] = static_cast<int>(per);
+        }
+        if (bx < bx_end) {
+            // The sequence holding page bx: the largest s with Hk scan[s] <= bx.
+            // It has pages, since bx < Hk scan[S].
+            int lo = 0, hi = p.S - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (static_cast<long long>(p.Hk) * scan[mid] <= bx)
+                    lo = mid;
+                else
+                    hi = mid - 1;
+            }
+            s = lo;
+            bn = scan[s + 1] - scan[s];
+            const long long off = bx - static_cast<long long>(p.Hk) * scan[s];
+            kvh = static_cast<int>(off / bn);
+            bj = static_cast<int>(off - static_cast<long long>(kvh) * bn);
+        }
+        __syncthreads();  // the scratch is page memory from here on
+        if (bx >= bx_end) return;  // no work for this CTA (same for all its threads)
     } else {
-        const long long u = unit - p.prefix_units;
-        kvh = static_cast<int>(u % p.Hk);
-        s = static_cast<int>((u / p.Hk) % p.S);
-        part = static_cast<int>(u / ((long long)p.Hk * p.S));
-        if (p.longest_first) {
-            // The unit's sequence index is a rank: find the sequence with that
-            // rank among all lengths, longest first, so that the longest work
-            // starts first and the last wave of CTAs is short.  Uses the start
-            // of shared memory, which holds no page yet.
-            int* lens = reinterpret_cast<int*>(smem);
-            const int cap = p.max_blocks * B;
-            const int len0 = max(0, min(__ldg(p.seq_lens), cap));
-            int differs = 0;
-            for (int i = threadIdx.x; i < p.S; i += W * 32) {
-                lens[i] = max(0, min(__ldg(p.seq_lens + i), cap));
-                differs |= lens[i] != len0;
-            }
-            // Equal lengths (a block-wide vote): index order is already longest
-            // first.  Otherwise every sequence's rank is counted and the one
-            // whose rank is the unit's index is picked.
-            if (__syncthreads_or(differs)) {
+        const long long unit = blockIdx.x;
+        pre = unit < p.prefix_units;
+        if (pre) {
+            kvh = static_cast<int>(unit % p.Hk);
+            rg = static_cast<int>((unit / p.Hk) % p.prefix_groups);
+            part = static_cast<int>(unit / ((long long)p.Hk * p.prefix_groups));
+            s = 0;
+        } else {
+            const long long u = unit - p.prefix_units;
+            kvh = static_cast<int>(u % p.Hk);
+            s = static_cast<int>((u / p.Hk) % p.S);
+            part = static_cast<int>(u / ((long long)p.Hk * p.S));
+            if (p.longest_first) {
+                // The unit's sequence index is a rank: find the sequence with
+                // that rank among all lengths, longest first, so that the
+                // longest work starts first and the last wave of CTAs is short.
+                // Uses the start of shared memory, which holds no page yet.
+                int* lens = reinterpret_cast<int*>(smem);
+                const int len0 = max(0, min(__ldg(p.seq_lens), t_cap));
+                int differs = 0;
                 for (int i = threadIdx.x; i < p.S; i += W * 32) {
-                    const int v = lens[i];
-                    int rank = 0;
-                    for (int j = 0; j < p.S; ++j) {
-                        const int w2 = lens[j];
-                        rank += (w2 > v) | ((w2 == v) & (j < i));
-                    }
-                    if (rank == s) lens[p.S] = i;
+                    lens[i] = max(0, min(__ldg(p.seq_lens + i), t_cap));
+                    differs |= lens[i] != len0;
                 }
-                __syncthreads();
-                s = lens[p.S];
+                // Equal lengths (a block-wide vote): index order is already
+                // longest first.  Otherwise every sequence's rank is counted and
+                // the one whose rank is the unit's index is picked.
+                if (__syncthreads_or(differs)) {
+                    for (int i = threadIdx.x; i < p.S; i += W * 32) {
+                        const int v = lens[i];
+                        int rank = 0;
+                        for (int j = 0; j < p.S; ++j) {
+                            const int w2 = lens[j];
+                            rank += (w2 > v) | ((w2 == v) & (j < i));
+                        }
+                        if (rank == s) lens[p.S] = i;
+                    }
+                    __syncthreads();
+                    s = lens[p.S];
+                }
+                __syncthreads();  // the scratch is page memory from here on
             }
-            __syncthreads();  // the scratch is page memory from here on
         }
     }
+
+    // Shared memory: per-warp page stages, then the mbarriers.  The ring keeps
+    // its stage / phase counters across a CTA's segments (every segment
+    // consumes all it issued).
+    const int NS = p.stages;
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t wstage0 = sbase + static_cast<uint32_t>(warp * NS * STAGE);
+    // mbarriers sit after the larger of the page stages and the merge buffer
+    // that later overlays them (the host sizes shared memory the same way).
+    const int stage_area = max(W * NS * STAGE, merge_smem_bytes<D, NH, W>());
+    const uint32_t bar0 = sbase + static_cast<uint32_t>(stage_area + warp * NS * 8);
+    if (lane == 0) {
+        for (int i = 0; i < NS; ++i) mbar_init(bar0 + 8 * i, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    int stage = 0;
+    uint32_t phase = 0;
+    int issue_stage = 0;
+
+    for (;;) {  // one segment per pass (a single pass unless balanced)
     const bool cascade = p.prefix_pages > 0;
     const int pg0 = pre ? 0 : p.prefix_pages;  // first page of this unit's page range
-    const int j0 = pg0 + part * p.PP;
+    const int j0 = p.balanced ? bj : pg0 + part * p.PP;
     const long long row0 = (long long)s * p.Hq + (long long)kvh * p.G;  // first q head row
     const int rows_total = p.S * p.G;  // query rows of one kv head (prefix units)
 
@@ -196,7 +307,8 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
     // the partition's end is readable), the raw query words and the scales.
     // Block-table window: lane l holds the id of this warp's page (wbase + l).
     const int32_t* btrow = p.bt + (long long)s * p.max_blocks;
-    const int jcap = min(j0 + p.PP, pre ? p.prefix_pages : p.max_blocks);
+    const int jcap = p.balanced ? min(bj + bn, p.max_blocks)
+                                : min(j0 + p.PP, pre ? p.prefix_pages : p.max_blocks);
     auto load_win = [&](int base) -> int {
         const int j = j0 + warp + W * (base + lane);
         return j < jcap ? __ldg(btrow + j) : -1;
@@ -249,14 +361,13 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
     } else {
         T = __ldg(p.seq_lens + s);
         uint32_t bad = 0;
-        const int t_cap = p.max_blocks * B;
         if (T < 0) { T = 0; bad = kDevSeqLen; }
         if (T > t_cap) { T = t_cap; bad = kDevSeqLen; }
         nb = (T + B - 1) / B;
-        const int covered = pg0 + p.P * p.PP;
+        const int covered = p.balanced ? nb : pg0 + p.P * p.PP;
         if (nb > covered) { nb = covered; T = nb * B; bad = kDevSeqLen; }
         if (cascade && T < p.prefix_pages * B) bad |= kDevPrefix;
-        if (bad && part == 0 && kvh == 0 && threadIdx.x == 0) atomicOr(p.status, bad);
+        if (bad && part == 0 && kvh == 0 && j0 == pg0 && threadIdx.x == 0) atomicOr(p.status, bad);
         if (cascade && part == 0 && kvh == 0 && warp == 0 && s > 0) {
             // The declared prefix must be the same physical blocks as row 0's.
             bool same = true;
@@ -266,8 +377,11 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
         }
     }
 
-    const int j1 = min(nb, j0 + p.PP);
-    const bool direct = !cascade && ((p.P == 1) || (nb <= p.PP));
+    // Balanced: the segment ends with the unit or with the CTA's range.
+    const int j1 = p.balanced ? static_cast<int>(min(static_cast<long long>(nb), j0 + (bx_end - bx)))
+                              : min(nb, j0 + p.PP);
+    const bool direct = !cascade && (p.balanced ? (j0 == 0 && j1 == nb)
+                                                : ((p.P == 1) || (nb <= p.PP)));
 
     if (j0 >= j1) {
         if (!cascade && part == 0) {  // empty sequence: defined as a zero output row
@@ -277,21 +391,8 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
         return;
     }
 
-    const int NS = p.stages;
     const int span = j1 - j0;
     const int n_my = span > warp ? (span - warp + W - 1) / W : 0;
-    const uint32_t sbase = smem_addr(smem);
-    const uint32_t wstage0 = sbase + static_cast<uint32_t>(warp * NS * STAGE);
-    // mbarriers sit after the larger of the page stages and the merge buffer
-    // that later overlays them (the host sizes shared memory the same way).
-    const int stage_area = max(W * NS * STAGE, merge_smem_bytes<D, NH, W>());
-    const uint32_t bar0 = sbase + static_cast<uint32_t>(stage_area + warp * NS * 8);
-
-    if (lane == 0) {
-        for (int i = 0; i < NS; ++i) mbar_init(bar0 + 8 * i, 1);
-        fence_mbar_init();
-    }
-    __syncwarp();
 
     int wbase = 0;
     uint32_t valid_mask = 0;  // bit per stage: the page in it had a legal block id
@@ -300,9 +401,9 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
     const size_t block_stride = static_cast<size_t>(p.Hk) * PAGE;
 
     // Issue the copies of this warp's i-th page (warp-uniform call, pages in
-    // increasing order).  Page i lives in stage i mod NS; `issue_stage` tracks
-    // that without a division.
-    int issue_stage = 0;
+    // increasing order).  Pages go to consecutive stages of the ring, starting
+    // where the consumer stands; `issue_stage` tracks that without a division.
+    issue_stage = stage;
     auto issue = [&](int i) {
         if (i >= wbase + 32) {
             win_a = win_b;
@@ -697,8 +798,6 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
 
     bool timed_out = false;
     int k = 0;
-    int stage = 0;
-    uint32_t phase = 0;
     for (; k < n_my; ++k) {
         const bool landed = mbar_wait_bounded(bar0 + 8 * stage, phase, p.wait_limit_ns);
         if (!__all_sync(kFull, landed)) {
@@ -775,6 +874,9 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
 
     const int rows_here = pre ? min(16, rows_total - rg * 16) : p.G;
     const int slot = pre ? part : (cascade ? p.prefix_parts : 0) + part;
+    // Balanced: slot 2 c + k of this CTA, G rows (see DecodeParams).
+    const long long br_row0 =
+        (2LL * blockIdx.x + (bx == bx_first ? 0 : 1)) * static_cast<long long>(p.G);
     for (int idx = threadIdx.x; idx < rows_here * D; idx += (W * 32)) {
         const int h = idx / D;
         const int d = idx - h * D;
@@ -797,7 +899,7 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
         if (direct) {
             p.out[row * D + d] = __float2bfloat16_rn(o);
         } else {
-            const long long prow = row * p.P_total + slot;
+            const long long prow = p.balanced ? br_row0 + h : row * p.P_total + slot;
             p.ws_o[prow * D + d] = o;
             if (d == 0) {
                 p.ws_m[prow] = M;
@@ -805,6 +907,23 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
             }
         }
     }
+
+    // ---------------- next segment (balanced ranges only)
+    if (!p.balanced) break;
+    // A barrier every thread reaches: the merge buffer it ends (which overlays
+    // the stages) is free again, and a wait that gave up anywhere stops the CTA.
+    if (__syncthreads_or(timed_out)) break;
+    bx += j1 - j0;
+    if (bx >= bx_end) break;
+    bj = 0;
+    if (++kvh == p.Hk) {
+        kvh = 0;
+        do {
+            ++s;
+            bn = pages_of(s);
+        } while (bn == 0 && s + 1 < p.S);
+    }
+    }  // segments
 }
 
 struct CombineParams {
@@ -815,6 +934,8 @@ struct CombineParams {
     const int32_t* seq_lens;
     int S, Hq, P, PP, max_blocks, B;
     int prefix_pages, prefix_parts, P_total;
+    int balanced, Hk, G;
+    const int* br_scan;  // balanced: per-sequence page prefix [S + 1], pages per CTA
 };
 
 // Log-sum-exp merge of the split-KV partials of one (sequence, q head) per
@@ -822,6 +943,11 @@ struct CombineParams {
 // Without a shared prefix, rows whose sequence fits in one partition were
 // written by the decode kernel and are skipped here.  With one, the slots are
 // the prefix partitions followed by the sequence's own partitions.
+// Balanced ranges: the unit's pages [off, off + n) were cut over CTAs
+// off / per .. (off + n - 1) / per; the first of them holds it in its slot 1
+// (its last segment) unless the unit starts its range, every other one in its
+// slot 0 (its first segment).  A unit inside one CTA was written by the decode
+// kernel; a sequence with no pages gets a zero row here.
 // Partitions with an empty sum are skipped.
 template <int D>
 __global__ void __launch_bounds__(kThreads) pa_combine_kernel(const CombineParams p) {
@@ -831,21 +957,49 @@ __global__ void __launch_bounds__(kThreads) pa_combine_kernel(const CombineParam
     const long long row = (long long)blockIdx.x * kWarps + warp;
     if (row >= (long long)p.S * p.Hq) return;
     const int s = static_cast<int>(row / p.Hq);
-    int T = __ldg(p.seq_lens + s);
-    T = max(0, min(T, p.max_blocks * p.B));
-    const int nb = (T + p.B - 1) / p.B;
     int nps;
-    if (p.prefix_pages > 0) {
-        const int own = nb > p.prefix_pages ? (nb - p.prefix_pages + p.PP - 1) / p.PP : 0;
-        nps = p.prefix_parts + min(p.P, own);
+    long long base = row * p.P_total;  // slot i is partial row base + i ...
+    long long br_c0 = 0, br_off = 0, br_per = 1;
+    int br_g = 0;
+    if (p.balanced) {
+        const int h = static_cast<int>(row - static_cast<long long>(s) * p.Hq);
+        const int c_s = __ldg(p.br_scan + s);
+        const int n_s = __ldg(p.br_scan + s + 1) - c_s;
+        br_per = __ldg(p.br_scan + p.S + 1);
+        br_g = h % p.G;
+        if (n_s == 0) {
+            nps = 0;
+        } else {
+            br_off = static_cast<long long>(p.Hk) * c_s + static_cast<long long>(h / p.G) * n_s;
+            br_c0 = br_off / br_per;
+            const long long c1 = (br_off + n_s - 1) / br_per;
+            if (c1 == br_c0) return;
+            nps = static_cast<int>(c1 - br_c0 + 1);
+        }
     } else {
-        nps = min(p.P, (nb + p.PP - 1) / p.PP);
-        if (nps <= 1) return;
+        int T = __ldg(p.seq_lens + s);
+        T = max(0, min(T, p.max_blocks * p.B));
+        const int nb = (T + p.B - 1) / p.B;
+        if (p.prefix_pages > 0) {
+            const int own = nb > p.prefix_pages ? (nb - p.prefix_pages + p.PP - 1) / p.PP : 0;
+            nps = p.prefix_parts + min(p.P, own);
+        } else {
+            nps = min(p.P, (nb + p.PP - 1) / p.PP);
+            if (nps <= 1) return;
+        }
     }
-    const long long base = row * p.P_total;
+    // ... or, balanced, slot 2 c + k of CTA c = c0 + i, row g of its G rows.
+    auto slot_row = [&](int i) -> long long {
+        if (!p.balanced) return base + i;
+        const long long c = br_c0 + i;
+        const int k = (i == 0 && br_off != br_c0 * br_per) ? 1 : 0;
+        return (2 * c + k) * p.G + br_g;
+    };
     float M = -INFINITY;
-    for (int i = lane; i < nps; i += 32)
-        if (p.ws_l[base + i] > 0.f) M = fmaxf(M, p.ws_m[base + i]);
+    for (int i = lane; i < nps; i += 32) {
+        const long long r = slot_row(i);
+        if (p.ws_l[r] > 0.f) M = fmaxf(M, p.ws_m[r]);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
     constexpr int PER = D / 32;
@@ -854,11 +1008,12 @@ __global__ void __launch_bounds__(kThreads) pa_combine_kernel(const CombineParam
     for (int i = 0; i < PER; ++i) a[i] = 0.f;
     float L = 0.f;
     for (int i = 0; i < nps; ++i) {
-        const float l = p.ws_l[base + i];
+        const long long r = slot_row(i);
+        const float l = p.ws_l[r];
         if (!(l > 0.f)) continue;
-        const float wt = exp2f(p.ws_m[base + i] - M) * l;
+        const float wt = exp2f(p.ws_m[r] - M) * l;
         L += wt;
-        const float* o = p.ws_o + (base + i) * D;
+        const float* o = p.ws_o + r * D;
 #pragma unroll
         for (int j = 0; j < PER; ++j) a[j] += wt * o[lane + 32 * j];
     }

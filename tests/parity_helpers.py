@@ -21,14 +21,15 @@ def kv_code(cfg):
     return oracle.KV_E4M3 if cfg.kv_dtype == W.FP8_E4M3 else oracle.KV_BF16
 
 
-def run_gpu(wl: W.Workload, partition_pages=0, out=None, ws=None, stream=None):
+def run_gpu(wl: W.Workload, partition_pages=0, out=None, ws=None, stream=None,
+            schedule="auto"):
     c = wl.cfg
     if out is None:
         out = torch.empty_like(wl.query)
     pa.decode(out, wl.query, wl.key_cache, wl.value_cache, c.num_kv_heads, c.scale,
               wl.block_tables, wl.seq_lens, c.block_size, c.max_seq_len, c.kv_dtype,
               wl.k_scale, wl.v_scale, workspace_tensor=ws, partition_pages=partition_pages,
-              stream=stream)
+              stream=stream, schedule=schedule)
     return out
 
 

@@ -102,6 +102,17 @@ def test_workspace_size_header_only_without_split():
     assert n == pa.WORKSPACE_HEADER_BYTES
 
 
+def test_balanced_workspace_layout():
+    # header, the per-sequence page scan (S + 2 ints, 256-byte aligned), then
+    # two slots of G rows of (D + 2) floats per CTA slot.
+    p = pa.plan(64, 32, 8, 128, 16, 4096, "bf16", num_sms=148, schedule="balanced")
+    assert p["balanced"] == 1 and p["num_partitions"] == 0 and p["grid_ctas"] == 3 * 148
+    scan = -(-(64 + 2) * 4 // 256) * 256
+    rows = 2 * p["grid_ctas"] * 4
+    expect = -(-(256 + scan + rows * 130 * 4) // 256) * 256
+    assert p["workspace_bytes"] == expect
+
+
 def _plan(idx, **kw):
     c = W.WORKLOADS[idx]
     return pa.plan(c.num_seqs, c.num_heads, c.num_kv_heads, c.head_size, c.block_size,
@@ -110,12 +121,17 @@ def _plan(idx, **kw):
 
 def test_planner_on_the_five_workloads():
     p1, p2, p3, p4, p5 = (_plan(i) for i in range(1, 6))
+    assert all(p["balanced"] == 0 for p in (p1, p2, p3, p4, p5))
     assert p1["num_partitions"] == 1 and p1["partition_pages"] == 16
     assert p2["num_partitions"] == 1 and p2["grid_ctas"] == 64 * 32
     assert p3["num_partitions"] == 1  # two waves of units; longest-first order
     assert p4["num_partitions"] == 1 and p4["grid_ctas"] == 256 * 8
     assert p5["num_partitions"] >= 4  # 64 (seq, kv head) units cannot fill 148 SMs
-    for p in (p1, p2, p3, p4, p5):
+    # balanced ranges on request: one wave of CTAs
+    q2, q3, q4 = (_plan(i, schedule="balanced") for i in (2, 3, 4))
+    for q in (q2, q3, q4):
+        assert q["balanced"] == 1 and q["grid_ctas"] == 3 * 148 and q["num_partitions"] == 0
+    for p in (p1, p2, p3, p4, p5, q2, q3, q4):
         assert p["smem_bytes"] <= 227 * 1024 and 2 <= p["stages"] <= 8
         P, PP = p["num_partitions"], p["partition_pages"]
     c5 = W.WORKLOADS[5]
@@ -133,6 +149,27 @@ def test_planner_splits_between_one_and_two_waves():
     # 1024 units (more than two waves) are not split.
     p = pa.plan(128, 32, 8, 128, 16, 16384, "bf16", num_sms=148)
     assert p["num_partitions"] == 1
+    assert pa.plan(128, 32, 8, 128, 16, 16384, "bf16", num_sms=148,
+                   schedule="partitioned") == p
+
+
+def test_balanced_schedule_limits():
+    # forced partitions or a shared prefix rule balanced ranges out
+    with pytest.raises(pa.PagedAttentionError):
+        pa.plan(64, 32, 8, 128, 16, 4096, "bf16", num_sms=148, schedule="balanced",
+                partition_pages=8)
+    with pytest.raises(pa.PagedAttentionError):
+        pa.plan(64, 32, 8, 128, 16, 4096, "bf16", num_sms=148, schedule="balanced",
+                shared_prefix_blocks=4)
+    # a tiny batch may ask for them
+    p = pa.plan(2, 8, 2, 64, 16, 40, "bf16", num_sms=148, schedule="balanced")
+    assert p["balanced"] == 1 and p["grid_ctas"] == 3 * 148
+    # e4m3 MMAs: two CTAs per SM
+    p = pa.plan(256, 32, 8, 128, 16, 16384, "fp8_e4m3", num_sms=148, fp8_compute=True,
+                schedule="balanced")
+    assert p["balanced"] == 1 and p["grid_ctas"] == 2 * 148
+    with pytest.raises(ValueError):
+        pa.plan(4, 8, 2, 64, 16, 40, "bf16", num_sms=148, schedule="sometimes")
 
 
 def test_forced_partitions():
@@ -158,6 +195,8 @@ def test_every_plan_fits_shared_memory():
                         for pp in (0, 1, 2, 3, 5, 16, 64):
                             p = pa.plan(4, 2 * G, 2, D, B, T, kv, partition_pages=pp, num_sms=148)
                             assert p["smem_bytes"] <= 227 * 1024 - 256, (D, B, kv, G, T, pp)
+                        p = pa.plan(4, 2 * G, 2, D, B, T, kv, num_sms=148, schedule="balanced")
+                        assert p["smem_bytes"] <= 227 * 1024 - 256, (D, B, kv, G, T)
 
 
 def test_alibi_with_shared_prefix_is_refused(L):

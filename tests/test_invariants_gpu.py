@@ -38,11 +38,15 @@ def _token_slot(wl, s, t):
 
 @pytest.mark.parametrize("kv", [W.BF16, W.FP8_E4M3, "fp8_compute"])
 @pytest.mark.parametrize("D,B", [(128, 16), (64, 32), (128, 32)])
-@pytest.mark.parametrize("pp", [0, 2])
+@pytest.mark.parametrize("pp", [0, 2, "balanced"])
 def test_one_hot_probe_bit_exact(kv, D, B, pp):
     f8c = kv == "fp8_compute"
     if f8c:
         kv = W.FP8_E4M3
+    # "balanced": one wave of CTAs over equal page ranges; this tiny batch gets
+    # about one page per CTA, so every unit is cut and merged by the combine.
+    schedule = "balanced" if pp == "balanced" else "auto"
+    pp = 0 if pp == "balanced" else pp
     lens = (3 * B + 5, B, 1, 7 * B - 1)
     cfg = _cfg(D=D, B=B, G=4, kv=kv, lens=lens)
     wl = W.make_workload(cfg, DEV, seq_lens=list(lens))
@@ -66,9 +70,9 @@ def test_one_hot_probe_bit_exact(kv, D, B, pp):
                 out = torch.empty_like(wl.query)
                 pa.decode(out, wl.query, kc, wl.value_cache, cfg.num_kv_heads, cfg.scale,
                           wl.block_tables, wl.seq_lens, B, cfg.max_seq_len, kv, wl.k_scale,
-                          wl.v_scale, partition_pages=pp, fp8_compute=True)
+                          wl.v_scale, partition_pages=pp, fp8_compute=True, schedule=schedule)
             else:
-                out = run_gpu(wl, partition_pages=pp)
+                out = run_gpu(wl, partition_pages=pp, schedule=schedule)
             torch.cuda.synchronize()
             for g in range(cfg.num_kv_heads):
                 v = wl.value_cache[pb, g, :, o]
