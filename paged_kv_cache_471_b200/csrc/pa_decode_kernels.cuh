@@ -286,643 +286,652 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
     int issue_stage = 0;
 
     for (;;) {  // one segment per pass (a single pass unless balanced)
-    const bool cascade = p.prefix_pages > 0;
-    const int pg0 = pre ? 0 : p.prefix_pages;  // first page of this unit's page range
-    const int j0 = p.balanced ? bj : pg0 + part * p.PP;
-    const long long row0 = (long long)s * p.Hq + (long long)kvh * p.G;  // first q head row
-    const int rows_total = p.S * p.G;  // query rows of one kv head (prefix units)
+        const bool cascade = p.prefix_pages > 0;
+        const int pg0 = pre ? 0 : p.prefix_pages;  // first page of this unit's page range
+        const int j0 = p.balanced ? bj : pg0 + part * p.PP;
+        const long long row0 = (long long)s * p.Hq + (long long)kvh * p.G;  // first q head row
+        const int rows_total = p.S * p.G;  // query rows of one kv head (prefix units)
 
-    // Query row (s*Hq + head) of local row lr = 8r + gq, or -1 when unused.
-    auto row_of = [&](int lr) -> long long {
-        if (pre) {
-            const int gi = rg * 16 + lr;
-            if (gi >= rows_total) return -1;
-            return (long long)(gi / p.G) * p.Hq + (long long)kvh * p.G + gi % p.G;
-        }
-        return lr < p.G ? row0 + lr : -1;
-    };
+        // Query row (s*Hq + head) of local row lr = 8r + gq, or -1 when unused.
+        auto row_of = [&](int lr) -> long long {
+            if (pre) {
+                const int gi = rg * 16 + lr;
+                if (gi >= rows_total) return -1;
+                return (long long)(gi / p.G) * p.Hq + (long long)kvh * p.G + gi % p.G;
+            }
+            return lr < p.G ? row0 + lr : -1;
+        };
 
-    // Loads that do not depend on the sequence length go out first, so their
-    // latencies overlap: the block-table window (every entry of the row up to
-    // the partition's end is readable), the raw query words and the scales.
-    // Block-table window: lane l holds the id of this warp's page (wbase + l).
-    const int32_t* btrow = p.bt + (long long)s * p.max_blocks;
-    const int jcap = p.balanced ? min(bj + bn, p.max_blocks)
-                                : min(j0 + p.PP, pre ? p.prefix_pages : p.max_blocks);
-    auto load_win = [&](int base) -> int {
-        const int j = j0 + warp + W * (base + lane);
-        return j < jcap ? __ldg(btrow + j) : -1;
-    };
-    int win_a = load_win(0);
-    int win_b = load_win(32);
-    // Raw query words of rows 8r + gq, in the order the fragments use.
-    uint32_t qraw[2][KT][2];
+        // Loads that do not depend on the sequence length go out first, so their
+        // latencies overlap: the block-table window (every entry of the row up to
+        // the partition's end is readable), the raw query words and the scales.
+        // Block-table window: lane l holds the id of this warp's page (wbase + l).
+        const int32_t* btrow = p.bt + (long long)s * p.max_blocks;
+        const int jcap = p.balanced ? min(bn, p.max_blocks)
+                                    : min(j0 + p.PP, pre ? p.prefix_pages : p.max_blocks);
+        auto load_win = [&](int base) -> int {
+            const int j = j0 + warp + W * (base + lane);
+            return j < jcap ? __ldg(btrow + j) : -1;
+        };
+        int win_a = load_win(0);
+        int win_b = load_win(32);
+        // Raw query words of rows 8r + gq, in the order the fragments use.
+        uint32_t qraw[2][KT][2];
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        const long long qr = (r < NH) ? row_of(8 * r + gq) : -1;
-        const bool ok = qr >= 0;
-        const uint16_t* qrow = p.q + (ok ? qr : 0) * D;
+        for (int r = 0; r < 2; ++r) {
+            const long long qr = (r < NH) ? row_of(8 * r + gq) : -1;
+            const bool ok = qr >= 0;
+            const uint16_t* qrow = p.q + (ok ? qr : 0) * D;
 #pragma unroll
-        for (int kt = 0; kt < KT; ++kt) {
-            uint32_t w0 = 0, w1 = 0;
-            if (ok) {
-                if constexpr (!FP8) {
-                    w0 = __ldg(reinterpret_cast<const unsigned int*>(qrow + 16 * kt + 2 * cq));
-                    w1 = __ldg(reinterpret_cast<const unsigned int*>(qrow + 16 * kt + 8 + 2 * cq));
-                } else {
-                    const uint2 w = __ldg(reinterpret_cast<const uint2*>(qrow + 16 * kt + 4 * cq));
-                    w0 = w.x;
-                    w1 = w.y;
+            for (int kt = 0; kt < KT; ++kt) {
+                uint32_t w0 = 0, w1 = 0;
+                if (ok) {
+                    if constexpr (!FP8) {
+                        const unsigned int* qw = reinterpret_cast<const unsigned int*>(qrow);
+                        w0 = __ldg(qw + 8 * kt + cq);
+                        w1 = __ldg(qw + 8 * kt + 4 + cq);
+                    } else {
+                        const uint2 w =
+                            __ldg(reinterpret_cast<const uint2*>(qrow + 16 * kt + 4 * cq));
+                        w0 = w.x;
+                        w1 = w.y;
+                    }
                 }
-            }
-            qraw[r][kt][0] = w0;
-            qraw[r][kt][1] = w1;
-        }
-    }
-    float k_scale = 1.f, v_scale = 1.f;
-    if constexpr (FP8) {
-        k_scale = __ldg(p.k_scale);
-        v_scale = __ldg(p.v_scale);
-    }
-    // ALiBi: logit of token t gains slope * (t - (T - 1)); kept in log2 units.
-    const bool has_alibi = p.alibi != nullptr;
-    float slope2[NH];
-#pragma unroll
-    for (int r = 0; r < NH; ++r) {
-        const long long qr = row_of(8 * r + gq);
-        slope2[r] = (has_alibi && qr >= 0) ? __ldg(p.alibi + qr % p.Hq) * 1.4426950408889634f : 0.f;
-    }
-
-    // ---- sequence length, with the device-side range checks
-    int T, nb;
-    if (pre) {
-        nb = p.prefix_pages;  // every prefix page is full
-        T = nb * B;
-    } else {
-        T = __ldg(p.seq_lens + s);
-        uint32_t bad = 0;
-        if (T < 0) { T = 0; bad = kDevSeqLen; }
-        if (T > t_cap) { T = t_cap; bad = kDevSeqLen; }
-        nb = (T + B - 1) / B;
-        const int covered = p.balanced ? nb : pg0 + p.P * p.PP;
-        if (nb > covered) { nb = covered; T = nb * B; bad = kDevSeqLen; }
-        if (cascade && T < p.prefix_pages * B) bad |= kDevPrefix;
-        if (bad && part == 0 && kvh == 0 && j0 == pg0 && threadIdx.x == 0) atomicOr(p.status, bad);
-        if (cascade && part == 0 && kvh == 0 && warp == 0 && s > 0) {
-            // The declared prefix must be the same physical blocks as row 0's.
-            bool same = true;
-            for (int j = lane; j < p.prefix_pages; j += 32)
-                same &= __ldg(btrow + j) == __ldg(p.bt + j);
-            if (!__all_sync(kFull, same) && lane == 0) atomicOr(p.status, kDevPrefix);
-        }
-    }
-
-    // Balanced: the segment ends with the unit or with the CTA's range.
-    const int j1 = p.balanced ? static_cast<int>(min(static_cast<long long>(nb), j0 + (bx_end - bx)))
-                              : min(nb, j0 + p.PP);
-    const bool direct = !cascade && (p.balanced ? (j0 == 0 && j1 == nb)
-                                                : ((p.P == 1) || (nb <= p.PP)));
-
-    if (j0 >= j1) {
-        if (!cascade && part == 0) {  // empty sequence: defined as a zero output row
-            for (int i = threadIdx.x; i < p.G * D; i += (W * 32))
-                p.out[row0 * D + i] = __float2bfloat16_rn(0.f);
-        }
-        return;
-    }
-
-    const int span = j1 - j0;
-    const int n_my = span > warp ? (span - warp + W - 1) / W : 0;
-
-    int wbase = 0;
-    uint32_t valid_mask = 0;  // bit per stage: the page in it had a legal block id
-
-    const size_t head_off = static_cast<size_t>(kvh) * PAGE;
-    const size_t block_stride = static_cast<size_t>(p.Hk) * PAGE;
-
-    // Issue the copies of this warp's i-th page (warp-uniform call, pages in
-    // increasing order).  Pages go to consecutive stages of the ring, starting
-    // where the consumer stands; `issue_stage` tracks that without a division.
-    issue_stage = stage;
-    auto issue = [&](int i) {
-        if (i >= wbase + 32) {
-            win_a = win_b;
-            win_b = load_win(wbase + 64);
-            wbase += 32;
-        }
-        const int pb = __shfl_sync(kFull, win_a, i & 31);
-        const int stage = issue_stage;
-        issue_stage = (issue_stage + 1 == NS) ? 0 : issue_stage + 1;
-        const uint32_t bar = bar0 + 8 * stage;
-        const bool ok = pb >= 0 && static_cast<long long>(pb) < p.num_blocks;
-        if (lane == 0) {
-            if (ok) {
-                const size_t off = static_cast<size_t>(pb) * block_stride + head_off;
-                const uint32_t dst = wstage0 + static_cast<uint32_t>(stage * STAGE);
-                mbar_arrive_expect_tx(bar, STAGE + p.stall_tx_bytes);
-                bulk_copy_g2s(dst, p.kc + off, PAGE, bar);
-                bulk_copy_g2s(dst + PAGE, p.vc + off, PAGE, bar);
-            } else {
-                mbar_arrive(bar);
-                atomicOr(p.status, kDevBadBlock);
+                qraw[r][kt][0] = w0;
+                qraw[r][kt][1] = w1;
             }
         }
-        valid_mask = ok ? (valid_mask | (1u << stage)) : (valid_mask & ~(1u << stage));
-    };
-
-    const int n_pro = n_my < NS ? n_my : NS;
-    for (int i = 0; i < n_pro; ++i) issue(i);
-
-    // ---- Q fragments (A operand of S = Q K^T; rows = heads 8r + gq)
-    uint32_t qa[F8MMA ? 1 : KT][4];
-    uint32_t qa8[F8MMA ? K32 : 1][2][4];  // e4m3 MMAs: [k-step][hi, lo][regs]
-    float qk_mul = p.scale_log2;
-    float out_mul = 1.f;
-    if constexpr (F8MMA) {
-        // e4m3 operands: q is scaled by 2^e so that max|q| 2^e < 256, then
-        // split into hi + lo e4m3 codes (about 2^-8 relative together); both
-        // halves multiply the same K bytes, so one accumulator takes both.
-        // Natural d order: register i holds d = 32 jp + 16 (i >> 1) + 4 cq + 0..3.
-        float amax = 0.f;
-#pragma unroll
-        for (int r = 0; r < 2; ++r)
-#pragma unroll
-            for (int kt = 0; kt < KT; ++kt) {
-                const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
-                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(w0)), fabsf(bf16_hi(w0))),
-                                         fmaxf(fabsf(bf16_lo(w1)), fabsf(bf16_hi(w1)))));
-            }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
-        int e = 0;
-        if (amax > 0.f && amax < INFINITY)
-            e = 7 - (static_cast<int>((__float_as_uint(amax) >> 23) & 0xff) - 127);
-        e = max(-100, min(100, e));
-        const float up = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
-        const float down = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
-#pragma unroll
-        for (int jp = 0; jp < K32; ++jp)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = i & 1, kt = 2 * jp + (i >> 1);
-                if (r >= NH) {  // rows 8..15 unused: zero codes
-                    qa8[jp][0][i] = 0u;
-                    qa8[jp][1][i] = 0u;
-                    continue;
-                }
-                const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
-                float unused;
-                const uint32_t a = split_e4m3x2(bf16_lo(w0) * up, bf16_hi(w0) * up, &unused);
-                const uint32_t b = split_e4m3x2(bf16_lo(w1) * up, bf16_hi(w1) * up, &unused);
-                qa8[jp][0][i] = __byte_perm(a, b, 0x5410);  // hi codes of d .. d+3
-                qa8[jp][1][i] = __byte_perm(a, b, 0x7632);  // lo codes
-            }
-        qk_mul = p.scale_log2 * k_scale * down;
-        out_mul = v_scale;
-    } else if constexpr (!FP8) {
-#pragma unroll
-        for (int r = 0; r < 2; ++r)
-#pragma unroll
-            for (int kt = 0; kt < KT; ++kt) {
-                qa[kt][r] = qraw[r][kt][0];
-                qa[kt][r + 2] = qraw[r][kt][1];
-            }
-    } else {
-        // f16 operands: q is scaled by 2^-e so that max|q| < 2^15 (f16 range);
-        // 2^e goes back into the logit multiplier.  Within each 16-wide chunk the
-        // k order is permuted to match the e4m3 byte order delivered by ldmatrix:
-        // k = 2c,2c+1 <-> d = 4c,4c+1 and k = 2c+8,2c+9 <-> d = 4c+2,4c+3.
-        float amax = 0.f;
-#pragma unroll
-        for (int r = 0; r < 2; ++r)
-#pragma unroll
-            for (int kt = 0; kt < KT; ++kt) {
-                const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
-                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(w0)), fabsf(bf16_hi(w0))),
-                                         fmaxf(fabsf(bf16_lo(w1)), fabsf(bf16_hi(w1)))));
-            }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
-        int ex = 0;
-        if (amax > 0.f && amax < INFINITY) ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xff) - 127;
-        const int e = ex > 14 ? ex - 14 : 0;
-        const float down = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
-        const float up = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
-#pragma unroll
-        for (int r = 0; r < 2; ++r)
-#pragma unroll
-            for (int kt = 0; kt < KT; ++kt) {
-                const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
-                qa[kt][r] = pack_f16x2(bf16_lo(w0) * down, bf16_hi(w0) * down);
-                qa[kt][r + 2] = pack_f16x2(bf16_lo(w1) * down, bf16_hi(w1) * down);
-            }
-        qk_mul = p.scale_log2 * k_scale * up;
-        out_mul = v_scale;
-    }
-
-    float m_run[NH], l_run[NH];
-    float acc[MT][NH][4];
-#pragma unroll
-    for (int r = 0; r < NH; ++r) {
-        m_run[r] = -INFINITY;
-        l_run[r] = 0.f;
-    }
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-        for (int r = 0; r < NH; ++r)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[mt][r][e] = 0.f;
-
-    const int quad0 = lane & ~3;
-    const int src0 = quad0 | ((2 * cq) & 3);
-    const int src1 = quad0 | ((2 * cq + 1) & 3);
-    const bool hi_half = cq >= 2;
-
-    // One landed page: S = Q K^T, online softmax, O^T += V^T P^T.  FULL pages
-    // (every slot a token) skip all masking.
-    auto page = [&](auto full_tag, auto alibi_tag, const uint32_t kbase, const int valid,
-                    const int pos0) {
-        constexpr bool FULL = decltype(full_tag)::value;
-        constexpr bool ALIBI = decltype(alibi_tag)::value;
-        const uint32_t vbase = kbase + PAGE;
-
-        // ---------------- S = Q K^T  (rows: heads, cols: tokens)
-        float sc[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
-        {
-            const int mi = lane >> 3, r8 = lane & 7;
-            if constexpr (!FP8) {
-#pragma unroll
-                for (int kt = 0; kt < KT; ++kt)
-#pragma unroll
-                    for (int np = 0; np < NT / 2; ++np) {
-                        const int tok = 8 * (2 * np + (mi >> 1)) + r8;
-                        const int chunk = 2 * kt + (mi & 1);
-                        uint32_t b0, b1, b2, b3;
-                        ldsm_x4(kbase + chunk * CHUNK + tok * 16, b0, b1, b2, b3);
-                        mma_bf16_16816(sc[2 * np], qa[kt], b0, b1);
-                        mma_bf16_16816(sc[2 * np + 1], qa[kt], b2, b3);
-                    }
-            } else if constexpr (F8MMA) {
-                // K bytes go into the MMA as they are: register = 4 e4m3 codes of
-                // d = 4 cq..4 cq+3 of a 16-d chunk of one token.
-#pragma unroll
-                for (int jp = 0; jp < K32; ++jp)
-#pragma unroll
-                    for (int np = 0; np < NT / 2; ++np) {
-                        const int tok = 8 * (2 * np + (mi & 1)) + r8;
-                        const int chunk = 2 * jp + (mi >> 1);
-                        uint32_t w0, w1, w2, w3;
-                        ldsm_x4(kbase + chunk * CHUNK + tok * 16, w0, w1, w2, w3);
-                        mma_e4m3_16832(sc[2 * np], qa8[jp][0], w0, w2);
-                        mma_e4m3_16832(sc[2 * np], qa8[jp][1], w0, w2);
-                        mma_e4m3_16832(sc[2 * np + 1], qa8[jp][0], w1, w3);
-                        mma_e4m3_16832(sc[2 * np + 1], qa8[jp][1], w1, w3);
-                    }
-            } else {
-#pragma unroll
-                for (int jp = 0; jp < KT / 2; ++jp)
-#pragma unroll
-                    for (int np = 0; np < NT / 2; ++np) {
-                        const int tok = 8 * (2 * np + (mi & 1)) + r8;
-                        const int chunk = 2 * jp + (mi >> 1);
-                        uint32_t w0, w1, w2, w3;
-                        ldsm_x4(kbase + chunk * CHUNK + tok * 16, w0, w1, w2, w3);
-                        mma_f16_16816(sc[2 * np], qa[2 * jp], e4m3_lo_pair(w0), e4m3_hi_pair(w0));
-                        mma_f16_16816(sc[2 * np + 1], qa[2 * jp], e4m3_lo_pair(w1), e4m3_hi_pair(w1));
-                        mma_f16_16816(sc[2 * np], qa[2 * jp + 1], e4m3_lo_pair(w2), e4m3_hi_pair(w2));
-                        mma_f16_16816(sc[2 * np + 1], qa[2 * jp + 1], e4m3_lo_pair(w3),
-                                      e4m3_hi_pair(w3));
-                    }
-            }
+        float k_scale = 1.f, v_scale = 1.f;
+        if constexpr (FP8) {
+            k_scale = __ldg(p.k_scale);
+            v_scale = __ldg(p.v_scale);
         }
-
-        // ---------------- online softmax (log2 domain), per head row
-        uint32_t pp[NH][NT];
-        float alpha[NH];
-        bool grew = false;
+        // ALiBi: logit of token t gains slope * (t - (T - 1)); kept in log2 units.
+        const bool has_alibi = p.alibi != nullptr;
+        float slope2[NH];
 #pragma unroll
         for (int r = 0; r < NH; ++r) {
-            float v[NT][2];
-            float mx = -INFINITY;
+            const long long qr = row_of(8 * r + gq);
+            slope2[r] =
+                (has_alibi && qr >= 0) ? __ldg(p.alibi + qr % p.Hq) * 1.4426950408889634f : 0.f;
+        }
+
+        // ---- sequence length, with the device-side range checks
+        int T, nb;
+        if (pre) {
+            nb = p.prefix_pages;  // every prefix page is full
+            T = nb * B;
+        } else {
+            T = __ldg(p.seq_lens + s);
+            uint32_t bad = 0;
+            if (T < 0) { T = 0; bad = kDevSeqLen; }
+            if (T > t_cap) { T = t_cap; bad = kDevSeqLen; }
+            nb = (T + B - 1) / B;
+            const int covered = p.balanced ? nb : pg0 + p.P * p.PP;
+            if (nb > covered) { nb = covered; T = nb * B; bad = kDevSeqLen; }
+            if (cascade && T < p.prefix_pages * B) bad |= kDevPrefix;
+            if (bad && part == 0 && kvh == 0 && j0 == pg0 && threadIdx.x == 0)
+                atomicOr(p.status, bad);
+            if (cascade && part == 0 && kvh == 0 && warp == 0 && s > 0) {
+                // The declared prefix must be the same physical blocks as row 0's.
+                bool same = true;
+                for (int j = lane; j < p.prefix_pages; j += 32)
+                    same &= __ldg(btrow + j) == __ldg(p.bt + j);
+                if (!__all_sync(kFull, same) && lane == 0) atomicOr(p.status, kDevPrefix);
+            }
+        }
+
+        // Balanced: the segment ends with the unit or with the CTA's range.
+        const int j1 = p.balanced
+                           ? static_cast<int>(min(static_cast<long long>(nb), j0 + (bx_end - bx)))
+                           : min(nb, j0 + p.PP);
+        const bool direct = !cascade && (p.balanced ? (j0 == 0 && j1 == nb)
+                                                    : ((p.P == 1) || (nb <= p.PP)));
+
+        if (j0 >= j1) {
+            if (!cascade && part == 0) {  // empty sequence: defined as a zero output row
+                for (int i = threadIdx.x; i < p.G * D; i += (W * 32))
+                    p.out[row0 * D + i] = __float2bfloat16_rn(0.f);
+            }
+            return;
+        }
+
+        const int span = j1 - j0;
+        const int n_my = span > warp ? (span - warp + W - 1) / W : 0;
+
+        int wbase = 0;
+        uint32_t valid_mask = 0;  // bit per stage: the page in it had a legal block id
+
+        const size_t head_off = static_cast<size_t>(kvh) * PAGE;
+        const size_t block_stride = static_cast<size_t>(p.Hk) * PAGE;
+
+        // Issue the copies of this warp's i-th page (warp-uniform call, pages in
+        // increasing order).  Pages go to consecutive stages of the ring, starting
+        // where the consumer stands; `issue_stage` tracks that without a division.
+        issue_stage = stage;
+        auto issue = [&](int i) {
+            if (i >= wbase + 32) {
+                win_a = win_b;
+                win_b = load_win(wbase + 64);
+                wbase += 32;
+            }
+            const int pb = __shfl_sync(kFull, win_a, i & 31);
+            const int stage = issue_stage;
+            issue_stage = (issue_stage + 1 == NS) ? 0 : issue_stage + 1;
+            const uint32_t bar = bar0 + 8 * stage;
+            const bool ok = pb >= 0 && static_cast<long long>(pb) < p.num_blocks;
+            if (lane == 0) {
+                if (ok) {
+                    const size_t off = static_cast<size_t>(pb) * block_stride + head_off;
+                    const uint32_t dst = wstage0 + static_cast<uint32_t>(stage * STAGE);
+                    mbar_arrive_expect_tx(bar, STAGE + p.stall_tx_bytes);
+                    bulk_copy_g2s(dst, p.kc + off, PAGE, bar);
+                    bulk_copy_g2s(dst + PAGE, p.vc + off, PAGE, bar);
+                } else {
+                    mbar_arrive(bar);
+                    atomicOr(p.status, kDevBadBlock);
+                }
+            }
+            valid_mask = ok ? (valid_mask | (1u << stage)) : (valid_mask & ~(1u << stage));
+        };
+
+        const int n_pro = n_my < NS ? n_my : NS;
+        for (int i = 0; i < n_pro; ++i) issue(i);
+
+        // ---- Q fragments (A operand of S = Q K^T; rows = heads 8r + gq)
+        uint32_t qa[F8MMA ? 1 : KT][4];
+        uint32_t qa8[F8MMA ? K32 : 1][2][4];  // e4m3 MMAs: [k-step][hi, lo][regs]
+        float qk_mul = p.scale_log2;
+        float out_mul = 1.f;
+        if constexpr (F8MMA) {
+            // e4m3 operands: q is scaled by 2^e so that max|q| 2^e < 256, then
+            // split into hi + lo e4m3 codes (about 2^-8 relative together); both
+            // halves multiply the same K bytes, so one accumulator takes both.
+            // Natural d order: register i holds d = 32 jp + 16 (i >> 1) + 4 cq + 0..3.
+            float amax = 0.f;
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int kt = 0; kt < KT; ++kt) {
+                    const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
+                    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(w0)), fabsf(bf16_hi(w0))),
+                                             fmaxf(fabsf(bf16_lo(w1)), fabsf(bf16_hi(w1)))));
+                }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+            int e = 0;
+            if (amax > 0.f && amax < INFINITY)
+                e = 7 - (static_cast<int>((__float_as_uint(amax) >> 23) & 0xff) - 127);
+            e = max(-100, min(100, e));
+            const float up = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+            const float down = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+#pragma unroll
+            for (int jp = 0; jp < K32; ++jp)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = i & 1, kt = 2 * jp + (i >> 1);
+                    if (r >= NH) {  // rows 8..15 unused: zero codes
+                        qa8[jp][0][i] = 0u;
+                        qa8[jp][1][i] = 0u;
+                        continue;
+                    }
+                    const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
+                    float unused;
+                    const uint32_t a = split_e4m3x2(bf16_lo(w0) * up, bf16_hi(w0) * up, &unused);
+                    const uint32_t b = split_e4m3x2(bf16_lo(w1) * up, bf16_hi(w1) * up, &unused);
+                    qa8[jp][0][i] = __byte_perm(a, b, 0x5410);  // hi codes of d .. d+3
+                    qa8[jp][1][i] = __byte_perm(a, b, 0x7632);  // lo codes
+                }
+            qk_mul = p.scale_log2 * k_scale * down;
+            out_mul = v_scale;
+        } else if constexpr (!FP8) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int kt = 0; kt < KT; ++kt) {
+                    qa[kt][r] = qraw[r][kt][0];
+                    qa[kt][r + 2] = qraw[r][kt][1];
+                }
+        } else {
+            // f16 operands: q is scaled by 2^-e so that max|q| < 2^15 (f16 range);
+            // 2^e goes back into the logit multiplier.  Within each 16-wide chunk the
+            // k order is permuted to match the e4m3 byte order delivered by ldmatrix:
+            // k = 2c,2c+1 <-> d = 4c,4c+1 and k = 2c+8,2c+9 <-> d = 4c+2,4c+3.
+            float amax = 0.f;
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int kt = 0; kt < KT; ++kt) {
+                    const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
+                    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(w0)), fabsf(bf16_hi(w0))),
+                                             fmaxf(fabsf(bf16_lo(w1)), fabsf(bf16_hi(w1)))));
+                }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+            int ex = 0;
+            if (amax > 0.f && amax < INFINITY)
+                ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xff) - 127;
+            const int e = ex > 14 ? ex - 14 : 0;
+            const float down = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+            const float up = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int kt = 0; kt < KT; ++kt) {
+                    const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
+                    qa[kt][r] = pack_f16x2(bf16_lo(w0) * down, bf16_hi(w0) * down);
+                    qa[kt][r + 2] = pack_f16x2(bf16_lo(w1) * down, bf16_hi(w1) * down);
+                }
+            qk_mul = p.scale_log2 * k_scale * up;
+            out_mul = v_scale;
+        }
+
+        float m_run[NH], l_run[NH];
+        float acc[MT][NH][4];
+#pragma unroll
+        for (int r = 0; r < NH; ++r) {
+            m_run[r] = -INFINITY;
+            l_run[r] = 0.f;
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int r = 0; r < NH; ++r)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[mt][r][e] = 0.f;
+
+        const int quad0 = lane & ~3;
+        const int src0 = quad0 | ((2 * cq) & 3);
+        const int src1 = quad0 | ((2 * cq + 1) & 3);
+        const bool hi_half = cq >= 2;
+
+        // One landed page: S = Q K^T, online softmax, O^T += V^T P^T.  FULL pages
+        // (every slot a token) skip all masking.
+        auto page = [&](auto full_tag, auto alibi_tag, const uint32_t kbase, const int valid,
+                        const int pos0) {
+            constexpr bool FULL = decltype(full_tag)::value;
+            constexpr bool ALIBI = decltype(alibi_tag)::value;
+            const uint32_t vbase = kbase + PAGE;
+
+            // ---------------- S = Q K^T  (rows: heads, cols: tokens)
+            float sc[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    float x = sc[nt][2 * r + e] * qk_mul;
-                    if constexpr (ALIBI)
-                        x = fmaf(slope2[r], static_cast<float>(pos0 + 8 * nt + 2 * cq + e), x);
-                    if constexpr (!FULL) {
-                        if (8 * nt + 2 * cq + e >= valid) x = -INFINITY;
-                    }
-                    v[nt][e] = x;
-                    mx = fmaxf(mx, x);
-                }
-            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-            const float m_new = fmaxf(m_run[r], mx);
-            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-            grew |= m_new > m_run[r];
-            alpha[r] = fast_exp2(m_run[r] - m_use);
-            m_run[r] = m_new;
-            float ls = 0.f;
+                for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
+            {
+                const int mi = lane >> 3, r8 = lane & 7;
+                if constexpr (!FP8) {
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const float p0 = fast_exp2(v[nt][0] - m_use);
-                const float p1 = fast_exp2(v[nt][1] - m_use);
-                uint32_t w;
-                if constexpr (F8MMA) {
-                    // weights x 256 as hi + lo e4m3 codes (hi pair | lo pair << 16);
-                    // the running sum uses the represented values, in the same x 256
-                    // units as the accumulator.
-                    float sum2;
-                    w = split_e4m3x2(p0 * 256.f, p1 * 256.f, &sum2);
-                    ls += sum2;
-                } else if constexpr (!FP8) {
-                    w = pack_bf16x2(p0, p1);
-                    ls += bf16_lo(w) + bf16_hi(w);
+                    for (int kt = 0; kt < KT; ++kt)
+#pragma unroll
+                        for (int np = 0; np < NT / 2; ++np) {
+                            const int tok = 8 * (2 * np + (mi >> 1)) + r8;
+                            const int chunk = 2 * kt + (mi & 1);
+                            uint32_t b0, b1, b2, b3;
+                            ldsm_x4(kbase + chunk * CHUNK + tok * 16, b0, b1, b2, b3);
+                            mma_bf16_16816(sc[2 * np], qa[kt], b0, b1);
+                            mma_bf16_16816(sc[2 * np + 1], qa[kt], b2, b3);
+                        }
+                } else if constexpr (F8MMA) {
+                    // K bytes go into the MMA as they are: register = 4 e4m3 codes of
+                    // d = 4 cq..4 cq+3 of a 16-d chunk of one token.
+#pragma unroll
+                    for (int jp = 0; jp < K32; ++jp)
+#pragma unroll
+                        for (int np = 0; np < NT / 2; ++np) {
+                            const int tok = 8 * (2 * np + (mi & 1)) + r8;
+                            const int chunk = 2 * jp + (mi >> 1);
+                            uint32_t w0, w1, w2, w3;
+                            ldsm_x4(kbase + chunk * CHUNK + tok * 16, w0, w1, w2, w3);
+                            mma_e4m3_16832(sc[2 * np], qa8[jp][0], w0, w2);
+                            mma_e4m3_16832(sc[2 * np], qa8[jp][1], w0, w2);
+                            mma_e4m3_16832(sc[2 * np + 1], qa8[jp][0], w1, w3);
+                            mma_e4m3_16832(sc[2 * np + 1], qa8[jp][1], w1, w3);
+                        }
                 } else {
-                    w = pack_f16x2(p0, p1);
-                    ls += f16_lo(w) + f16_hi(w);
+#pragma unroll
+                    for (int jp = 0; jp < KT / 2; ++jp)
+#pragma unroll
+                        for (int np = 0; np < NT / 2; ++np) {
+                            const int tok = 8 * (2 * np + (mi & 1)) + r8;
+                            const int chunk = 2 * jp + (mi >> 1);
+                            uint32_t w0, w1, w2, w3;
+                            ldsm_x4(kbase + chunk * CHUNK + tok * 16, w0, w1, w2, w3);
+                            const uint32_t(&qlo)[4] = qa[2 * jp];
+                            const uint32_t(&qhi)[4] = qa[2 * jp + 1];
+                            mma_f16_16816(sc[2 * np], qlo, e4m3_lo_pair(w0), e4m3_hi_pair(w0));
+                            mma_f16_16816(sc[2 * np + 1], qlo, e4m3_lo_pair(w1), e4m3_hi_pair(w1));
+                            mma_f16_16816(sc[2 * np], qhi, e4m3_lo_pair(w2), e4m3_hi_pair(w2));
+                            mma_f16_16816(sc[2 * np + 1], qhi, e4m3_lo_pair(w3), e4m3_hi_pair(w3));
+                        }
                 }
-                pp[r][nt] = w;
             }
-            l_run[r] = l_run[r] * alpha[r] + ls;
-        }
 
-        // ---------------- rescale O^T columns (heads 8r + 2cq, 8r + 2cq + 1),
-        // only when some row maximum of the warp moved.
-        if (__any_sync(kFull, grew)) {
+            // ---------------- online softmax (log2 domain), per head row
+            uint32_t pp[NH][NT];
+            float alpha[NH];
+            bool grew = false;
 #pragma unroll
             for (int r = 0; r < NH; ++r) {
-                const float a0 = __shfl_sync(kFull, alpha[r], 8 * cq);
-                const float a1 = __shfl_sync(kFull, alpha[r], 8 * cq + 4);
+                float v[NT][2];
+                float mx = -INFINITY;
 #pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    acc[mt][r][0] *= a0;
-                    acc[mt][r][1] *= a1;
-                    acc[mt][r][2] *= a0;
-                    acc[mt][r][3] *= a1;
-                }
-            }
-        }
-
-        if constexpr (F8MMA) {
-            // O^T += V^T P^T with one 32-token e4m3 k-step per page: tokens
-            // 16 kk + 4 cq .. +3 of each k-tile come from the same quad shuffles
-            // as below; V bytes go into the MMA as they are.  Block size 16
-            // leaves the upper 16 tokens of the step empty (zeros).
-            uint32_t bh[NH][2], bl[NH][2];
+                for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int kk = 0; kk < 2; ++kk)
+                    for (int e = 0; e < 2; ++e) {
+                        float x = sc[nt][2 * r + e] * qk_mul;
+                        if constexpr (ALIBI)
+                            x = fmaf(slope2[r], static_cast<float>(pos0 + 8 * nt + 2 * cq + e), x);
+                        if constexpr (!FULL) {
+                            if (8 * nt + 2 * cq + e >= valid) x = -INFINITY;
+                        }
+                        v[nt][e] = x;
+                        mx = fmaxf(mx, x);
+                    }
+                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+                const float m_new = fmaxf(m_run[r], mx);
+                const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+                grew |= m_new > m_run[r];
+                alpha[r] = fast_exp2(m_run[r] - m_use);
+                m_run[r] = m_new;
+                float ls = 0.f;
 #pragma unroll
-                for (int r = 0; r < NH; ++r) {
-                    if (kk < KK) {
-                        const uint32_t x0 = __shfl_sync(kFull, pp[r][2 * kk], src0);
-                        const uint32_t y0 = __shfl_sync(kFull, pp[r][2 * kk + 1], src0);
-                        const uint32_t x1 = __shfl_sync(kFull, pp[r][2 * kk], src1);
-                        const uint32_t y1 = __shfl_sync(kFull, pp[r][2 * kk + 1], src1);
-                        const uint32_t u0 = hi_half ? y0 : x0;  // tokens 4cq, 4cq+1
-                        const uint32_t u1 = hi_half ? y1 : x1;  // tokens 4cq+2, 4cq+3
-                        bh[r][kk] = __byte_perm(u0, u1, 0x5410);
-                        bl[r][kk] = __byte_perm(u0, u1, 0x7632);
+                for (int nt = 0; nt < NT; ++nt) {
+                    const float p0 = fast_exp2(v[nt][0] - m_use);
+                    const float p1 = fast_exp2(v[nt][1] - m_use);
+                    uint32_t w;
+                    if constexpr (F8MMA) {
+                        // weights x 256 as hi + lo e4m3 codes (hi pair | lo pair << 16);
+                        // the running sum uses the represented values, in the same x 256
+                        // units as the accumulator.
+                        float sum2;
+                        w = split_e4m3x2(p0 * 256.f, p1 * 256.f, &sum2);
+                        ls += sum2;
+                    } else if constexpr (!FP8) {
+                        w = pack_bf16x2(p0, p1);
+                        ls += bf16_lo(w) + bf16_hi(w);
                     } else {
-                        bh[r][kk] = 0u;
-                        bl[r][kk] = 0u;
+                        w = pack_f16x2(p0, p1);
+                        ls += f16_lo(w) + f16_hi(w);
                     }
+                    pp[r][nt] = w;
                 }
-            uint32_t vmask[2] = {kFull, kFull};
-            if constexpr (!FULL) {
-#pragma unroll
-                for (int kk = 0; kk < KK; ++kk) {
-                    const int t0 = 16 * kk + 4 * cq;
-                    vmask[kk] = (t0 < valid ? 0x000000ffu : 0u) | (t0 + 1 < valid ? 0x0000ff00u : 0u) |
-                                (t0 + 2 < valid ? 0x00ff0000u : 0u) | (t0 + 3 < valid ? 0xff000000u : 0u);
-                }
+                l_run[r] = l_run[r] * alpha[r] + ls;
             }
-#pragma unroll
-            for (int mp = 0; mp < MT / 2; ++mp) {
-                uint32_t w[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
-#pragma unroll
-                for (int kk = 0; kk < KK; ++kk) {
-                    ldsm_x4(vbase + (32 * mp + lane) * B + kk * 16, w[kk][0], w[kk][1], w[kk][2],
-                            w[kk][3]);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) w[kk][i] &= vmask[kk];
-                }
-                const uint32_t a0[4] = {w[0][0], w[0][1], w[1][0], w[1][1]};
-                const uint32_t a1[4] = {w[0][2], w[0][3], w[1][2], w[1][3]};
+
+            // ---------------- rescale O^T columns (heads 8r + 2cq, 8r + 2cq + 1),
+            // only when some row maximum of the warp moved.
+            if (__any_sync(kFull, grew)) {
 #pragma unroll
                 for (int r = 0; r < NH; ++r) {
-                    mma_e4m3_16832(acc[2 * mp][r], a0, bh[r][0], bh[r][1]);
-                    mma_e4m3_16832(acc[2 * mp][r], a0, bl[r][0], bl[r][1]);
-                    mma_e4m3_16832(acc[2 * mp + 1][r], a1, bh[r][0], bh[r][1]);
-                    mma_e4m3_16832(acc[2 * mp + 1][r], a1, bl[r][0], bl[r][1]);
+                    const float a0 = __shfl_sync(kFull, alpha[r], 8 * cq);
+                    const float a1 = __shfl_sync(kFull, alpha[r], 8 * cq + 4);
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        acc[mt][r][0] *= a0;
+                        acc[mt][r][1] *= a1;
+                        acc[mt][r][2] *= a0;
+                        acc[mt][r][3] *= a1;
+                    }
                 }
             }
-        } else {
-        // ---------------- O^T += V^T P^T  (rows: head dim, cols: heads, k: tokens)
-        // Per 16-token k-tile, thread cq holds V for tokens 4cq..4cq+3 (one
-        // contiguous 4-token group per row), so k = 2cq,2cq+1 <-> tokens
-        // 4cq,4cq+1 and k = 2cq+8,2cq+9 <-> 4cq+2,4cq+3; P is regrouped to
-        // that order with quad shuffles.
+
+            if constexpr (F8MMA) {
+                // O^T += V^T P^T with one 32-token e4m3 k-step per page: tokens
+                // 16 kk + 4 cq .. +3 of each k-tile come from the same quad shuffles
+                // as below; V bytes go into the MMA as they are.  Block size 16
+                // leaves the upper 16 tokens of the step empty (zeros).
+                uint32_t bh[NH][2], bl[NH][2];
 #pragma unroll
-        for (int kk = 0; kk < KK; ++kk) {
-            uint32_t pb0[NH], pb1[NH];
-#pragma unroll
-            for (int r = 0; r < NH; ++r) {
-                const uint32_t x0 = __shfl_sync(kFull, pp[r][2 * kk], src0);
-                const uint32_t y0 = __shfl_sync(kFull, pp[r][2 * kk + 1], src0);
-                const uint32_t x1 = __shfl_sync(kFull, pp[r][2 * kk], src1);
-                const uint32_t y1 = __shfl_sync(kFull, pp[r][2 * kk + 1], src1);
-                pb0[r] = hi_half ? y0 : x0;
-                pb1[r] = hi_half ? y1 : x1;
-            }
-            // Slots past the sequence end may hold anything (even NaN); their
-            // weights are 0, but 0 * NaN is NaN, so their V is zeroed.
-            uint32_t mlo = kFull, mhi = kFull;
-            if constexpr (!FULL) {
-                const int t0 = 16 * kk + 4 * cq;
-                mlo = (t0 < valid ? 0x0000ffffu : 0u) | (t0 + 1 < valid ? 0xffff0000u : 0u);
-                mhi = (t0 + 2 < valid ? 0x0000ffffu : 0u) | (t0 + 3 < valid ? 0xffff0000u : 0u);
-            }
-            if constexpr (!FP8) {
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    const uint32_t ra = vbase + (16 * mt + gq) * (B * 2) + kk * 32 + cq * 8;
-                    const uint2 va = lds64(ra);
-                    const uint2 vb = lds64(ra + 8 * (B * 2));
-                    uint32_t a[4] = {va.x, vb.x, va.y, vb.y};
-                    if constexpr (!FULL) {
-                        a[0] &= mlo;
-                        a[1] &= mlo;
-                        a[2] &= mhi;
-                        a[3] &= mhi;
-                    }
-#pragma unroll
-                    for (int r = 0; r < NH; ++r) mma_bf16_16816(acc[mt][r], a, pb0[r], pb1[r]);
-                }
-            } else {
-#pragma unroll
-                for (int mp = 0; mp < MT / 2; ++mp) {
-                    uint32_t w0, w1, w2, w3;
-                    ldsm_x4(vbase + (32 * mp + lane) * B + kk * 16, w0, w1, w2, w3);
-                    uint32_t a0[4] = {e4m3_lo_pair(w0), e4m3_lo_pair(w1), e4m3_hi_pair(w0),
-                                      e4m3_hi_pair(w1)};
-                    uint32_t a1[4] = {e4m3_lo_pair(w2), e4m3_lo_pair(w3), e4m3_hi_pair(w2),
-                                      e4m3_hi_pair(w3)};
-                    if constexpr (!FULL) {
-                        a0[0] &= mlo;
-                        a0[1] &= mlo;
-                        a0[2] &= mhi;
-                        a0[3] &= mhi;
-                        a1[0] &= mlo;
-                        a1[1] &= mlo;
-                        a1[2] &= mhi;
-                        a1[3] &= mhi;
-                    }
+                for (int kk = 0; kk < 2; ++kk)
 #pragma unroll
                     for (int r = 0; r < NH; ++r) {
-                        mma_f16_16816(acc[2 * mp][r], a0, pb0[r], pb1[r]);
-                        mma_f16_16816(acc[2 * mp + 1][r], a1, pb0[r], pb1[r]);
+                        if (kk < KK) {
+                            const uint32_t x0 = __shfl_sync(kFull, pp[r][2 * kk], src0);
+                            const uint32_t y0 = __shfl_sync(kFull, pp[r][2 * kk + 1], src0);
+                            const uint32_t x1 = __shfl_sync(kFull, pp[r][2 * kk], src1);
+                            const uint32_t y1 = __shfl_sync(kFull, pp[r][2 * kk + 1], src1);
+                            const uint32_t u0 = hi_half ? y0 : x0;  // tokens 4cq, 4cq+1
+                            const uint32_t u1 = hi_half ? y1 : x1;  // tokens 4cq+2, 4cq+3
+                            bh[r][kk] = __byte_perm(u0, u1, 0x5410);
+                            bl[r][kk] = __byte_perm(u0, u1, 0x7632);
+                        } else {
+                            bh[r][kk] = 0u;
+                            bl[r][kk] = 0u;
+                        }
+                    }
+                uint32_t vmask[2] = {kFull, kFull};
+                if constexpr (!FULL) {
+#pragma unroll
+                    for (int kk = 0; kk < KK; ++kk) {
+                        const int t0 = 16 * kk + 4 * cq;
+                        vmask[kk] = (t0 < valid ? 0x000000ffu : 0u) |
+                                    (t0 + 1 < valid ? 0x0000ff00u : 0u) |
+                                    (t0 + 2 < valid ? 0x00ff0000u : 0u) |
+                                    (t0 + 3 < valid ? 0xff000000u : 0u);
+                    }
+                }
+#pragma unroll
+                for (int mp = 0; mp < MT / 2; ++mp) {
+                    uint32_t w[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
+#pragma unroll
+                    for (int kk = 0; kk < KK; ++kk) {
+                        ldsm_x4(vbase + (32 * mp + lane) * B + kk * 16, w[kk][0], w[kk][1],
+                                w[kk][2], w[kk][3]);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) w[kk][i] &= vmask[kk];
+                    }
+                    const uint32_t a0[4] = {w[0][0], w[0][1], w[1][0], w[1][1]};
+                    const uint32_t a1[4] = {w[0][2], w[0][3], w[1][2], w[1][3]};
+#pragma unroll
+                    for (int r = 0; r < NH; ++r) {
+                        mma_e4m3_16832(acc[2 * mp][r], a0, bh[r][0], bh[r][1]);
+                        mma_e4m3_16832(acc[2 * mp][r], a0, bl[r][0], bl[r][1]);
+                        mma_e4m3_16832(acc[2 * mp + 1][r], a1, bh[r][0], bh[r][1]);
+                        mma_e4m3_16832(acc[2 * mp + 1][r], a1, bl[r][0], bl[r][1]);
+                    }
+                }
+            } else {
+            // ---------------- O^T += V^T P^T  (rows: head dim, cols: heads, k: tokens)
+            // Per 16-token k-tile, thread cq holds V for tokens 4cq..4cq+3 (one
+            // contiguous 4-token group per row), so k = 2cq,2cq+1 <-> tokens
+            // 4cq,4cq+1 and k = 2cq+8,2cq+9 <-> 4cq+2,4cq+3; P is regrouped to
+            // that order with quad shuffles.
+#pragma unroll
+            for (int kk = 0; kk < KK; ++kk) {
+                uint32_t pb0[NH], pb1[NH];
+#pragma unroll
+                for (int r = 0; r < NH; ++r) {
+                    const uint32_t x0 = __shfl_sync(kFull, pp[r][2 * kk], src0);
+                    const uint32_t y0 = __shfl_sync(kFull, pp[r][2 * kk + 1], src0);
+                    const uint32_t x1 = __shfl_sync(kFull, pp[r][2 * kk], src1);
+                    const uint32_t y1 = __shfl_sync(kFull, pp[r][2 * kk + 1], src1);
+                    pb0[r] = hi_half ? y0 : x0;
+                    pb1[r] = hi_half ? y1 : x1;
+                }
+                // Slots past the sequence end may hold anything (even NaN); their
+                // weights are 0, but 0 * NaN is NaN, so their V is zeroed.
+                uint32_t mlo = kFull, mhi = kFull;
+                if constexpr (!FULL) {
+                    const int t0 = 16 * kk + 4 * cq;
+                    mlo = (t0 < valid ? 0x0000ffffu : 0u) | (t0 + 1 < valid ? 0xffff0000u : 0u);
+                    mhi = (t0 + 2 < valid ? 0x0000ffffu : 0u) | (t0 + 3 < valid ? 0xffff0000u : 0u);
+                }
+                if constexpr (!FP8) {
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        const uint32_t ra = vbase + (16 * mt + gq) * (B * 2) + kk * 32 + cq * 8;
+                        const uint2 va = lds64(ra);
+                        const uint2 vb = lds64(ra + 8 * (B * 2));
+                        uint32_t a[4] = {va.x, vb.x, va.y, vb.y};
+                        if constexpr (!FULL) {
+                            a[0] &= mlo;
+                            a[1] &= mlo;
+                            a[2] &= mhi;
+                            a[3] &= mhi;
+                        }
+#pragma unroll
+                        for (int r = 0; r < NH; ++r) mma_bf16_16816(acc[mt][r], a, pb0[r], pb1[r]);
+                    }
+                } else {
+#pragma unroll
+                    for (int mp = 0; mp < MT / 2; ++mp) {
+                        uint32_t w0, w1, w2, w3;
+                        ldsm_x4(vbase + (32 * mp + lane) * B + kk * 16, w0, w1, w2, w3);
+                        uint32_t a0[4] = {e4m3_lo_pair(w0), e4m3_lo_pair(w1), e4m3_hi_pair(w0),
+                                          e4m3_hi_pair(w1)};
+                        uint32_t a1[4] = {e4m3_lo_pair(w2), e4m3_lo_pair(w3), e4m3_hi_pair(w2),
+                                          e4m3_hi_pair(w3)};
+                        if constexpr (!FULL) {
+                            a0[0] &= mlo;
+                            a0[1] &= mlo;
+                            a0[2] &= mhi;
+                            a0[3] &= mhi;
+                            a1[0] &= mlo;
+                            a1[1] &= mlo;
+                            a1[2] &= mhi;
+                            a1[3] &= mhi;
+                        }
+#pragma unroll
+                        for (int r = 0; r < NH; ++r) {
+                            mma_f16_16816(acc[2 * mp][r], a0, pb0[r], pb1[r]);
+                            mma_f16_16816(acc[2 * mp + 1][r], a1, pb0[r], pb1[r]);
+                        }
                     }
                 }
             }
-        }
-        }  // e4m3 MMAs or f16/bf16 MMAs
-    };
+            }  // e4m3 MMAs or f16/bf16 MMAs
+        };
 
-    bool timed_out = false;
-    int k = 0;
-    for (; k < n_my; ++k) {
-        const bool landed = mbar_wait_bounded(bar0 + 8 * stage, phase, p.wait_limit_ns);
-        if (!__all_sync(kFull, landed)) {
-            timed_out = true;
-            break;
-        }
-        const int jg = j0 + warp + W * k;
-        const int valid = ((valid_mask >> stage) & 1u) ? min(B, T - jg * B) : 0;
-        const uint32_t kbase = wstage0 + static_cast<uint32_t>(stage * STAGE);
-        const int pos0 = jg * B - (T - 1);  // ALiBi position of the page's first slot
-        if (!has_alibi) {
-            if (valid == B)
-                page(std::true_type{}, std::false_type{}, kbase, valid, pos0);
-            else
-                page(std::false_type{}, std::false_type{}, kbase, valid, pos0);
-        } else {
-            if (valid == B)
-                page(std::true_type{}, std::true_type{}, kbase, valid, pos0);
-            else
-                page(std::false_type{}, std::true_type{}, kbase, valid, pos0);
-        }
-        __syncwarp();
-        if (k + NS < n_my) issue(k + NS);
-        if (++stage == NS) {
-            stage = 0;
-            phase ^= 1u;
-        }
-    }
-
-    if (timed_out) {
-        // Let the copies already in flight land (bounded) before the CTA's
-        // shared memory can be handed to anyone else, then report.
-        const int last = min(n_my, k + NS);
-        for (int i = k; i < last; ++i) {
-            (void)mbar_wait_bounded(bar0 + 8 * stage, phase, p.wait_limit_ns);
+        bool timed_out = false;
+        int k = 0;
+        for (; k < n_my; ++k) {
+            const bool landed = mbar_wait_bounded(bar0 + 8 * stage, phase, p.wait_limit_ns);
+            if (!__all_sync(kFull, landed)) {
+                timed_out = true;
+                break;
+            }
+            const int jg = j0 + warp + W * k;
+            const int valid = ((valid_mask >> stage) & 1u) ? min(B, T - jg * B) : 0;
+            const uint32_t kbase = wstage0 + static_cast<uint32_t>(stage * STAGE);
+            const int pos0 = jg * B - (T - 1);  // ALiBi position of the page's first slot
+            if (!has_alibi) {
+                if (valid == B)
+                    page(std::true_type{}, std::false_type{}, kbase, valid, pos0);
+                else
+                    page(std::false_type{}, std::false_type{}, kbase, valid, pos0);
+            } else {
+                if (valid == B)
+                    page(std::true_type{}, std::true_type{}, kbase, valid, pos0);
+                else
+                    page(std::false_type{}, std::true_type{}, kbase, valid, pos0);
+            }
+            __syncwarp();
+            if (k + NS < n_my) issue(k + NS);
             if (++stage == NS) {
                 stage = 0;
                 phase ^= 1u;
             }
         }
-        if (lane == 0) atomicOr(p.status, kDevTimeout);
-    }
 
-    // ---------------- merge the four warps' partial softmax states
-#pragma unroll
-    for (int r = 0; r < NH; ++r) {
-        l_run[r] += __shfl_xor_sync(kFull, l_run[r], 1);
-        l_run[r] += __shfl_xor_sync(kFull, l_run[r], 2);
-    }
-    __syncthreads();  // every warp is done with its stages
-    float* s_acc = reinterpret_cast<float*>(smem);
-    float* s_m = s_acc + W * NH * 8 * RS;
-    float* s_l = s_m + W * 16;
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
+        if (timed_out) {
+            // Let the copies already in flight land (bounded) before the CTA's
+            // shared memory can be handed to anyone else, then report.
+            const int last = min(n_my, k + NS);
+            for (int i = k; i < last; ++i) {
+                (void)mbar_wait_bounded(bar0 + 8 * stage, phase, p.wait_limit_ns);
+                if (++stage == NS) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (lane == 0) atomicOr(p.status, kDevTimeout);
+        }
+
+        // ---------------- merge the four warps' partial softmax states
 #pragma unroll
         for (int r = 0; r < NH; ++r) {
-            const int h = 8 * r + 2 * cq;
-            const int d = 16 * mt + gq;
-            float* base = s_acc + (warp * NH * 8 + h) * RS + d;
-            base[0] = acc[mt][r][0];
-            base[RS] = acc[mt][r][1];
-            base[8] = acc[mt][r][2];
-            base[RS + 8] = acc[mt][r][3];
+            l_run[r] += __shfl_xor_sync(kFull, l_run[r], 1);
+            l_run[r] += __shfl_xor_sync(kFull, l_run[r], 2);
         }
-    if (cq == 0) {
+        __syncthreads();  // every warp is done with its stages
+        float* s_acc = reinterpret_cast<float*>(smem);
+        float* s_m = s_acc + W * NH * 8 * RS;
+        float* s_l = s_m + W * 16;
 #pragma unroll
-        for (int r = 0; r < NH; ++r) {
-            s_m[warp * 16 + 8 * r + gq] = m_run[r];
-            s_l[warp * 16 + 8 * r + gq] = timed_out ? 0.f : l_run[r];
-        }
-    }
-    __syncthreads();
-
-    const int rows_here = pre ? min(16, rows_total - rg * 16) : p.G;
-    const int slot = pre ? part : (cascade ? p.prefix_parts : 0) + part;
-    // Balanced: slot 2 c + k of this CTA, G rows (see DecodeParams).
-    const long long br_row0 =
-        (2LL * blockIdx.x + (bx == bx_first ? 0 : 1)) * static_cast<long long>(p.G);
-    for (int idx = threadIdx.x; idx < rows_here * D; idx += (W * 32)) {
-        const int h = idx / D;
-        const int d = idx - h * D;
-        float M = -INFINITY;
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-        for (int w = 0; w < W; ++w)
-            if (s_l[w * 16 + h] > 0.f) M = fmaxf(M, s_m[w * 16 + h]);
-        float L = 0.f, O = 0.f;
+            for (int r = 0; r < NH; ++r) {
+                const int h = 8 * r + 2 * cq;
+                const int d = 16 * mt + gq;
+                float* base = s_acc + (warp * NH * 8 + h) * RS + d;
+                base[0] = acc[mt][r][0];
+                base[RS] = acc[mt][r][1];
+                base[8] = acc[mt][r][2];
+                base[RS + 8] = acc[mt][r][3];
+            }
+        if (cq == 0) {
 #pragma unroll
-        for (int w = 0; w < W; ++w) {
-            const float l = s_l[w * 16 + h];
-            if (l > 0.f) {
-                const float wt = exp2f(s_m[w * 16 + h] - M);
-                L += wt * l;
-                O += wt * s_acc[(w * NH * 8 + h) * RS + d];
+            for (int r = 0; r < NH; ++r) {
+                s_m[warp * 16 + 8 * r + gq] = m_run[r];
+                s_l[warp * 16 + 8 * r + gq] = timed_out ? 0.f : l_run[r];
             }
         }
-        const float o = L > 0.f ? (O / L) * out_mul : 0.f;
-        const long long row = row_of(h);
-        if (direct) {
-            p.out[row * D + d] = __float2bfloat16_rn(o);
-        } else {
-            const long long prow = p.balanced ? br_row0 + h : row * p.P_total + slot;
-            p.ws_o[prow * D + d] = o;
-            if (d == 0) {
-                p.ws_m[prow] = M;
-                p.ws_l[prow] = L;
+        __syncthreads();
+
+        const int rows_here = pre ? min(16, rows_total - rg * 16) : p.G;
+        const int slot = pre ? part : (cascade ? p.prefix_parts : 0) + part;
+        // Balanced: slot 2 c + k of this CTA, G rows (see DecodeParams).
+        const long long br_row0 =
+            (2LL * blockIdx.x + (bx == bx_first ? 0 : 1)) * static_cast<long long>(p.G);
+        for (int idx = threadIdx.x; idx < rows_here * D; idx += (W * 32)) {
+            const int h = idx / D;
+            const int d = idx - h * D;
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < W; ++w)
+                if (s_l[w * 16 + h] > 0.f) M = fmaxf(M, s_m[w * 16 + h]);
+            float L = 0.f, O = 0.f;
+#pragma unroll
+            for (int w = 0; w < W; ++w) {
+                const float l = s_l[w * 16 + h];
+                if (l > 0.f) {
+                    const float wt = exp2f(s_m[w * 16 + h] - M);
+                    L += wt * l;
+                    O += wt * s_acc[(w * NH * 8 + h) * RS + d];
+                }
+            }
+            const float o = L > 0.f ? (O / L) * out_mul : 0.f;
+            const long long row = row_of(h);
+            if (direct) {
+                p.out[row * D + d] = __float2bfloat16_rn(o);
+            } else {
+                const long long prow = p.balanced ? br_row0 + h : row * p.P_total + slot;
+                p.ws_o[prow * D + d] = o;
+                if (d == 0) {
+                    p.ws_m[prow] = M;
+                    p.ws_l[prow] = L;
+                }
             }
         }
-    }
 
-    // ---------------- next segment (balanced ranges only)
-    if (!p.balanced) break;
-    // A barrier every thread reaches: the merge buffer it ends (which overlays
-    // the stages) is free again, and a wait that gave up anywhere stops the CTA.
-    if (__syncthreads_or(timed_out)) break;
-    bx += j1 - j0;
-    if (bx >= bx_end) break;
-    bj = 0;
-    if (++kvh == p.Hk) {
-        kvh = 0;
-        do {
-            ++s;
-            bn = pages_of(s);
-        } while (bn == 0 && s + 1 < p.S);
-    }
+        // ---------------- next segment (balanced ranges only)
+        if (!p.balanced) break;
+        // A barrier every thread reaches: the merge buffer it ends (which overlays
+        // the stages) is free again, and a wait that gave up anywhere stops the CTA.
+        if (__syncthreads_or(timed_out)) break;
+        bx += j1 - j0;
+        if (bx >= bx_end) break;
+        bj = 0;
+        if (++kvh == p.Hk) {
+            kvh = 0;
+            do {
+                ++s;
+                bn = pages_of(s);
+            } while (bn == 0 && s + 1 < p.S);
+        }
     }  // segments
 }
 
