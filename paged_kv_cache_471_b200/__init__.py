@@ -232,6 +232,12 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
     value_cache: [num_blocks, num_kv_heads, head_size, block_size]; bf16, or
     uint8 / float8_e4m3fn holding e4m3 codes when kv_dtype is "fp8_e4m3"
     (then k_scale / v_scale are 1-element fp32 CUDA tensors).
+
+    The keyword options are those of pa_options in include/pagedattn.h:
+    partition_pages, stages, shared_prefix_blocks, alibi_slopes ([num_heads]
+    fp32), fp8_compute, test_stall_copies, and schedule ("auto",
+    "partitioned" or "balanced").  workspace_tensor defaults to a cached
+    zeroed buffer per device; stream defaults to the current stream.
     """
     import torch
     code = kv_dtype_code(kv_dtype)
