@@ -277,11 +277,11 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
     # The library plans for, and launches on, the current device: make it the
     # tensors' device for the call.
     with torch.cuda.device(dev):
-        need = workspace_size(S, Hq, num_kv_heads, D, block_size, max_seq_len, code,
-                              partition_pages, shared_prefix_blocks=shared_prefix_blocks,
-                              fp8_compute=fp8_compute and code == PA_KV_FP8_E4M3,
-                              schedule=schedule, stages=stages)
-        if workspace_tensor is None:
+        if workspace_tensor is None:  # (a given one is size-checked by the library)
+            need = workspace_size(S, Hq, num_kv_heads, D, block_size, max_seq_len, code,
+                                  partition_pages, shared_prefix_blocks=shared_prefix_blocks,
+                                  fp8_compute=fp8_compute and code == PA_KV_FP8_E4M3,
+                                  schedule=schedule, stages=stages)
             workspace_tensor = workspace(need, dev)
         ws = _ptr(workspace_tensor, "workspace", None, dev)
         rc = lib().pa_decode_ex(*args_ptrs, S, Hq, int(num_kv_heads), D, float(scale), bt,
