@@ -112,7 +112,10 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         schedule != PA_SCHEDULE_PARTITIONED)
         return fail(PA_ERR_INVALID_ARG, "%s", "opts->schedule");
     const bool f8mma = opts && opts->fp8_compute && kv_dtype == PA_KV_FP8_E4M3;
-    const size_t stage = 2ull * head_size * block_size * elem_bytes(kv_dtype);
+    // A stage holds a K and a V page; 16-token e4m3 pages with f16 MMAs go in
+    // pairs (pa_decode_kernels.cuh, pair_pages).
+    const bool pair = kv_dtype == PA_KV_FP8_E4M3 && block_size == 16 && !f8mma;
+    const size_t stage = 2ull * head_size * block_size * elem_bytes(kv_dtype) * (pair ? 2 : 1);
     const int W = pa::decode_warps(static_cast<long long>(stage));
     int ns = kDefaultStages;
     if (opts && opts->stages > 0) ns = opts->stages;
@@ -216,7 +219,7 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
     // Short partitions: give each warp a buffer for every page it will read
     // (up to 4), so all copies are in flight after one block-table read.
     if (!(opts && opts->stages > 0)) {
-        const long long per_warp = (pp + W - 1) / W;
+        const long long per_warp = ((pp + (pair ? 1 : 0)) / (pair ? 2 : 1) + W - 1) / W;
         const size_t want = static_cast<size_t>(W) * per_warp * (stage + 8);
         if (per_warp > ns && per_warp <= kMaxShortStages && want <= kShortStagesSmem) {
             ns = static_cast<int>(per_warp);

@@ -110,22 +110,38 @@ constexpr int merge_smem_bytes() {
 // smaller pages get four.
 constexpr int decode_warps(long long stage_bytes) { return stage_bytes >= 16384 ? 2 : 4; }
 
+// Whether a stage holds two 16-token pages (e4m3 pages with f16 MMAs).
+template <int B, bool FP8, bool F8MMA>
+constexpr bool pair_pages() {
+    return FP8 && !F8MMA && B == 16;
+}
+
 template <int D, int B, bool FP8>
 constexpr int decode_warps() {
     return decode_warps(2LL * D * B * (FP8 ? 1 : 2));
 }
 
+// The paired 8-row form is held to three CTAs per SM (170 registers), the
+// residency of the other 8-row forms.
 template <int D, int B, bool FP8, int NH, int W, bool F8MMA>
-__global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(W * 32, (pair_pages<B, FP8, F8MMA>() && NH == 1) ? 3 : 1)
+    pa_decode_kernel(const DecodeParams p) {
     static_assert(!F8MMA || FP8, "e4m3 MMAs need e4m3 pages");
     constexpr int ELEM = FP8 ? 1 : 2;
     constexpr int K32 = D / 32;  // 32-wide k-steps over the head dim (e4m3 MMA)
     constexpr int PAGE = D * B * ELEM;  // one K (or V) page of one kv head
-    constexpr int STAGE = 2 * PAGE;
-    constexpr int NT = B / 8;   // 8-token n-tiles per page (QK)
+    // 16-token e4m3 pages (f16 MMAs) go in pairs: a stage holds two
+    // consecutive logical blocks of the unit (K a, K b, V a, V b), so a warp
+    // keeps as many bytes in flight as with 32-token pages, and one pass of
+    // the page code covers 32 tokens.
+    constexpr bool PAIR = pair_pages<B, FP8, F8MMA>();
+    constexpr int NPG = PAIR ? 2 : 1;  // logical pages per stage
+    constexpr int BT = B * NPG;        // tokens per stage
+    constexpr int STAGE = 2 * PAGE * NPG;
+    constexpr int NT = BT / 8;  // 8-token n-tiles per stage (QK)
     constexpr int KT = D / 16;  // 16-wide k-tiles over the head dim (QK)
     constexpr int MT = D / 16;  // 16-row m-tiles over the head dim (PV)
-    constexpr int KK = B / 16;  // 16-token k-tiles per page (PV)
+    constexpr int KK = BT / 16; // 16-token k-tiles per stage (PV)
     constexpr int CHUNK = B * 16;  // bytes of one 16-byte column group of a K page
     constexpr int RS = D + 4;      // padded row stride of the merge buffer
 
@@ -309,12 +325,15 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
         const int32_t* btrow = p.bt + (long long)s * p.max_blocks;
         const int jcap = p.balanced ? min(bn, p.max_blocks)
                                     : min(j0 + p.PP, pre ? p.prefix_pages : p.max_blocks);
-        auto load_win = [&](int base) -> int {
-            const int j = j0 + warp + W * (base + lane);
+        // (A stage's first page; with pairs, `off` = 1 reads its second.)
+        auto load_win = [&](int base, int off) -> int {
+            const int j = j0 + NPG * (warp + W * (base + lane)) + off;
             return j < jcap ? __ldg(btrow + j) : -1;
         };
-        int win_a = load_win(0);
-        int win_b = load_win(32);
+        int win_a = load_win(0, 0);
+        int win_b = load_win(32, 0);
+        int win_a2 = PAIR ? load_win(0, 1) : -1;
+        int win_b2 = PAIR ? load_win(32, 1) : -1;
         // Raw query words of rows 8r + gq, in the order the fragments use.
         uint32_t qraw[2][KT][2];
 #pragma unroll
@@ -396,11 +415,12 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
             return;
         }
 
-        const int span = j1 - j0;
+        const int span = (j1 - j0 + NPG - 1) / NPG;  // stages of this segment
         const int n_my = span > warp ? (span - warp + W - 1) / W : 0;
 
         int wbase = 0;
-        uint32_t valid_mask = 0;  // bit per stage: the page in it had a legal block id
+        // Bit NPG * stage (+ 1): the stage's (second) page had a legal block id.
+        uint32_t valid_mask = 0;
 
         const size_t head_off = static_cast<size_t>(kvh) * PAGE;
         const size_t block_stride = static_cast<size_t>(p.Hk) * PAGE;
@@ -412,27 +432,45 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
         auto issue = [&](int i) {
             if (i >= wbase + 32) {
                 win_a = win_b;
-                win_b = load_win(wbase + 64);
+                win_b = load_win(wbase + 64, 0);
+                if constexpr (PAIR) {
+                    win_a2 = win_b2;
+                    win_b2 = load_win(wbase + 64, 1);
+                }
                 wbase += 32;
             }
             const int pb = __shfl_sync(kFull, win_a, i & 31);
+            const int pb2 = PAIR ? __shfl_sync(kFull, win_a2, i & 31) : -1;
             const int stage = issue_stage;
             issue_stage = (issue_stage + 1 == NS) ? 0 : issue_stage + 1;
             const uint32_t bar = bar0 + 8 * stage;
             const bool ok = pb >= 0 && static_cast<long long>(pb) < p.num_blocks;
+            // With pairs, the second page belongs to the stage only inside the segment.
+            const bool has2 = PAIR && j0 + NPG * (warp + W * i) + 1 < j1;
+            const bool ok2 = has2 && pb2 >= 0 && static_cast<long long>(pb2) < p.num_blocks;
             if (lane == 0) {
-                if (ok) {
-                    const size_t off = static_cast<size_t>(pb) * block_stride + head_off;
-                    const uint32_t dst = wstage0 + static_cast<uint32_t>(stage * STAGE);
-                    mbar_arrive_expect_tx(bar, STAGE + p.stall_tx_bytes);
-                    bulk_copy_g2s(dst, p.kc + off, PAGE, bar);
-                    bulk_copy_g2s(dst + PAGE, p.vc + off, PAGE, bar);
+                const uint32_t bytes = (ok ? 2 * PAGE : 0) + (ok2 ? 2 * PAGE : 0);
+                const uint32_t dst = wstage0 + static_cast<uint32_t>(stage * STAGE);
+                if (bytes) {
+                    mbar_arrive_expect_tx(bar, bytes + p.stall_tx_bytes);
+                    if (ok) {
+                        const size_t off = static_cast<size_t>(pb) * block_stride + head_off;
+                        bulk_copy_g2s(dst, p.kc + off, PAGE, bar);
+                        bulk_copy_g2s(dst + NPG * PAGE, p.vc + off, PAGE, bar);
+                    }
+                    if (ok2) {
+                        const size_t off = static_cast<size_t>(pb2) * block_stride + head_off;
+                        bulk_copy_g2s(dst + PAGE, p.kc + off, PAGE, bar);
+                        bulk_copy_g2s(dst + 3 * PAGE, p.vc + off, PAGE, bar);
+                    }
                 } else {
                     mbar_arrive(bar);
-                    atomicOr(p.status, kDevBadBlock);
                 }
+                if (!ok || (has2 && !ok2)) atomicOr(p.status, kDevBadBlock);
             }
-            valid_mask = ok ? (valid_mask | (1u << stage)) : (valid_mask & ~(1u << stage));
+            const uint32_t bits = (ok ? 1u : 0u) | (ok2 ? 2u : 0u);
+            constexpr uint32_t kStageBits = PAIR ? 3u : 1u;
+            valid_mask = (valid_mask & ~(kStageBits << (NPG * stage))) | (bits << (NPG * stage));
         };
 
         const int n_pro = n_my < NS ? n_my : NS;
@@ -547,11 +585,16 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
 
         // One landed page: S = Q K^T, online softmax, O^T += V^T P^T.  FULL pages
         // (every slot a token) skip all masking.
+        // `valid` (`valid2`): tokens of the stage's (second) page that count.
         auto page = [&](auto full_tag, auto alibi_tag, const uint32_t kbase, const int valid,
-                        const int pos0) {
+                        const int valid2, const int pos0) {
             constexpr bool FULL = decltype(full_tag)::value;
             constexpr bool ALIBI = decltype(alibi_tag)::value;
-            const uint32_t vbase = kbase + PAGE;
+            const uint32_t vbase = kbase + NPG * PAGE;
+            auto counts = [&](int tk) {  // token tk of the stage is part of the sequence
+                if constexpr (PAIR) return tk < B ? tk < valid : tk - B < valid2;
+                return tk < valid;
+            };
 
             // ---------------- S = Q K^T  (rows: heads, cols: tokens)
             float sc[NT][4];
@@ -596,8 +639,12 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
                         for (int np = 0; np < NT / 2; ++np) {
                             const int tok = 8 * (2 * np + (mi & 1)) + r8;
                             const int chunk = 2 * jp + (mi >> 1);
+                            // With pairs, tokens 16 np .. 16 np + 15 are page np's.
+                            const uint32_t ka = PAIR ? kbase + np * PAGE + chunk * CHUNK +
+                                                           (tok & 15) * 16
+                                                     : kbase + chunk * CHUNK + tok * 16;
                             uint32_t w0, w1, w2, w3;
-                            ldsm_x4(kbase + chunk * CHUNK + tok * 16, w0, w1, w2, w3);
+                            ldsm_x4(ka, w0, w1, w2, w3);
                             const uint32_t(&qlo)[4] = qa[2 * jp];
                             const uint32_t(&qhi)[4] = qa[2 * jp + 1];
                             mma_f16_16816(sc[2 * np], qlo, e4m3_lo_pair(w0), e4m3_hi_pair(w0));
@@ -624,7 +671,7 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
                         if constexpr (ALIBI)
                             x = fmaf(slope2[r], static_cast<float>(pos0 + 8 * nt + 2 * cq + e), x);
                         if constexpr (!FULL) {
-                            if (8 * nt + 2 * cq + e >= valid) x = -INFINITY;
+                            if (!counts(8 * nt + 2 * cq + e)) x = -INFINITY;
                         }
                         v[nt][e] = x;
                         mx = fmaxf(mx, x);
@@ -756,8 +803,8 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
                 uint32_t mlo = kFull, mhi = kFull;
                 if constexpr (!FULL) {
                     const int t0 = 16 * kk + 4 * cq;
-                    mlo = (t0 < valid ? 0x0000ffffu : 0u) | (t0 + 1 < valid ? 0xffff0000u : 0u);
-                    mhi = (t0 + 2 < valid ? 0x0000ffffu : 0u) | (t0 + 3 < valid ? 0xffff0000u : 0u);
+                    mlo = (counts(t0) ? 0x0000ffffu : 0u) | (counts(t0 + 1) ? 0xffff0000u : 0u);
+                    mhi = (counts(t0 + 2) ? 0x0000ffffu : 0u) | (counts(t0 + 3) ? 0xffff0000u : 0u);
                 }
                 if constexpr (!FP8) {
 #pragma unroll
@@ -779,7 +826,10 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
 #pragma unroll
                     for (int mp = 0; mp < MT / 2; ++mp) {
                         uint32_t w0, w1, w2, w3;
-                        ldsm_x4(vbase + (32 * mp + lane) * B + kk * 16, w0, w1, w2, w3);
+                        // With pairs, k-tile kk is page kk's 16 tokens.
+                        ldsm_x4(PAIR ? vbase + kk * PAGE + (32 * mp + lane) * B
+                                     : vbase + (32 * mp + lane) * B + kk * 16,
+                                w0, w1, w2, w3);
                         uint32_t a0[4] = {e4m3_lo_pair(w0), e4m3_lo_pair(w1), e4m3_hi_pair(w0),
                                           e4m3_hi_pair(w1)};
                         uint32_t a1[4] = {e4m3_lo_pair(w2), e4m3_lo_pair(w3), e4m3_hi_pair(w2),
@@ -813,20 +863,23 @@ __global__ void __launch_bounds__(W * 32, 1) pa_decode_kernel(const DecodeParams
                 timed_out = true;
                 break;
             }
-            const int jg = j0 + warp + W * k;
-            const int valid = ((valid_mask >> stage) & 1u) ? min(B, T - jg * B) : 0;
+            const int jg = j0 + NPG * (warp + W * k);  // the stage's first logical page
+            const int valid = ((valid_mask >> (NPG * stage)) & 1u) ? min(B, T - jg * B) : 0;
+            const int valid2 =
+                (PAIR && ((valid_mask >> (NPG * stage + 1)) & 1u)) ? min(B, T - (jg + 1) * B) : 0;
+            const bool full = valid == B && (!PAIR || valid2 == B);
             const uint32_t kbase = wstage0 + static_cast<uint32_t>(stage * STAGE);
-            const int pos0 = jg * B - (T - 1);  // ALiBi position of the page's first slot
+            const int pos0 = jg * B - (T - 1);  // ALiBi position of the stage's first slot
             if (!has_alibi) {
-                if (valid == B)
-                    page(std::true_type{}, std::false_type{}, kbase, valid, pos0);
+                if (full)
+                    page(std::true_type{}, std::false_type{}, kbase, valid, valid2, pos0);
                 else
-                    page(std::false_type{}, std::false_type{}, kbase, valid, pos0);
+                    page(std::false_type{}, std::false_type{}, kbase, valid, valid2, pos0);
             } else {
-                if (valid == B)
-                    page(std::true_type{}, std::true_type{}, kbase, valid, pos0);
+                if (full)
+                    page(std::true_type{}, std::true_type{}, kbase, valid, valid2, pos0);
                 else
-                    page(std::false_type{}, std::true_type{}, kbase, valid, pos0);
+                    page(std::false_type{}, std::true_type{}, kbase, valid, valid2, pos0);
             }
             __syncwarp();
             if (k + NS < n_my) issue(k + NS);
