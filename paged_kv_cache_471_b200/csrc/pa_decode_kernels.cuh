@@ -110,10 +110,10 @@ constexpr int merge_smem_bytes() {
 // smaller pages get four.
 constexpr int decode_warps(long long stage_bytes) { return stage_bytes >= 16384 ? 2 : 4; }
 
-// Whether a stage holds two 16-token pages (e4m3 pages with f16 MMAs).
+// Whether a stage holds two 16-token pages (e4m3 pages).
 template <int B, bool FP8, bool F8MMA>
 constexpr bool pair_pages() {
-    return FP8 && !F8MMA && B == 16;
+    return FP8 && B == 16;
 }
 
 template <int D, int B, bool FP8>
@@ -121,16 +121,17 @@ constexpr int decode_warps() {
     return decode_warps(2LL * D * B * (FP8 ? 1 : 2));
 }
 
-// The paired 8-row form is held to three CTAs per SM (170 registers), the
-// residency of the other 8-row forms.
+// The paired 8-row form with f16 MMAs is held to three CTAs per SM (170
+// registers), the residency of the other 8-row forms.
 template <int D, int B, bool FP8, int NH, int W, bool F8MMA>
-__global__ void __launch_bounds__(W * 32, (pair_pages<B, FP8, F8MMA>() && NH == 1) ? 3 : 1)
+__global__ void __launch_bounds__(W * 32,
+                                  (pair_pages<B, FP8, F8MMA>() && !F8MMA && NH == 1) ? 3 : 1)
     pa_decode_kernel(const DecodeParams p) {
     static_assert(!F8MMA || FP8, "e4m3 MMAs need e4m3 pages");
     constexpr int ELEM = FP8 ? 1 : 2;
     constexpr int K32 = D / 32;  // 32-wide k-steps over the head dim (e4m3 MMA)
     constexpr int PAGE = D * B * ELEM;  // one K (or V) page of one kv head
-    // 16-token e4m3 pages (f16 MMAs) go in pairs: a stage holds two
+    // 16-token e4m3 pages go in pairs: a stage holds two
     // consecutive logical blocks of the unit (K a, K b, V a, V b), so a warp
     // keeps as many bytes in flight as with 32-token pages, and one pass of
     // the page code covers 32 tokens.
@@ -625,8 +626,11 @@ __global__ void __launch_bounds__(W * 32, (pair_pages<B, FP8, F8MMA>() && NH == 
                         for (int np = 0; np < NT / 2; ++np) {
                             const int tok = 8 * (2 * np + (mi & 1)) + r8;
                             const int chunk = 2 * jp + (mi >> 1);
+                            const uint32_t ka = PAIR ? kbase + np * PAGE + chunk * CHUNK +
+                                                           (tok & 15) * 16
+                                                     : kbase + chunk * CHUNK + tok * 16;
                             uint32_t w0, w1, w2, w3;
-                            ldsm_x4(kbase + chunk * CHUNK + tok * 16, w0, w1, w2, w3);
+                            ldsm_x4(ka, w0, w1, w2, w3);
                             mma_e4m3_16832(sc[2 * np], qa8[jp][0], w0, w2);
                             mma_e4m3_16832(sc[2 * np], qa8[jp][1], w0, w2);
                             mma_e4m3_16832(sc[2 * np + 1], qa8[jp][0], w1, w3);
@@ -726,10 +730,10 @@ __global__ void __launch_bounds__(W * 32, (pair_pages<B, FP8, F8MMA>() && NH == 
             }
 
             if constexpr (F8MMA) {
-                // O^T += V^T P^T with one 32-token e4m3 k-step per page: tokens
+                // O^T += V^T P^T with one 32-token e4m3 k-step per stage: tokens
                 // 16 kk + 4 cq .. +3 of each k-tile come from the same quad shuffles
-                // as below; V bytes go into the MMA as they are.  Block size 16
-                // leaves the upper 16 tokens of the step empty (zeros).
+                // as below; V bytes go into the MMA as they are (with paired
+                // 16-token pages, k-tile kk is page kk).
                 uint32_t bh[NH][2], bl[NH][2];
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk)
@@ -754,10 +758,10 @@ __global__ void __launch_bounds__(W * 32, (pair_pages<B, FP8, F8MMA>() && NH == 
 #pragma unroll
                     for (int kk = 0; kk < KK; ++kk) {
                         const int t0 = 16 * kk + 4 * cq;
-                        vmask[kk] = (t0 < valid ? 0x000000ffu : 0u) |
-                                    (t0 + 1 < valid ? 0x0000ff00u : 0u) |
-                                    (t0 + 2 < valid ? 0x00ff0000u : 0u) |
-                                    (t0 + 3 < valid ? 0xff000000u : 0u);
+                        vmask[kk] = (counts(t0) ? 0x000000ffu : 0u) |
+                                    (counts(t0 + 1) ? 0x0000ff00u : 0u) |
+                                    (counts(t0 + 2) ? 0x00ff0000u : 0u) |
+                                    (counts(t0 + 3) ? 0xff000000u : 0u);
                     }
                 }
 #pragma unroll
@@ -765,8 +769,9 @@ __global__ void __launch_bounds__(W * 32, (pair_pages<B, FP8, F8MMA>() && NH == 
                     uint32_t w[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
 #pragma unroll
                     for (int kk = 0; kk < KK; ++kk) {
-                        ldsm_x4(vbase + (32 * mp + lane) * B + kk * 16, w[kk][0], w[kk][1],
-                                w[kk][2], w[kk][3]);
+                        ldsm_x4(PAIR ? vbase + kk * PAGE + (32 * mp + lane) * B
+                                     : vbase + (32 * mp + lane) * B + kk * 16,
+                                w[kk][0], w[kk][1], w[kk][2], w[kk][3]);
 #pragma unroll
                         for (int i = 0; i < 4; ++i) w[kk][i] &= vmask[kk];
                     }
