@@ -112,9 +112,10 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         schedule != PA_SCHEDULE_PARTITIONED)
         return fail(PA_ERR_INVALID_ARG, "%s", "opts->schedule");
     const bool f8mma = opts && opts->fp8_compute && kv_dtype == PA_KV_FP8_E4M3;
-    // A stage holds a K and a V page; 16-token e4m3 pages go in pairs
-    // (pa_decode_kernels.cuh, pair_pages).
-    const bool pair = kv_dtype == PA_KV_FP8_E4M3 && block_size == 16;
+    // A stage holds a K and a V page; small pages (16-token e4m3 pages, and
+    // 16-token bf16 pages of head size 64) go in pairs (pa_decode_kernels.cuh,
+    // pair_pages).
+    const bool pair = block_size == 16 && (kv_dtype == PA_KV_FP8_E4M3 || head_size == 64);
     const size_t stage = 2ull * head_size * block_size * elem_bytes(kv_dtype) * (pair ? 2 : 1);
     const int W = pa::decode_warps(static_cast<long long>(stage));
     int ns = kDefaultStages;

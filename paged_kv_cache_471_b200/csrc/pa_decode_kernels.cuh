@@ -110,10 +110,13 @@ constexpr int merge_smem_bytes() {
 // smaller pages get four.
 constexpr int decode_warps(long long stage_bytes) { return stage_bytes >= 16384 ? 2 : 4; }
 
-// Whether a stage holds two 16-token pages (e4m3 pages).
-template <int B, bool FP8, bool F8MMA>
+// Whether a stage holds two 16-token pages: e4m3 pages, and bf16 pages of
+// head size 64 (2 KiB at most).  Pairs double a warp's bytes in flight at
+// the same warps per SM; measured on B200, 4 KiB pages stream faster than
+// 2 KiB ones (bf16 pages of head size 128 are 4 KiB already).
+template <int D, int B, bool FP8, bool F8MMA>
 constexpr bool pair_pages() {
-    return FP8 && B == 16;
+    return B == 16 && (FP8 || D == 64);
 }
 
 template <int D, int B, bool FP8>
@@ -125,17 +128,17 @@ constexpr int decode_warps() {
 // registers), the residency of the other 8-row forms.
 template <int D, int B, bool FP8, int NH, int W, bool F8MMA>
 __global__ void __launch_bounds__(W * 32,
-                                  (pair_pages<B, FP8, F8MMA>() && !F8MMA && NH == 1) ? 3 : 1)
+                                  (pair_pages<D, B, FP8, F8MMA>() && !F8MMA && NH == 1) ? 3 : 1)
     pa_decode_kernel(const DecodeParams p) {
     static_assert(!F8MMA || FP8, "e4m3 MMAs need e4m3 pages");
     constexpr int ELEM = FP8 ? 1 : 2;
     constexpr int K32 = D / 32;  // 32-wide k-steps over the head dim (e4m3 MMA)
     constexpr int PAGE = D * B * ELEM;  // one K (or V) page of one kv head
-    // 16-token e4m3 pages go in pairs: a stage holds two
+    // Small pages go in pairs (pair_pages): a stage holds two
     // consecutive logical blocks of the unit (K a, K b, V a, V b), so a warp
     // keeps as many bytes in flight as with 32-token pages, and one pass of
     // the page code covers 32 tokens.
-    constexpr bool PAIR = pair_pages<B, FP8, F8MMA>();
+    constexpr bool PAIR = pair_pages<D, B, FP8, F8MMA>();
     constexpr int NPG = PAIR ? 2 : 1;  // logical pages per stage
     constexpr int BT = B * NPG;        // tokens per stage
     constexpr int STAGE = 2 * PAGE * NPG;
@@ -612,8 +615,11 @@ __global__ void __launch_bounds__(W * 32,
                         for (int np = 0; np < NT / 2; ++np) {
                             const int tok = 8 * (2 * np + (mi >> 1)) + r8;
                             const int chunk = 2 * kt + (mi & 1);
+                            const uint32_t ka = PAIR ? kbase + np * PAGE + chunk * CHUNK +
+                                                           (tok & 15) * 16
+                                                     : kbase + chunk * CHUNK + tok * 16;
                             uint32_t b0, b1, b2, b3;
-                            ldsm_x4(kbase + chunk * CHUNK + tok * 16, b0, b1, b2, b3);
+                            ldsm_x4(ka, b0, b1, b2, b3);
                             mma_bf16_16816(sc[2 * np], qa[kt], b0, b1);
                             mma_bf16_16816(sc[2 * np + 1], qa[kt], b2, b3);
                         }
@@ -814,7 +820,9 @@ __global__ void __launch_bounds__(W * 32,
                 if constexpr (!FP8) {
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt) {
-                        const uint32_t ra = vbase + (16 * mt + gq) * (B * 2) + kk * 32 + cq * 8;
+                        const uint32_t ra =
+                            PAIR ? vbase + kk * PAGE + (16 * mt + gq) * (B * 2) + cq * 8
+                                 : vbase + (16 * mt + gq) * (B * 2) + kk * 32 + cq * 8;
                         const uint2 va = lds64(ra);
                         const uint2 vb = lds64(ra + 8 * (B * 2));
                         uint32_t a[4] = {va.x, vb.x, va.y, vb.y};
