@@ -248,6 +248,49 @@ def test_writes_stay_inside_out_and_workspace(case):
     compare(out, run_oracle(wl), c.kv_dtype, case)
 
 
+@pytest.mark.parametrize("kv", [W.FP8_E4M3, "fp8_compute", "bf16_d64"])
+@pytest.mark.parametrize("bad,hot", [(2, 3), (3, 2), (4, 1)])
+def test_bad_block_in_a_paired_stage(kv, bad, hot):
+    """Small pages travel in pairs (logical blocks 0+1, 2+3, 4 of a 5-block
+    sequence).  A bad block id in one page of a pair skips that page only:
+    with a one-hot query on a token of another page, the output stays that
+    token's V row bit for bit, and the bad-id flag is set."""
+    f8c = kv == "fp8_compute"
+    D = 64 if kv == "bf16_d64" else 128
+    kv = W.BF16 if kv == "bf16_d64" else W.FP8_E4M3
+    B = 16
+    lens = [5 * B]
+    cfg = _cfg(D=D, B=B, G=4, kv=kv, lens=lens, extra_blocks=4, seed=91)
+    wl = W.make_workload(cfg, DEV, seq_lens=lens)
+    kc = wl.key_cache
+    for t in range(lens[0]):
+        pb, o = _token_slot(wl, 0, t)
+        kc[pb, :, 0, o, 0] = 0
+    q = torch.zeros_like(wl.query)
+    q[:, :, 0] = 4096.0
+    wl.query = q
+    t_star = hot * B + 5
+    pb, o = _token_slot(wl, 0, t_star)
+    kc[pb, :, 0, o, 0] = 1.0 if kv == W.BF16 else torch.full_like(kc[pb, :, 0, o, 0], 0x7E)
+    wl.block_tables[0, bad] = cfg.num_blocks + 7  # out of range
+    ws = torch.zeros(pa.workspace_size(1, cfg.num_heads, cfg.num_kv_heads, D, B, lens[0], kv,
+                                       fp8_compute=f8c), dtype=torch.uint8, device=DEV)
+    out = torch.empty_like(wl.query)
+    pa.decode(out, wl.query, kc, wl.value_cache, cfg.num_kv_heads, cfg.scale, wl.block_tables,
+              wl.seq_lens, B, cfg.max_seq_len, kv, wl.k_scale, wl.v_scale, workspace_tensor=ws,
+              **({"fp8_compute": True} if f8c else {}))
+    torch.cuda.synchronize()
+    assert pa.read_status(ws) & pa.PA_DEV_BAD_BLOCK_ID
+    for g in range(cfg.num_kv_heads):
+        v = wl.value_cache[pb, g, :, o]
+        if kv == W.BF16:
+            want = v
+        else:
+            want = (v.view(torch.float8_e4m3fn).float() * cfg.v_scale).to(torch.bfloat16)
+        for h in range(g * cfg.group, (g + 1) * cfg.group):
+            assert torch.equal(out[0, h].view(torch.int16), want.view(torch.int16)), (g, h)
+
+
 def test_bad_block_id_and_length_flags():
     lens = [100, 64]
     cfg = _cfg(lens=lens)
