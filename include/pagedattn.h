@@ -181,10 +181,15 @@ pa_status pa_plan_decode(pa_plan* plan, int num_seqs, int num_heads, int num_kv_
 /*
  * Workspace bytes pa_decode needs (>= PA_WORKSPACE_HEADER_BYTES), or 0 when the
  * sizes are invalid.  Layout: a 256-byte header whose first uint32 is the
- * status word, then (when P > 1) per (seq, query head, partition) an fp32
- * partial output [head_size], and fp32 running max (log2 domain) and sum.
- * The caller zeroes the workspace once after allocating it; pa_decode never
- * clears the status word (it is sticky) and overwrites the partials.
+ * status word, then (when P > 1 or a shared prefix is declared) per (seq,
+ * query head, partition) an fp32 partial output [head_size], and fp32 running
+ * max (log2 domain) and sum.  Under PA_SCHEDULE_BALANCED, after the header:
+ * the per-sequence page prefix and the pages per CTA (num_seqs + 2 ints,
+ * padded to 256 bytes), then two slots of G query rows per CTA, each an fp32
+ * partial [head_size] with its max and sum.  The sizes depend on the options
+ * (pass the ones pa_decode_ex will get).  The caller zeroes the workspace once
+ * after allocating it; pa_decode never clears the status word (it is sticky)
+ * and overwrites the rest.
  */
 size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_size,
                                 int block_size, int max_seq_len, pa_kv_dtype kv_dtype,
