@@ -54,14 +54,20 @@ def measured_hbm_peak():
 
 
 def kernel_source_hash() -> str:
-    """Hash of the device-code sources (the .cuh kernel headers); host-side
-    ABI code does not change what the kernels read or write."""
+    """Hash of the device code: the .cuh kernel headers with comments and
+    whitespace removed (host-side ABI code does not change what the kernels
+    read or write, and neither do comments)."""
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_471_b200", "csrc")
     for name in sorted(n for n in os.listdir(csrc) if n.endswith(".cuh")):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode())
-            h.update(f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        text = " ".join(text.split())
+        h.update(name.encode())
+        h.update(text.encode())
     return h.hexdigest()[:16]
 
 

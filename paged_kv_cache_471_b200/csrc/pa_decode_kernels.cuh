@@ -4,14 +4,15 @@
 // with balanced ranges, one wave of CTAs that each walk an equal contiguous
 // share of all (sequence, kv head, page) work, one unit segment at a time
 // (see DecodeParams::balanced).  Within a segment, four warps (two for 16 KiB
-// pages), each an independent producer/consumer pipeline over its share of
-// the segment's pages (pages w, w+4, w+8, ... of the segment).
+// stages), each an independent producer/consumer pipeline over its share of
+// the segment's stages (stages w, w+4, w+8, ... of the segment).  A stage is
+// one page, or two consecutive pages when pages are small (pair_pages).
 //   * Lane 0 of a warp reads the block table (the page table of
 //     "Why PagedAttention was retired", section 1), widens the physical id to
 //     64 bits, and moves the whole (block, kv head) K page and V page --
 //     each one contiguous run of head_size*block_size elements in the cache
-//     layouts of section 2 -- into a shared-memory stage with two 1-D bulk
-//     async copies that complete on the stage's mbarrier.
+//     layouts of section 2 -- into a shared-memory stage with 1-D bulk async
+//     copies (two per page) that complete on the stage's mbarrier.
 //   * The warp consumes a landed page once: S = Q K^T on the tensor cores
 //     (m16n8k16, heads on M, tokens on N, head dim on K), online softmax in
 //     fp32 registers (row max/sum over the quad by shuffles), then
