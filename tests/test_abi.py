@@ -172,6 +172,25 @@ def test_balanced_schedule_limits():
         pa.plan(4, 8, 2, 64, 16, 40, "bf16", num_sms=148, schedule="sometimes")
 
 
+def test_paired_small_pages_fill_the_stage_memory():
+    # 16-token e4m3 pages, and bf16 pages of head size 64, go two per stage:
+    # the same 64 KiB of stages per CTA (4 warps x 2 stages x 8 KiB) as bf16
+    # pages of head size 128, with 3 CTAs per SM.
+    for kv, D in (("fp8_e4m3", 128), ("bf16", 64), ("bf16", 128)):
+        p = pa.plan(256, 32, 8, D, 16, 16384, kv, num_sms=148)
+        assert p["warps_per_cta"] == 4 and p["stages"] == 2, (kv, D, p)
+        assert p["smem_bytes"] == 4 * 2 * 8192 + 4 * 2 * 8, (kv, D, p)
+    # e4m3 with FP8 MMAs pairs too; 2 CTAs per SM for its larger register use
+    p = pa.plan(256, 32, 8, 128, 16, 16384, "fp8_e4m3", num_sms=148, fp8_compute=True,
+                schedule="balanced")
+    assert p["smem_bytes"] == 4 * 2 * 8192 + 4 * 2 * 8 and p["grid_ctas"] == 2 * 148
+    # pages of 4 KiB or more are not paired
+    p = pa.plan(256, 32, 8, 128, 32, 16384, "fp8_e4m3", num_sms=148)
+    assert p["smem_bytes"] == 4 * 2 * 8192 + 4 * 2 * 8
+    p = pa.plan(256, 32, 8, 64, 16, 16384, "fp8_e4m3", num_sms=148)
+    assert p["smem_bytes"] == 4 * 2 * 4096 + 4 * 2 * 8
+
+
 def test_forced_partitions():
     p = _plan(2, partition_pages=7)
     assert p["partition_pages"] == 7 and p["num_partitions"] == -(-256 // 7)
