@@ -76,10 +76,23 @@ double oracle_e4m3_to_double(uint8_t code) {
     return sign ? -v : v;
 }
 
+/* The 256 e4m3 values, each from oracle_e4m3_to_double (a cache of that
+ * function's results, so a long e4m3 sequence does not redo the ldexp per
+ * element).  Filled before any worker thread reads it. */
+static double e4m3_value[256];
+static int e4m3_value_ready = 0;
+
+static void fill_e4m3_values(void) {
+    int c;
+    if (e4m3_value_ready) return;
+    for (c = 0; c < 256; ++c) e4m3_value[c] = oracle_e4m3_to_double((uint8_t)c);
+    e4m3_value_ready = 1;
+}
+
 static double load_elem(const void* base, int64_t idx, int kv_dtype, double scl) {
     if (kv_dtype == ORACLE_KV_BF16)
         return oracle_bf16_to_double(((const uint16_t*)base)[idx]);
-    return oracle_e4m3_to_double(((const uint8_t*)base)[idx]) * scl;
+    return e4m3_value[((const uint8_t*)base)[idx]] * scl;
 }
 
 /* One (s, h) output row.  logit: scratch of at least T doubles. */
@@ -140,6 +153,7 @@ int oracle_pa_decode(double* out, const uint16_t* query, const void* key_cache,
         return -1;
     int G = Hq / Hk;
     int n_rows = pairs ? n_pairs : S * Hq;
+    fill_e4m3_values();
     int max_T = 0, i;
     for (i = 0; i < S; ++i)
         if (seq_lens[i] > max_T) max_T = seq_lens[i];

@@ -367,6 +367,46 @@ def pin_alibi_zero_slopes_is_plain(lib):
     assert np.array_equal(a, b), "zero ALiBi slopes must leave the output unchanged"
 
 
+def _pair_list(c, seed, n):
+    """n (sequence, q head) pairs in random order, with repeats, covering the
+    first and last row; every pair's head runs over all of a kv head's group."""
+    g = torch.Generator().manual_seed(seed)
+    pairs = [(0, 0), (c.S - 1, c.Hq - 1)]
+    for _ in range(n):
+        pairs.append((int(torch.randint(0, c.S, (1,), generator=g)),
+                      int(torch.randint(0, c.Hq, (1,), generator=g))))
+    pairs.append(pairs[2])  # a repeated row
+    perm = torch.randperm(len(pairs), generator=g).tolist()
+    return [pairs[i] for i in perm]
+
+
+def pin_sampled_rows(lib):
+    """The oracle's sampled-row mode (an explicit list of (s, h) pairs, the
+    mode the full-size GPU checks read their references through): each
+    listed row must equal dense SDPA on the contiguous K/V of that
+    (sequence, query head) to 1e-12, and must be bit-identical to the same
+    row of the whole-batch result."""
+    for i, kw in enumerate(DENSE_CASES[1:] + [DENSE_CASES[0]]):
+        c = Case(**kw)
+        pairs = _pair_list(c, 70 + i, 3 * c.S * c.Hq // 2)
+        got = c.run(lib, pairs=pairs)
+        assert got.shape == (len(pairs), c.D), got.shape
+        dense = c.dense()
+        full = c.run(lib)
+        for r, (s, h) in enumerate(pairs):
+            err = np.max(np.abs(got[r] - dense[s, h]))
+            assert err < 1e-12, f"sampled row {r} = ({s}, {h}) of {kw}: {err}"
+            assert np.array_equal(got[r], full[s, h]), f"sampled row ({s}, {h}) of {kw}"
+    # ALiBi slopes follow the listed query head, not the row's position.
+    c = Case(**DENSE_CASES[1])
+    sl = _slopes(c.Hq, 23)
+    pairs = _pair_list(c, 80, 12)
+    got = c.run(lib, pairs=pairs, alibi_slopes=sl)
+    dense = c.dense(alibi_slopes=sl)
+    for r, (s, h) in enumerate(pairs):
+        assert np.max(np.abs(got[r] - dense[s, h])) < 1e-12, f"sampled ALiBi row ({s}, {h})"
+
+
 ALL_PINS = [pin_golden, pin_dense_equivalence, pin_permutation_invariance, pin_uniform_logits,
             pin_seq_len_one, pin_brute_force, pin_e4m3_table, pin_bf16_table, pin_alibi_dense,
-            pin_alibi_brute_force, pin_alibi_zero_slopes_is_plain]
+            pin_alibi_brute_force, pin_alibi_zero_slopes_is_plain, pin_sampled_rows]

@@ -48,6 +48,15 @@ MUTANTS = {
                      "load_elem(value_cache, vi, kv_dtype, k_scale)"),
     "ALiBi bias sign": ("slope * (double)(t - (T - 1));", "slope * (double)((T - 1) - t);"),
     "ALiBi slope of the kv head": ("(double)alibi_slopes[h]", "(double)alibi_slopes[h / G]"),
+    # the sampled-row mode (rows listed as (s, h) pairs)
+    "pairs: s and h swapped": ("int s = pairs ? pairs[2 * i] : i / Hq;\n            int h = pairs ? pairs[2 * i + 1] : i % Hq;",
+                               "int s = pairs ? pairs[2 * i + 1] % S : i / Hq;\n            int h = pairs ? pairs[2 * i] : i % Hq;"),
+    "pairs: first pair for every row": ("int s = pairs ? pairs[2 * i] : i / Hq;\n            int h = pairs ? pairs[2 * i + 1] : i % Hq;",
+                                        "int s = pairs ? pairs[0] : i / Hq;\n            int h = pairs ? pairs[1] : i % Hq;"),
+    "pairs: last pair dropped": ("int n_rows = pairs ? n_pairs : S * Hq;",
+                                 "int n_rows = pairs ? n_pairs - 1 : S * Hq;"),
+    "pairs: row order reversed": ("one_row(out + (int64_t)i * D,",
+                                  "one_row(out + (int64_t)(pairs ? n_rows - 1 - i : i) * D,"),
     "last token dropped": ("for (t = 0; t < T; ++t) {\n        int64_t pb = (int64_t)bt_row[t / B];\n        int o = t % B;\n        double p",
                            "for (t = 0; t < T - (T > 1); ++t) {\n        int64_t pb = (int64_t)bt_row[t / B];\n        int o = t % B;\n        double p"),
 }
