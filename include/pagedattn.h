@@ -31,8 +31,10 @@
  *    for every grid ahead of them before touching memory, so stream order
  *    holds for all they read and write; only their launch overlaps the
  *    previous kernel's end.
- *  - Argument errors are returned synchronously, before any launch, and
- *    before any CUDA call.  pa_last_error_detail() then names the argument.
+ *  - Argument errors are returned synchronously, before any launch.  The
+ *    pointer and size checks come before any CUDA call; checks that depend
+ *    on the plan (shared memory, workspace size) follow a query of the
+ *    current device's SM count.  pa_last_error_detail() names the argument.
  *  - Launch failures return PA_ERR_CUDA.
  *  - Device data is not read on the host.  Kernels check every block id
  *    they use against [0, num_blocks) and every seq_len against
@@ -202,8 +204,11 @@ size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, i
  *  key_cache    [num_blocks, num_kv_heads, head_size/x, block_size, x] of kv_dtype.
  *  value_cache  [num_blocks, num_kv_heads, head_size, block_size] of kv_dtype.
  *  scale        logit scale (typically 1/sqrt(head_size)); finite.
- *  block_tables int32 [num_seqs, max_blocks_per_seq]; entries past a
- *               sequence's last block are never read.
+ *  block_tables int32 [num_seqs, max_blocks_per_seq].  Entries past a
+ *               sequence's last block may be loaded (a warp prefetches its
+ *               row up to the end of its partition) but their values are
+ *               never used as block ids, so any value is fine there (-1,
+ *               stale ids); every entry of a row must be readable memory.
  *  seq_lens     int32 [num_seqs]; 0 gives a zero output row.
  *  max_seq_len  upper bound of seq_lens, used only to plan the split.
  *  num_blocks   blocks in each cache (bounds for block ids).
@@ -245,15 +250,21 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
  * are rejected with PA_ERR_WORKSPACE_TOO_SMALL before anything is launched.
  * No allocation is made: no cudaMalloc, cudaFree or allocating library call.
  *
- * The first call on each device looks up the array's device address (with
- * that device current); make that first call before any stream capture.
- * Every call on a device shares the one array and it keeps the last call's
+ * The array's device address is looked up once per CUDA context (with
+ * cudaGetSymbolAddress, in the caller's current context) and cached under the
+ * context's unique id: each context -- another context on the same device,
+ * or the new primary context after cudaDeviceReset -- has its own copy of
+ * the array at its own address.  The first call in a context does that
+ * lookup, which may load the library's device code into the context; make
+ * that first call before any stream capture.
+ * Every call in a context shares the one array and it keeps the last call's
  * contents; calls that can overlap on the GPU (other streams, other host
  * threads) race on it and must be serialised by the caller.  Nothing in the
  * array needs to start at zero: each call writes every partial it reads.  The
  * device-side range-check bits (PA_DEV_*) of this entry point are recorded in
  * the array but are not reported; use pa_decode with a workspace to read them.
- * Other arguments, pointers and errors are those of pa_decode.
+ * Other arguments, pointers and errors are those of pa_decode, and are
+ * checked before the scratch size.
  */
 #define PA_NOALLOC_SCRATCH_BYTES (16u << 20)
 

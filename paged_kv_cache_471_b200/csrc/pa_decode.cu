@@ -1,12 +1,14 @@
 // C ABI of libpagedattn: argument checks, the split-KV planner, and the
 // launches of pa_decode_kernel / pa_combine_kernel.  See include/pagedattn.h
 // for the contract of each entry point.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "pa_decode_kernels.cuh"
 #include "pagedattn.h"
@@ -340,32 +342,137 @@ cudaError_t launch_combine(const pa::CombineParams& c, int D, cudaStream_t st) {
                    : launch_pdl(pa::pa_combine_kernel<128>, grid, pa::kThreads, 0, st, c);
 }
 
+// Every check pa_decode makes before planning, except on the workspace.
+// *empty is set for a batch of no sequences (nothing to launch; its pointers
+// are not looked at).
+pa_status check_args(const void* out, const void* query, const void* key_cache,
+                     const void* value_cache, int num_seqs, int num_heads, int num_kv_heads,
+                     int head_size, float scale, const int32_t* block_tables,
+                     int max_blocks_per_seq, const int32_t* seq_lens, int block_size,
+                     int max_seq_len, int64_t num_blocks, pa_kv_dtype kv_dtype,
+                     const float* k_scale, const float* v_scale, const pa_options* opts,
+                     bool* empty) {
+    *empty = false;
+    pa_status st = check_sizes(num_seqs, num_heads, num_kv_heads, head_size, block_size,
+                               max_seq_len, kv_dtype);
+    if (st != PA_OK) return st;
+    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "%s", "scale is not finite");
+    if (max_blocks_per_seq < 1) return fail(PA_ERR_INVALID_ARG, "%s", "max_blocks_per_seq < 1");
+    if (static_cast<long long>(max_seq_len) > static_cast<long long>(max_blocks_per_seq) * block_size)
+        return fail(PA_ERR_INVALID_ARG, "%s", "max_seq_len > max_blocks_per_seq * block_size");
+    if (num_blocks < 1) return fail(PA_ERR_INVALID_ARG, "%s", "num_blocks < 1");
+    if (num_seqs == 0) {
+        *empty = true;
+        return PA_OK;
+    }
+    const struct {
+        const void* p;
+        size_t a;
+        const char* name;
+    } ptrs[] = {{out, 16, "out"},
+                {query, 16, "query"},
+                {key_cache, 16, "key_cache"},
+                {value_cache, 16, "value_cache"},
+                {block_tables, 4, "block_tables"},
+                {seq_lens, 4, "seq_lens"}};
+    for (const auto& q : ptrs) {
+        if (!q.p) return fail(PA_ERR_INVALID_ARG, "%s is NULL", q.name);
+        if (!aligned(q.p, q.a)) return fail(PA_ERR_INVALID_ARG, "%s is misaligned", q.name);
+    }
+    if (opts && opts->fp8_compute && kv_dtype != PA_KV_FP8_E4M3)
+        return fail(PA_ERR_INVALID_ARG, "%s", "fp8_compute needs an e4m3 KV cache");
+    if (opts && opts->alibi_slopes && !aligned(opts->alibi_slopes, 4))
+        return fail(PA_ERR_INVALID_ARG, "%s", "alibi_slopes is misaligned");
+    if (kv_dtype == PA_KV_FP8_E4M3) {
+        if (!k_scale || !v_scale)
+            return fail(PA_ERR_INVALID_ARG, "%s", "k_scale and v_scale are required for FP8");
+        if (!aligned(k_scale, 4) || !aligned(v_scale, 4))
+            return fail(PA_ERR_INVALID_ARG, "%s", "k_scale / v_scale misaligned");
+    }
+    return PA_OK;
+}
+
 // Scratch of pa_decode_noalloc: one fixed array per device, in the
 // library's own device memory (no allocation at call time).
 constexpr size_t kNoallocScratchBytes = PA_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
-// Device address of g_noalloc_scratch on the current device.  In host code the
-// array's name is only a host-side stand-in, so the address is looked up once
-// per device with that device current, and cached.
+// Device address of g_noalloc_scratch in the calling thread's current
+// context.  In host code the array's name is only a host-side stand-in, so
+// the address is looked up with cudaGetSymbolAddress, once per context: a
+// context is a separate address space (another context on the same device,
+// or the new primary context after cudaDeviceReset, has its own copy of the
+// array), so the cache is keyed by the context's unique id and not by the
+// device number.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// The current context's unique id (never reused within a process), or 0 when
+// no context is current or the driver cannot say.
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(f);
+        (void)cudaGetLastError();
+    });
+    if (!get_current || !get_id) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+    if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
 pa_status noalloc_scratch(void** out) {
-    static std::atomic<void*> addr[kMaxDevices];
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-    const bool cached = dev >= 0 && dev < kMaxDevices;
-    if (cached) {
-        void* p = addr[dev].load(std::memory_order_acquire);
-        if (p) {
-            *out = p;
-            return PA_OK;
-        }
+    struct Entry {
+        unsigned long long ctx;
+        void* addr;
+    };
+    static std::mutex mu;
+    static Entry cache[kMaxDevices];
+    static int n_cached = 0;
+    unsigned long long ctx = current_context_id();
+    if (ctx != 0) {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < n_cached; ++i)
+            if (cache[i].ctx == ctx) {
+                *out = cache[i].addr;
+                return PA_OK;
+            }
     }
+    // First call in this context (or the context is not known): look the
+    // address up.  This binds the device's primary context to the thread when
+    // none is current yet, and may load the library's device code into it.
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p)
         return fail(PA_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
-    if (cached) addr[dev].store(p, std::memory_order_release);
+    if (ctx == 0) ctx = current_context_id();
+    if (ctx != 0) {
+        std::lock_guard<std::mutex> lock(mu);
+        int slot = -1;
+        for (int i = 0; i < n_cached; ++i)
+            if (cache[i].ctx == ctx) slot = i;
+        if (slot < 0) {
+            // A full table drops its oldest entry (contexts come and go).
+            if (n_cached == kMaxDevices) {
+                for (int i = 1; i < n_cached; ++i) cache[i - 1] = cache[i];
+                --n_cached;
+            }
+            slot = n_cached++;
+        }
+        cache[slot] = Entry{ctx, p};
+    }
     *out = p;
     return PA_OK;
 }
@@ -402,40 +509,14 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
                        const float* k_scale, const float* v_scale, void* workspace,
                        size_t workspace_bytes, void* stream, const pa_options* opts) {
     g_detail[0] = 0;
-    pa_status st = check_sizes(num_seqs, num_heads, num_kv_heads, head_size, block_size,
-                               max_seq_len, kv_dtype);
-    if (st != PA_OK) return st;
-    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "%s", "scale is not finite");
-    if (max_blocks_per_seq < 1) return fail(PA_ERR_INVALID_ARG, "%s", "max_blocks_per_seq < 1");
-    if (static_cast<long long>(max_seq_len) > static_cast<long long>(max_blocks_per_seq) * block_size)
-        return fail(PA_ERR_INVALID_ARG, "%s", "max_seq_len > max_blocks_per_seq * block_size");
-    if (num_blocks < 1) return fail(PA_ERR_INVALID_ARG, "%s", "num_blocks < 1");
-    if (num_seqs == 0) return PA_OK;
-    const struct {
-        const void* p;
-        size_t a;
-        const char* name;
-    } ptrs[] = {{out, 16, "out"},
-                {query, 16, "query"},
-                {key_cache, 16, "key_cache"},
-                {value_cache, 16, "value_cache"},
-                {block_tables, 4, "block_tables"},
-                {seq_lens, 4, "seq_lens"},
-                {workspace, 16, "workspace"}};
-    for (const auto& q : ptrs) {
-        if (!q.p) return fail(PA_ERR_INVALID_ARG, "%s is NULL", q.name);
-        if (!aligned(q.p, q.a)) return fail(PA_ERR_INVALID_ARG, "%s is misaligned", q.name);
-    }
-    if (opts && opts->fp8_compute && kv_dtype != PA_KV_FP8_E4M3)
-        return fail(PA_ERR_INVALID_ARG, "%s", "fp8_compute needs an e4m3 KV cache");
-    if (opts && opts->alibi_slopes && !aligned(opts->alibi_slopes, 4))
-        return fail(PA_ERR_INVALID_ARG, "%s", "alibi_slopes is misaligned");
-    if (kv_dtype == PA_KV_FP8_E4M3) {
-        if (!k_scale || !v_scale)
-            return fail(PA_ERR_INVALID_ARG, "%s", "k_scale and v_scale are required for FP8");
-        if (!aligned(k_scale, 4) || !aligned(v_scale, 4))
-            return fail(PA_ERR_INVALID_ARG, "%s", "k_scale / v_scale misaligned");
-    }
+    bool empty = false;
+    pa_status st = check_args(out, query, key_cache, value_cache, num_seqs, num_heads,
+                              num_kv_heads, head_size, scale, block_tables, max_blocks_per_seq,
+                              seq_lens, block_size, max_seq_len, num_blocks, kv_dtype, k_scale,
+                              v_scale, opts, &empty);
+    if (st != PA_OK || empty) return st;
+    if (!workspace) return fail(PA_ERR_INVALID_ARG, "%s", "workspace is NULL");
+    if (!aligned(workspace, 16)) return fail(PA_ERR_INVALID_ARG, "%s", "workspace is misaligned");
     pa_plan pl;
     st = plan(&pl, num_seqs, num_heads, num_kv_heads, head_size, block_size, max_seq_len, kv_dtype,
               opts);
@@ -545,10 +626,14 @@ pa_status pa_decode_noalloc(void* out, const void* query, const void* key_cache,
                             int max_seq_len, int64_t num_blocks, pa_kv_dtype kv_dtype,
                             const float* k_scale, const float* v_scale, void* stream) {
     g_detail[0] = 0;
-    pa_status st = check_sizes(num_seqs, num_heads, num_kv_heads, head_size, block_size,
-                               max_seq_len, kv_dtype);
-    if (st != PA_OK) return st;
-    if (num_seqs == 0) return PA_OK;
+    // The argument checks of pa_decode come first, so a bad argument is
+    // reported as such whatever the problem's size.
+    bool empty = false;
+    pa_status st = check_args(out, query, key_cache, value_cache, num_seqs, num_heads,
+                              num_kv_heads, head_size, scale, block_tables, max_blocks_per_seq,
+                              seq_lens, block_size, max_seq_len, num_blocks, kv_dtype, k_scale,
+                              v_scale, nullptr, &empty);
+    if (st != PA_OK || empty) return st;
     pa_plan pl;
     st = plan(&pl, num_seqs, num_heads, num_kv_heads, head_size, block_size, max_seq_len, kv_dtype,
               nullptr);

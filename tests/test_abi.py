@@ -224,3 +224,28 @@ def test_alibi_with_shared_prefix_is_refused(L):
     assert rc == pa.PA_ERR_UNSUPPORTED
     rc = _decode(L, opts=ctypes.byref(pa.Options(0, 148, 0, 0, ctypes.c_void_p(0x80002))))
     assert rc == pa.PA_ERR_INVALID_ARG  # misaligned slopes
+
+
+def _noalloc(L, **over):
+    args = dict(out=0x10000, query=0x20000, key_cache=0x30000, value_cache=0x40000,
+                num_seqs=64, num_heads=128, num_kv_heads=8, head_size=128, scale=0.088,
+                block_tables=0x50000, max_blocks_per_seq=32768, seq_lens=0x60000,
+                block_size=16, max_seq_len=524288, num_blocks=1 << 20, kv_dtype=0,
+                k_scale=None, v_scale=None, stream=None)
+    args.update(over)
+    return L.pa_decode_noalloc(*args.values())
+
+
+@pytest.mark.parametrize("over", [dict(out=None), dict(query=0x20002), dict(seq_lens=None),
+                                  dict(scale=float("inf")), dict(num_blocks=0),
+                                  dict(kv_dtype=1), dict(max_seq_len=524289)])
+def test_noalloc_reports_argument_errors_before_the_scratch_size(L, over):
+    # A problem far beyond the built-in scratch, with one bad argument: the
+    # argument is what is reported (the checks run before planning, so no
+    # CUDA call is needed to get there).
+    assert _noalloc(L, **over) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_last_error_detail().decode() != ""
+
+
+def test_noalloc_zero_sequences_is_a_no_op(L):
+    assert _noalloc(L, num_seqs=0, out=None, query=None) == pa.PA_OK

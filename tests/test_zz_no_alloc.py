@@ -87,3 +87,24 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
         torch.cuda.current_stream(DEV).cuda_stream)
     assert rc == pa.PA_ERR_WORKSPACE_TOO_SMALL
     assert b"built-in scratch" in L.pa_last_error_detail()
+
+
+def test_noalloc_same_shape_long_then_short():
+    """One shape called twice: first with long sequences (every partition of
+    every row written), then with short ones -- empty, under one partition,
+    just over one -- so the scratch still holds the first call's partials in
+    slots the second call does not write.  The second output must match the
+    oracle: a call reads only partials it wrote itself."""
+    L = pa.lib()
+    cfg = W.reduced(4, num_seqs=4, seq_len_hi=6000, seq_len_lo=5000)
+    p = pa.plan(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_size, cfg.block_size,
+                cfg.max_seq_len, cfg.kv_dtype)
+    assert p["num_partitions"] > 2 and p["workspace_bytes"] <= pa.NOALLOC_SCRATCH_BYTES
+    span = p["partition_pages"] * cfg.block_size  # tokens per partition
+    long_wl = W.make_workload(cfg, DEV, seq_lens=[6000, 5999, 5500, 6000])
+    short_wl = W.make_workload(cfg, DEV, seq_lens=[0, 7, span - 1, span + 5])
+    for wl in (long_wl, short_wl):
+        out = torch.full_like(wl.query, float("nan"))
+        assert _noalloc(L, wl, out) == pa.PA_OK, L.pa_last_error_detail()
+        torch.cuda.synchronize()
+        compare(out, run_oracle(wl), cfg.kv_dtype, f"noalloc {wl.seq_lens.tolist()}")
