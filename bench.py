@@ -11,6 +11,12 @@ planner splits).  Default workload: the Llama-style MHA decode batch
 per step: larger than L2, so no flush is needed between steps; smaller
 workloads flush L2 by writing a 256 MiB buffer between timed steps).
 
+On one GPU, with one workload asked for (the default), the line also
+carries `per_config`: for each of the five workloads, its own timed region of
+at least 0.3 s, with GB/s, % of the 8 TB/s spec and of the measured copy
+rate, the roofline fraction and DRAM traffic, the plan, and the SM clock
+sampled every 5 ms (at least 12 samples).
+
 With N > 1 (torchrun), every rank runs its own batch of the same workload
 (weak scaling, no collective on the data path); the time is the max over ranks.
 
@@ -39,6 +45,7 @@ UNIT = "GB/s"
 SPEC_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_NAME = "pa_decode_kernel"
+DATA = "synthetic (seeded N(0,1) K/V/Q, seeded random block tables)"
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
@@ -205,7 +212,8 @@ def workload_config(idx: int, num_seqs: int = 0):
 
 
 def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, num_seqs=0,
-             cascade=True, alibi=False, schedule="auto"):
+             cascade=True, alibi=False, schedule="auto", min_region_ms=0.0,
+             min_clock_samples=12, extras=True):
     import torch
 
     import paged_kv_cache_471_b200 as pa
@@ -243,6 +251,19 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
             scratch.fill_(1)
         step()
     torch.cuda.synchronize(device)
+    # Estimated time of one call (warm), to size a timed region of at least
+    # min_region_ms and the extra calls that keep the clock sampler busy.
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(3):
+        if flush:
+            scratch.fill_(1)
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    est_ms = max(e0.elapsed_time(e1) / 3, 1e-3)
+    if min_region_ms > 0:
+        steps = max(steps, int(math.ceil(min_region_ms / est_ms)))
 
     # Per-launch device time: events bracket only the pa_decode call.  Large
     # workloads are timed as `steps` bare back-to-back calls (an event between
@@ -265,7 +286,12 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
     t_end = torch.cuda.Event(enable_timing=True)
     barrier(device)
     torch.cuda.synchronize(device)
-    with ClockSampler(device) as clk:
+    # Clocks are sampled every 5 ms through the timed region and the
+    # per-launch pass after it; when those are too short for
+    # min_clock_samples samples, the same calls keep running, untimed, until
+    # there are enough.
+    extra_calls = 0
+    with ClockSampler(device, period_s=0.005) as clk:
         t_start.record(stream)
         if flush:
             per_launch_pass()
@@ -274,10 +300,17 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
                 step()
         t_end.record(stream)
         torch.cuda.synchronize(device)
-    barrier(device)
-    if not flush:
-        per_launch_pass()
-        torch.cuda.synchronize(device)
+        region_samples = len(clk.samples)
+        barrier(device)
+        if not flush:
+            per_launch_pass()
+            torch.cuda.synchronize(device)
+        chunk = max(1, int(20.0 / est_ms))
+        while clk.ok and len(clk.samples) < min_clock_samples and extra_calls < 200000:
+            for _ in range(chunk):
+                step()
+            torch.cuda.synchronize(device)
+            extra_calls += chunk
     kern_ms = [a.elapsed_time(b) for a, b in ev]
     region_ms = t_start.elapsed_time(t_end)
     # With flushes in the timed region, the step time is the per-call event
@@ -287,7 +320,7 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
     status = pa.read_status(ws)
 
     extra = {}
-    if flush:
+    if flush and extras:
         # Small workloads: also the time per call of back-to-back calls with a
         # warm L2 (bound by the host's launch rate for tiny batches) and of 100
         # calls replayed from one CUDA graph (no launch overhead), labelled as
@@ -326,9 +359,14 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
         extra["graph_of_100_ms_per_call"] = round(g0.elapsed_time(g1) / 500, 5)
         del graph
 
+    clocks = clk.summary()
+    clocks["samples_in_timed_region"] = region_samples
+    clocks["sampled_over"] = ("the timed region and the per-launch pass"
+                              + (f", then {extra_calls} more of the same calls" if extra_calls
+                                 else ""))
     res = dict(cfg=cfg, wl=wl, plan=plan, alg_bytes=alg_bytes, kern_ms=kern_ms,
                region_ms=region_ms, step_ms=step_ms, local_step_ms=local_step_ms, flush=flush,
-               clocks=clk.summary(), status=status,
+               steps=steps, clocks=clocks, status=status,
                launches_per_step=1 + (plan["num_partitions"] > 1 or prefix > 0
                                       or plan["balanced"] == 1),
                shared_prefix_blocks=prefix, alibi=alibi, extra=extra)
@@ -451,6 +489,24 @@ def cpu_sample(idx: int, wl, budget_s: float = 12.0, max_seqs=None):
 
 
 # --------------------------------------------------------------------------- main
+def workload_config_dict(idx, cfg, wl, alg_bytes, n_gpus):
+    """The line's `config`: what the workload is (the same for both arms)."""
+    return {
+        "workload": cfg.name,
+        "config_index": idx,
+        "num_seqs": cfg.num_seqs, "num_heads": cfg.num_heads,
+        "num_kv_heads": cfg.num_kv_heads, "head_size": cfg.head_size,
+        "block_size": cfg.block_size, "num_blocks": cfg.num_blocks,
+        "kv_dtype": cfg.kv_dtype,
+        "shared_prefix_blocks": cfg.shared_prefix_blocks,
+        "sum_seq_lens": int(wl.seq_lens.sum()),
+        "bytes_per_step": alg_bytes,
+        "logical_bytes_per_step": wl.kv_bytes + wl.q_out_bytes,
+        "parallelism": f"weak x{n_gpus} (independent batches per GPU)" if n_gpus > 1
+        else "1 GPU",
+    }
+
+
 def result_line(idx, r, n_gpus, steps, warmup, cpu=None):
     cfg = r["cfg"]
     peak, peak_kind = measured_hbm_peak()
@@ -472,31 +528,21 @@ def result_line(idx, r, n_gpus, steps, warmup, cpu=None):
         "vs_baseline": None,
         "dtype": "fp8_e4m3 KV, f16 MMA, fp32 softmax" if cfg.kv_dtype == "fp8_e4m3"
         else "bf16",
-        "data": "synthetic (seeded N(0,1) K/V/Q, seeded random block tables)",
-        "config": {
-            "workload": cfg.name,
-            "config_index": idx,
-            "num_seqs": cfg.num_seqs, "num_heads": cfg.num_heads,
-            "num_kv_heads": cfg.num_kv_heads, "head_size": cfg.head_size,
-            "block_size": cfg.block_size, "num_blocks": cfg.num_blocks,
-            "sum_seq_lens": int(r["wl"].seq_lens.sum()),
-            "bytes_per_step": r["alg_bytes"],
-            "logical_bytes_per_step": r["wl"].kv_bytes + r["wl"].q_out_bytes,
-            "seqs_per_s": round(cfg.num_seqs * n_gpus / (r["step_ms"] * 1e-3), 1),
-            "pct_of_8TBs_spec": round(100 * gbs / SPEC_HBM_GBS, 2),
-            f"pct_of_{peak_kind}_hbm": round(100 * gbs / peak, 2),
-            "l2": ("flushed between steps (256 MiB write, excluded from step time)"
-                   if r["flush"] else "inputs larger than L2, no flush"),
-            "plan": r["plan"],
-            "shared_prefix_blocks_declared": r["shared_prefix_blocks"],
-            "alibi": r["alibi"],
-            **{k: v for k, v in r["extra"].items()},
-            **({"warm_l2_back_to_back_gbs": round(r["alg_bytes"] / (r["extra"]["warm_l2_back_to_back_ms_per_call"] * 1e-3) / 1e9, 2),
-                "graph_of_100_gbs": round(r["alg_bytes"] / (r["extra"]["graph_of_100_ms_per_call"] * 1e-3) / 1e9, 2)}
-               if r["extra"] else {}),
-            "parallelism": f"weak x{n_gpus} (independent batches per GPU)" if n_gpus > 1
-            else "1 GPU",
-        },
+        "data": DATA,
+        "config": workload_config_dict(idx, cfg, r["wl"], r["alg_bytes"], n_gpus),
+        "seqs_per_s": round(cfg.num_seqs * n_gpus / (r["step_ms"] * 1e-3), 1),
+        "pct_of_8TBs_spec": round(100 * gbs / SPEC_HBM_GBS, 2),
+        f"pct_of_{peak_kind}_hbm": round(100 * gbs / peak, 2),
+        "l2": ("flushed between steps (256 MiB write, excluded from step time)"
+               if r["flush"] else "inputs larger than L2, no flush"),
+        "plan": r["plan"],
+        "shared_prefix_blocks_declared": r["shared_prefix_blocks"],
+        "alibi": r["alibi"],
+        **({"small_workload": {
+            **r["extra"],
+            "warm_l2_back_to_back_gbs": round(r["alg_bytes"] / (r["extra"]["warm_l2_back_to_back_ms_per_call"] * 1e-3) / 1e9, 2),
+            "graph_of_100_gbs": round(r["alg_bytes"] / (r["extra"]["graph_of_100_ms_per_call"] * 1e-3) / 1e9, 2)}}
+           if r["extra"] else {}),
         "roofline": {
             "bound": "hbm",
             "achieved": round(achieved, 2),
@@ -533,6 +579,45 @@ def result_line(idx, r, n_gpus, steps, warmup, cpu=None):
             "sample": f"{cpu['seqs']} of {cfg.num_seqs} sequences (all heads) x {cpu['reps']} "
                       f"repetitions, {cpu['seconds']:.1f} s, fp64 C + OpenMP"}
     return line
+
+
+def config_entry(idx, r):
+    """One workload's figures for the per_config object of the default line:
+    the same quantities as the line's own, for a timed region of at least
+    0.3 s (so that the clock sampler sees it many times)."""
+    cfg = r["cfg"]
+    peak, peak_kind = measured_hbm_peak()
+    gbs = r["alg_bytes"] / (r["step_ms"] * 1e-3) / 1e9
+    ent = {
+        "workload": cfg.name,
+        "steps": r["steps"],
+        "ms_per_step": round(r["step_ms"], 5),
+        "gbs": round(gbs, 2),
+        "pct_of_8TBs_spec": round(100 * gbs / SPEC_HBM_GBS, 2),
+        f"pct_of_{peak_kind}_hbm": round(100 * gbs / peak, 2),
+        "seqs_per_s": round(cfg.num_seqs / (r["step_ms"] * 1e-3), 1),
+        "bytes_per_step": r["alg_bytes"],
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(gbs / peak, 4),
+                     "traffic": traffic_per_launch(idx)},
+        "launch_ms": {"mean": round(sum(r["kern_ms"]) / len(r["kern_ms"]), 5),
+                      "median": round(statistics.median(r["kern_ms"]), 5),
+                      "min": round(min(r["kern_ms"]), 5)},
+        "plan": r["plan"],
+        "shared_prefix_blocks_declared": r["shared_prefix_blocks"],
+        "l2": ("flushed between steps (256 MiB write, excluded from step time)"
+               if r["flush"] else "inputs larger than L2, no flush"),
+        "clocks": r["clocks"],
+        "device_status": r["status"],
+    }
+    if cfg.shared_prefix_blocks:
+        logical = r["wl"].kv_bytes + r["wl"].q_out_bytes
+        ent["bytes_counted"] = "unique (shared prefix blocks once)"
+        ent["logical_bytes_per_step"] = logical
+        ent["logical_gbs"] = round(logical / (r["step_ms"] * 1e-3) / 1e9, 2)
+    for k, v in r["extra"].items():
+        ent[k] = v
+    return ent
 
 
 def run_copy_blocks(args, device):
@@ -598,8 +683,8 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg.name, "config_index": idx},
+        "vs_baseline": None, "dtype": "f64", "data": DATA,
+        "config": workload_config_dict(idx, cfg, wl, bytes_of(wl), args.gpus),
         "cpu_baseline": {"value": round(gbs, 4), "unit": UNIT, "cores": per[0]["threads"],
                          "kind": "oracle",
                          "sample": f"per step {per[0]['seqs']} sequence(s) of {cfg.num_seqs}, "
@@ -627,6 +712,8 @@ def main(argv=None):
                     help="how CTAs share the work (pa_options.schedule)")
     ap.add_argument("--no-cascade", action="store_true",
                     help="do not declare a workload's shared prefix (plain per-sequence decode)")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per_config figures of the other workloads (1 GPU only)")
     ap.add_argument("--num-seqs", type=int, default=0,
                     help="run the workload with fewer sequences (profiling captures only)")
     ap.add_argument("--ref-budget", type=float, default=20.0,
@@ -664,10 +751,24 @@ def main(argv=None):
         cpu = None
         if rank == 0 and ws == 1 and not args.no_cpu and idx == cfg_ids[0]:
             cpu = cpu_sample(idx, r["wl"])
-        if rank == 0:
-            print(json.dumps(result_line(idx, r, ws, args.steps, args.warmup, cpu)), flush=True)
+        line = result_line(idx, r, ws, args.steps, args.warmup, cpu) if rank == 0 else None
         del r
         torch.cuda.empty_cache()
+        # One GPU, one workload asked for: the line also carries every
+        # workload's figures (each its own timed region of >= 0.3 s).
+        if (ws == 1 and len(cfg_ids) == 1 and not args.no_per_config and not args.num_seqs
+                and not args.alibi and args.schedule == "auto"):
+            per = {}
+            for j in (1, 2, 3, 4, 5):
+                rj = time_gpu(j, args.steps, args.warmup, device, want_e2e=False,
+                              min_region_ms=300.0, extras=(j == 1),
+                              cascade=not args.no_cascade)
+                per[str(j)] = config_entry(j, rj)
+                del rj
+                torch.cuda.empty_cache()
+            line["per_config"] = per
+        if rank == 0:
+            print(json.dumps(line), flush=True)
     if ws > 1:
         dist.barrier(device_ids=[device.index])
         dist.destroy_process_group()
