@@ -368,7 +368,7 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
                region_ms=region_ms, step_ms=step_ms, local_step_ms=local_step_ms, flush=flush,
                steps=steps, clocks=clocks, status=status,
                launches_per_step=1 + (plan["num_partitions"] > 1 or prefix > 0
-                                      or plan["balanced"] == 1),
+                                      or plan["balanced"] == 1 or plan["dynamic"] == 1),
                shared_prefix_blocks=prefix, alibi=alibi, extra=extra)
 
     if want_e2e:
@@ -708,7 +708,8 @@ def main(argv=None):
     ap.add_argument("--extra", default="", choices=["", "copy_blocks"],
                     help="measure a side kernel instead of decode")
     ap.add_argument("--alibi", action="store_true", help="decode with ALiBi slopes")
-    ap.add_argument("--schedule", default="auto", choices=["auto", "balanced", "partitioned"],
+    ap.add_argument("--schedule", default="auto",
+                    choices=["auto", "balanced", "partitioned", "dynamic"],
                     help="how CTAs share the work (pa_options.schedule)")
     ap.add_argument("--no-cascade", action="store_true",
                     help="do not declare a workload's shared prefix (plain per-sequence decode)")

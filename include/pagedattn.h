@@ -156,6 +156,7 @@ typedef struct pa_options {
 #define PA_SCHEDULE_AUTO 0
 #define PA_SCHEDULE_BALANCED 1
 #define PA_SCHEDULE_PARTITIONED 2
+#define PA_SCHEDULE_DYNAMIC 3
 
 /* What pa_decode will launch for a given problem. */
 typedef struct pa_plan {
@@ -170,6 +171,10 @@ typedef struct pa_plan {
     int prefix_groups;      /* 16-query-row groups per kv head streaming the prefix     */
     int balanced;           /* 1: balanced page ranges (num_partitions and
                                partition_pages are then 0), 0: fixed partitions        */
+    int dynamic;            /* 1: the dynamic schedule; num_partitions and
+                               prefix_partitions are then the partial slots per query
+                               row of a (sequence, kv head) unit and of a prefix unit,
+                               partition_pages is 0, grid_ctas an upper bound          */
 } pa_plan;
 
 /*

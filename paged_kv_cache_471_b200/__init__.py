@@ -59,7 +59,8 @@ class Plan(ctypes.Structure):
                 ("stages", ctypes.c_int), ("warps_per_cta", ctypes.c_int),
                 ("grid_ctas", ctypes.c_longlong), ("smem_bytes", ctypes.c_size_t),
                 ("workspace_bytes", ctypes.c_size_t), ("prefix_partitions", ctypes.c_int),
-                ("prefix_groups", ctypes.c_int), ("balanced", ctypes.c_int)]
+                ("prefix_groups", ctypes.c_int), ("balanced", ctypes.c_int),
+                ("dynamic", ctypes.c_int)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}
@@ -144,7 +145,7 @@ def _check(rc: int):
                                       f"{L.pa_last_error_detail().decode()}")
 
 
-SCHEDULES = {"auto": 0, "balanced": 1, "partitioned": 2}
+SCHEDULES = {"auto": 0, "balanced": 1, "partitioned": 2, "dynamic": 3}
 
 
 def _opts(partition_pages=0, num_sms=0, stages=0, shared_prefix_blocks=0, alibi_ptr=None,
@@ -236,7 +237,7 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
     The keyword options are those of pa_options in include/pagedattn.h:
     partition_pages, stages, shared_prefix_blocks, alibi_slopes ([num_heads]
     fp32), fp8_compute, test_stall_copies, and schedule ("auto",
-    "partitioned" or "balanced").  workspace_tensor defaults to a cached
+    "partitioned", "balanced" or "dynamic").  workspace_tensor defaults to a cached
     zeroed buffer per device; stream defaults to the current stream.
     """
     import torch

@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "pa_decode_dynamic.cuh"
 #include "pa_decode_kernels.cuh"
 #include "pagedattn.h"
 
@@ -31,6 +32,7 @@ constexpr size_t kShortStagesSmem = 96 * 1024;  // keep >= 2 CTAs per SM
 constexpr long long kMaxCtasPerSm = 3;
 constexpr int kMaxForcedStages = 16;
 constexpr int kMaxDevices = 64;
+constexpr long long kMaxDynSlots = 64;  // partial slots per row and unit kind (dynamic schedule)
 
 thread_local char g_detail[256] = "";
 
@@ -111,7 +113,7 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         return fail(PA_ERR_UNSUPPORTED, "%s", "ALiBi slopes with a shared prefix");
     const int schedule = opts ? opts->schedule : PA_SCHEDULE_AUTO;
     if (schedule != PA_SCHEDULE_AUTO && schedule != PA_SCHEDULE_BALANCED &&
-        schedule != PA_SCHEDULE_PARTITIONED)
+        schedule != PA_SCHEDULE_PARTITIONED && schedule != PA_SCHEDULE_DYNAMIC)
         return fail(PA_ERR_INVALID_ARG, "%s", "opts->schedule");
     const bool f8mma = opts && opts->fp8_compute && kv_dtype == PA_KV_FP8_E4M3;
     // A stage holds a K and a V page; small pages (16-token e4m3 pages, and
@@ -146,6 +148,44 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
     // shared prefix, no forced partitions, the per-sequence page scan in the
     // stage area, and page counts in int.
     const bool forced_pp = opts && opts->partition_pages > 0;
+    pl->dynamic = 0;
+    if (schedule == PA_SCHEDULE_DYNAMIC) {
+        // Persistent warps claiming pages (pa_decode_dynamic.cuh): one wave of
+        // CTAs; per query row, a slot per warp that read its unit (at most
+        // kslots), for the prefix unit and the row's own unit.
+        if (forced_pp)
+            return fail(PA_ERR_UNSUPPORTED, "%s", "the dynamic schedule takes no forced partitions");
+        const long long groups =
+            cascade ? (static_cast<long long>(num_seqs) * (num_heads / num_kv_heads) + 15) / 16 : 0;
+        const long long units_pre = static_cast<long long>(num_kv_heads) * groups;
+        const long long n_units = units_pre + units;
+        if (n_units >= (1ll << 30) || static_cast<long long>(num_seqs) * num_heads >= (1ll << 31))
+            return fail(PA_ERR_INVALID_ARG, "%s", "batch too large for the dynamic schedule");
+        const long long warps = slots * W;
+        long long kslots = n_units > 0 ? 2 * ((warps + n_units - 1) / n_units) + 2 : 2;
+        if (kslots > kMaxDynSlots) kslots = kMaxDynSlots;
+        const long long k_total = (cascade ? 2 : 1) * kslots;
+        const size_t dsmem = static_cast<size_t>(W) * ns * (stage + 8 + 16);
+        if (dsmem > kMaxSmemPerCta - kStaticSmemReserve)
+            return fail(PA_ERR_INVALID_ARG, "%s", "too many stages for shared memory");
+        size_t ws = PA_WORKSPACE_HEADER_BYTES;
+        ws += (static_cast<size_t>(n_units) * 16 + 255) & ~static_cast<size_t>(255);
+        ws += static_cast<size_t>(num_seqs) * num_heads * k_total *
+              (static_cast<size_t>(head_size) + 2) * sizeof(float);
+        ws = (ws + 255) & ~static_cast<size_t>(255);
+        pl->num_partitions = static_cast<int>(kslots);
+        pl->partition_pages = 0;
+        pl->stages = ns;
+        pl->warps_per_cta = W;
+        pl->grid_ctas = slots;
+        pl->smem_bytes = dsmem;
+        pl->workspace_bytes = ws;
+        pl->prefix_partitions = cascade ? static_cast<int>(kslots) : 0;
+        pl->prefix_groups = static_cast<int>(groups);
+        pl->balanced = 0;
+        pl->dynamic = 1;
+        return PA_OK;
+    }
     const bool br_fits = !cascade && !forced_pp && num_seqs > 0 &&
                          (static_cast<size_t>(num_seqs) + 1 + 32 * W) * 4 <= stage_area &&
                          units * (pages_max + 1) < (1ll << 31);
@@ -282,9 +322,9 @@ cudaError_t ensure_smem(K kernel, std::atomic<int>* done) {
 // gap between back-to-back calls and between decode and combine.  Both
 // kernels wait (griddepcontrol.wait) before touching memory, so stream order
 // is kept for everything they read and write.
-template <typename Params>
-cudaError_t launch_pdl(void (*kern)(Params), unsigned grid, unsigned block, size_t smem,
-                       cudaStream_t st, const Params& p) {
+template <typename... Params>
+cudaError_t launch_pdl(void (*kern)(Params...), unsigned grid, unsigned block, size_t smem,
+                       cudaStream_t st, const Params&... p) {
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -295,7 +335,7 @@ cudaError_t launch_pdl(void (*kern)(Params), unsigned grid, unsigned block, size
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p...);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
@@ -333,6 +373,52 @@ cudaError_t launch_any(const pa::DecodeParams& p, int D, int B, bool fp8, bool f
                                 : launch_dtype<64, 32>(p, fp8, f8mma, grid, smem, st);
     return B == 16 ? launch_dtype<128, 16>(p, fp8, f8mma, grid, smem, st)
                    : launch_dtype<128, 32>(p, fp8, f8mma, grid, smem, st);
+}
+
+// The dynamic schedule's persistent grid: at most the CTAs that can be
+// resident at once (the planner's slots, bounded by the occupancy of this
+// kernel form), so that every warp runs from the start.
+template <int D, int B, bool FP8, int NH, bool F8MMA>
+cudaError_t launch_dyn(const pa::DecodeParams& p, pa::DynParams t, long long grid, size_t smem,
+                       cudaStream_t st) {
+    static std::atomic<int> done[kMaxDevices];
+    constexpr int W = pa::decode_warps<D, B, FP8>();
+    auto kern = pa::pa_decode_dyn_kernel<D, B, FP8, NH, W, F8MMA>;
+    if (smem > kMaxSmemPerCta - kStaticSmemReserve) return cudaErrorInvalidValue;
+    cudaError_t e = ensure_smem(kern, done);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0, sms = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, W * 32, smem);
+    if (e != cudaSuccess) return e;
+    if (device_sms(&sms) != 0) return cudaErrorInvalidDevice;
+    const long long resident = static_cast<long long>(per_sm) * sms;
+    if (resident > 0 && grid > resident) grid = resident;
+    if (grid < 1) grid = 1;
+    t.total_warps = static_cast<int>(grid * W);
+    return launch_pdl(kern, static_cast<unsigned>(grid), W * 32, smem, st, p, t);
+}
+
+template <int D, int B, bool FP8, bool F8MMA>
+cudaError_t launch_dyn_nh(const pa::DecodeParams& p, const pa::DynParams& t, long long grid,
+                          size_t smem, cudaStream_t st) {
+    return (p.G > 8 || p.prefix_pages > 0) ? launch_dyn<D, B, FP8, 2, F8MMA>(p, t, grid, smem, st)
+                                           : launch_dyn<D, B, FP8, 1, F8MMA>(p, t, grid, smem, st);
+}
+
+template <int D, int B>
+cudaError_t launch_dyn_dtype(const pa::DecodeParams& p, const pa::DynParams& t, bool fp8,
+                             bool f8mma, long long grid, size_t smem, cudaStream_t st) {
+    if (!fp8) return launch_dyn_nh<D, B, false, false>(p, t, grid, smem, st);
+    return f8mma ? launch_dyn_nh<D, B, true, true>(p, t, grid, smem, st)
+                 : launch_dyn_nh<D, B, true, false>(p, t, grid, smem, st);
+}
+
+cudaError_t launch_dyn_any(const pa::DecodeParams& p, const pa::DynParams& t, int D, int B,
+                           bool fp8, bool f8mma, long long grid, size_t smem, cudaStream_t st) {
+    if (D == 64) return B == 16 ? launch_dyn_dtype<64, 16>(p, t, fp8, f8mma, grid, smem, st)
+                                : launch_dyn_dtype<64, 32>(p, t, fp8, f8mma, grid, smem, st);
+    return B == 16 ? launch_dyn_dtype<128, 16>(p, t, fp8, f8mma, grid, smem, st)
+                   : launch_dyn_dtype<128, 32>(p, t, fp8, f8mma, grid, smem, st);
 }
 
 cudaError_t launch_combine(const pa::CombineParams& c, int D, cudaStream_t st) {
@@ -578,11 +664,65 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool f8mma = opts && opts->fp8_compute && kv_dtype == PA_KV_FP8_E4M3;
+    if (pl.dynamic) {
+        // [header: status, ..., generation / unit cursor / warps finished at
+        //  byte 64][unit counters, 16 bytes per unit][partials: rows x slots]
+        const bool pair =
+            block_size == 16 && (kv_dtype == PA_KV_FP8_E4M3 || head_size == 64);
+        const int npg = pair ? 2 : 1;
+        pa::DynParams t;
+        std::memset(&t, 0, sizeof t);
+        t.units_pre = num_kv_heads * pl.prefix_groups;
+        t.units = t.units_pre + num_seqs * num_kv_heads;
+        t.k_pre = pl.prefix_partitions;
+        t.k_own = pl.num_partitions;
+        t.k_total = t.k_pre + t.k_own;
+        t.step_min = 4 * npg;
+        t.step_max = 32 * npg;
+        t.probe_rounds = (t.units + 31) / 32 < 8 ? (t.units + 31) / 32 : 8;
+        t.hdr = reinterpret_cast<unsigned int*>(ws + 4 * pa::kDynHeaderWord);
+        t.uw = reinterpret_cast<unsigned long long*>(ws + PA_WORKSPACE_HEADER_BYTES);
+        const size_t uw_bytes =
+            (static_cast<size_t>(t.units) * 16 + 255) & ~static_cast<size_t>(255);
+        float* dpart = reinterpret_cast<float*>(ws + PA_WORKSPACE_HEADER_BYTES + uw_bytes);
+        const size_t drows = static_cast<size_t>(num_seqs) * num_heads * t.k_total;
+        p.ws_o = dpart;
+        p.ws_m = dpart + drows * head_size;
+        p.ws_l = p.ws_m + drows;
+        cudaError_t e = launch_dyn_any(p, t, head_size, block_size, kv_dtype == PA_KV_FP8_E4M3,
+                                       f8mma, pl.grid_ctas, pl.smem_bytes, s);
+        if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+        pa::CombineParams c;
+        std::memset(&c, 0, sizeof c);
+        c.out = p.out;
+        c.ws_o = p.ws_o;
+        c.ws_m = p.ws_m;
+        c.ws_l = p.ws_l;
+        c.seq_lens = seq_lens;
+        c.S = num_seqs;
+        c.Hq = num_heads;
+        c.max_blocks = max_blocks_per_seq;
+        c.B = block_size;
+        c.prefix_pages = p.prefix_pages;
+        c.Hk = num_kv_heads;
+        c.G = num_heads / num_kv_heads;
+        c.dynamic = 1;
+        c.dyn_units_pre = t.units_pre;
+        c.dyn_k_pre = t.k_pre;
+        c.dyn_k_own = t.k_own;
+        c.dyn_k_total = t.k_total;
+        c.dyn_hdr = t.hdr;
+        c.dyn_uw = t.uw;
+        e = launch_combine(c, head_size, s);
+        if (e != cudaSuccess) return fail(PA_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
+        return PA_OK;
+    }
     cudaError_t e = launch_any(p, head_size, block_size, kv_dtype == PA_KV_FP8_E4M3, f8mma,
                                pl.grid_ctas, pl.smem_bytes, s);
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
     if (pl.balanced || pl.num_partitions > 1 || p.prefix_pages > 0) {
         pa::CombineParams c;
+        std::memset(&c, 0, sizeof c);
         c.out = p.out;
         c.ws_o = p.ws_o;
         c.ws_m = p.ws_m;

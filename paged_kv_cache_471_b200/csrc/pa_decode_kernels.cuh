@@ -125,6 +125,432 @@ constexpr int decode_warps() {
     return decode_warps(2LL * D * B * (FP8 ? 1 : 2));
 }
 
+// One warp's attention state over a run of pages of one unit, and the work
+// on one landed page: the query as MMA operands, the running (max, sum) of
+// its rows and the O^T accumulator, all in registers.  Rows are query heads
+// 8r + gq of the unit (NH blocks of 8 MMA rows); the page body is shared by
+// every schedule of the decode kernel.
+template <int D, int B, bool FP8, int NH, bool F8MMA>
+struct WarpAttn {
+    static constexpr int ELEM = FP8 ? 1 : 2;
+    static constexpr int K32 = D / 32;  // 32-wide k-steps over the head dim (e4m3 MMA)
+    static constexpr int PAGE = D * B * ELEM;  // one K (or V) page of one kv head
+    static constexpr bool PAIR = pair_pages<D, B, FP8, F8MMA>();
+    static constexpr int NPG = PAIR ? 2 : 1;  // logical pages per stage
+    static constexpr int BT = B * NPG;        // tokens per stage
+    static constexpr int NT = BT / 8;  // 8-token n-tiles per stage (QK)
+    static constexpr int KT = D / 16;  // 16-wide k-tiles over the head dim (QK)
+    static constexpr int MT = D / 16;  // 16-row m-tiles over the head dim (PV)
+    static constexpr int KK = BT / 16; // 16-token k-tiles per stage (PV)
+    static constexpr int CHUNK = B * 16;  // bytes of one 16-byte column group of a K page
+
+    int lane, gq, cq;
+    int src0, src1;
+    bool hi_half;
+    uint32_t qa[F8MMA ? 1 : KT][4];
+    uint32_t qa8[F8MMA ? K32 : 1][2][4];  // e4m3 MMAs: [k-step][hi, lo][regs]
+    float qk_mul, out_mul;
+    float slope2[NH];  // ALiBi slope of each row in log2 units (0 without ALiBi)
+    float m_run[NH], l_run[NH];
+    float acc[MT][NH][4];
+
+    __device__ __forceinline__ explicit WarpAttn(int lane_) {
+        lane = lane_;
+        gq = lane >> 2;  // fragment row group
+        cq = lane & 3;   // thread in quad
+        const int quad0 = lane & ~3;
+        src0 = quad0 | ((2 * cq) & 3);
+        src1 = quad0 | ((2 * cq + 1) & 3);
+        hi_half = cq >= 2;
+    }
+
+    // Q fragments (A operand of S = Q K^T; rows = heads 8r + gq) from the raw
+    // bf16 query words of rows 8r + gq, in the order the fragments use, and
+    // the logit multiplier (log2 domain) and output multiplier that go with them.
+    __device__ __forceinline__ void load_q(const uint32_t (&qraw)[2][KT][2], float scale_log2,
+                                           float k_scale, float v_scale) {
+        qk_mul = scale_log2;
+        out_mul = 1.f;
+        if constexpr (F8MMA) {
+            // e4m3 operands: q is scaled by 2^e so that max|q| 2^e < 256, then
+            // split into hi + lo e4m3 codes (about 2^-8 relative together); both
+            // halves multiply the same K bytes, so one accumulator takes both.
+            // Natural d order: register i holds d = 32 jp + 16 (i >> 1) + 4 cq + 0..3.
+            float amax = 0.f;
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int kt = 0; kt < KT; ++kt) {
+                    const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
+                    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(w0)), fabsf(bf16_hi(w0))),
+                                             fmaxf(fabsf(bf16_lo(w1)), fabsf(bf16_hi(w1)))));
+                }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+            int e = 0;
+            if (amax > 0.f && amax < INFINITY)
+                e = 7 - (static_cast<int>((__float_as_uint(amax) >> 23) & 0xff) - 127);
+            e = max(-100, min(100, e));
+            const float up = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+            const float down = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+#pragma unroll
+            for (int jp = 0; jp < K32; ++jp)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = i & 1, kt = 2 * jp + (i >> 1);
+                    if (r >= NH) {  // rows 8..15 unused: zero codes
+                        qa8[jp][0][i] = 0u;
+                        qa8[jp][1][i] = 0u;
+                        continue;
+                    }
+                    const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
+                    float unused;
+                    const uint32_t a = split_e4m3x2(bf16_lo(w0) * up, bf16_hi(w0) * up, &unused);
+                    const uint32_t b = split_e4m3x2(bf16_lo(w1) * up, bf16_hi(w1) * up, &unused);
+                    qa8[jp][0][i] = __byte_perm(a, b, 0x5410);  // hi codes of d .. d+3
+                    qa8[jp][1][i] = __byte_perm(a, b, 0x7632);  // lo codes
+                }
+            qk_mul = scale_log2 * k_scale * down;
+            out_mul = v_scale;
+        } else if constexpr (!FP8) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int kt = 0; kt < KT; ++kt) {
+                    qa[kt][r] = qraw[r][kt][0];
+                    qa[kt][r + 2] = qraw[r][kt][1];
+                }
+        } else {
+            // f16 operands: q is scaled by 2^-e so that max|q| < 2^15 (f16 range);
+            // 2^e goes back into the logit multiplier.  Within each 16-wide chunk the
+            // k order is permuted to match the e4m3 byte order delivered by ldmatrix:
+            // k = 2c,2c+1 <-> d = 4c,4c+1 and k = 2c+8,2c+9 <-> d = 4c+2,4c+3.
+            float amax = 0.f;
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int kt = 0; kt < KT; ++kt) {
+                    const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
+                    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(w0)), fabsf(bf16_hi(w0))),
+                                             fmaxf(fabsf(bf16_lo(w1)), fabsf(bf16_hi(w1)))));
+                }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+            int ex = 0;
+            if (amax > 0.f && amax < INFINITY)
+                ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xff) - 127;
+            const int e = ex > 14 ? ex - 14 : 0;
+            const float down = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+            const float up = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int kt = 0; kt < KT; ++kt) {
+                    const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
+                    qa[kt][r] = pack_f16x2(bf16_lo(w0) * down, bf16_hi(w0) * down);
+                    qa[kt][r + 2] = pack_f16x2(bf16_lo(w1) * down, bf16_hi(w1) * down);
+                }
+            qk_mul = scale_log2 * k_scale * up;
+            out_mul = v_scale;
+        }
+    }
+
+    // Fresh running state: max -inf, sum 0, accumulator 0.
+    __device__ __forceinline__ void reset() {
+#pragma unroll
+        for (int r = 0; r < NH; ++r) {
+            m_run[r] = -INFINITY;
+            l_run[r] = 0.f;
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int r = 0; r < NH; ++r)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[mt][r][e] = 0.f;
+    }
+
+    // One landed page: S = Q K^T, online softmax, O^T += V^T P^T.  FULL pages
+    // (every slot a token) skip all masking.
+    // `valid` (`valid2`): tokens of the stage's (second) page that count.
+    template <bool FULL, bool ALIBI>
+    __device__ __forceinline__ void page(const uint32_t kbase, const int valid, const int valid2,
+                                         const int pos0) {
+        const uint32_t vbase = kbase + NPG * PAGE;
+        auto counts = [&](int tk) {  // token tk of the stage is part of the sequence
+            if constexpr (PAIR) return tk < B ? tk < valid : tk - B < valid2;
+            return tk < valid;
+        };
+
+        // ---------------- S = Q K^T  (rows: heads, cols: tokens)
+        float sc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
+        {
+            const int mi = lane >> 3, r8 = lane & 7;
+            if constexpr (!FP8) {
+#pragma unroll
+                for (int kt = 0; kt < KT; ++kt)
+#pragma unroll
+                    for (int np = 0; np < NT / 2; ++np) {
+                        const int tok = 8 * (2 * np + (mi >> 1)) + r8;
+                        const int chunk = 2 * kt + (mi & 1);
+                        const uint32_t ka = PAIR ? kbase + np * PAGE + chunk * CHUNK +
+                                                       (tok & 15) * 16
+                                                 : kbase + chunk * CHUNK + tok * 16;
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4(ka, b0, b1, b2, b3);
+                        mma_bf16_16816(sc[2 * np], qa[kt], b0, b1);
+                        mma_bf16_16816(sc[2 * np + 1], qa[kt], b2, b3);
+                    }
+            } else if constexpr (F8MMA) {
+                // K bytes go into the MMA as they are: register = 4 e4m3 codes of
+                // d = 4 cq..4 cq+3 of a 16-d chunk of one token.
+#pragma unroll
+                for (int jp = 0; jp < K32; ++jp)
+#pragma unroll
+                    for (int np = 0; np < NT / 2; ++np) {
+                        const int tok = 8 * (2 * np + (mi & 1)) + r8;
+                        const int chunk = 2 * jp + (mi >> 1);
+                        const uint32_t ka = PAIR ? kbase + np * PAGE + chunk * CHUNK +
+                                                       (tok & 15) * 16
+                                                 : kbase + chunk * CHUNK + tok * 16;
+                        uint32_t w0, w1, w2, w3;
+                        ldsm_x4(ka, w0, w1, w2, w3);
+                        mma_e4m3_16832(sc[2 * np], qa8[jp][0], w0, w2);
+                        mma_e4m3_16832(sc[2 * np], qa8[jp][1], w0, w2);
+                        mma_e4m3_16832(sc[2 * np + 1], qa8[jp][0], w1, w3);
+                        mma_e4m3_16832(sc[2 * np + 1], qa8[jp][1], w1, w3);
+                    }
+            } else {
+#pragma unroll
+                for (int jp = 0; jp < KT / 2; ++jp)
+#pragma unroll
+                    for (int np = 0; np < NT / 2; ++np) {
+                        const int tok = 8 * (2 * np + (mi & 1)) + r8;
+                        const int chunk = 2 * jp + (mi >> 1);
+                        // With pairs, tokens 16 np .. 16 np + 15 are page np's.
+                        const uint32_t ka = PAIR ? kbase + np * PAGE + chunk * CHUNK +
+                                                       (tok & 15) * 16
+                                                 : kbase + chunk * CHUNK + tok * 16;
+                        uint32_t w0, w1, w2, w3;
+                        ldsm_x4(ka, w0, w1, w2, w3);
+                        const uint32_t(&qlo)[4] = qa[2 * jp];
+                        const uint32_t(&qhi)[4] = qa[2 * jp + 1];
+                        mma_f16_16816(sc[2 * np], qlo, e4m3_lo_pair(w0), e4m3_hi_pair(w0));
+                        mma_f16_16816(sc[2 * np + 1], qlo, e4m3_lo_pair(w1), e4m3_hi_pair(w1));
+                        mma_f16_16816(sc[2 * np], qhi, e4m3_lo_pair(w2), e4m3_hi_pair(w2));
+                        mma_f16_16816(sc[2 * np + 1], qhi, e4m3_lo_pair(w3), e4m3_hi_pair(w3));
+                    }
+            }
+        }
+
+        // ---------------- online softmax (log2 domain), per head row
+        uint32_t pp[NH][NT];
+        float alpha[NH];
+        bool grew = false;
+#pragma unroll
+        for (int r = 0; r < NH; ++r) {
+            float v[NT][2];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    float x = sc[nt][2 * r + e] * qk_mul;
+                    if constexpr (ALIBI)
+                        x = fmaf(slope2[r], static_cast<float>(pos0 + 8 * nt + 2 * cq + e), x);
+                    if constexpr (!FULL) {
+                        if (!counts(8 * nt + 2 * cq + e)) x = -INFINITY;
+                    }
+                    v[nt][e] = x;
+                    mx = fmaxf(mx, x);
+                }
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+            const float m_new = fmaxf(m_run[r], mx);
+            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+            grew |= m_new > m_run[r];
+            alpha[r] = fast_exp2(m_run[r] - m_use);
+            m_run[r] = m_new;
+            float ls = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const float p0 = fast_exp2(v[nt][0] - m_use);
+                const float p1 = fast_exp2(v[nt][1] - m_use);
+                uint32_t w;
+                if constexpr (F8MMA) {
+                    // weights x 256 as hi + lo e4m3 codes (hi pair | lo pair << 16);
+                    // the running sum uses the represented values, in the same x 256
+                    // units as the accumulator.
+                    float sum2;
+                    w = split_e4m3x2(p0 * 256.f, p1 * 256.f, &sum2);
+                    ls += sum2;
+                } else if constexpr (!FP8) {
+                    w = pack_bf16x2(p0, p1);
+                    ls += bf16_lo(w) + bf16_hi(w);
+                } else {
+                    w = pack_f16x2(p0, p1);
+                    ls += f16_lo(w) + f16_hi(w);
+                }
+                pp[r][nt] = w;
+            }
+            l_run[r] = l_run[r] * alpha[r] + ls;
+        }
+
+        // ---------------- rescale O^T columns (heads 8r + 2cq, 8r + 2cq + 1),
+        // only when some row maximum of the warp moved.
+        if (__any_sync(kFull, grew)) {
+#pragma unroll
+            for (int r = 0; r < NH; ++r) {
+                const float a0 = __shfl_sync(kFull, alpha[r], 8 * cq);
+                const float a1 = __shfl_sync(kFull, alpha[r], 8 * cq + 4);
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    acc[mt][r][0] *= a0;
+                    acc[mt][r][1] *= a1;
+                    acc[mt][r][2] *= a0;
+                    acc[mt][r][3] *= a1;
+                }
+            }
+        }
+
+        if constexpr (F8MMA) {
+            // O^T += V^T P^T with one 32-token e4m3 k-step per stage: tokens
+            // 16 kk + 4 cq .. +3 of each k-tile come from the same quad shuffles
+            // as below; V bytes go into the MMA as they are (with paired
+            // 16-token pages, k-tile kk is page kk).
+            uint32_t bh[NH][2], bl[NH][2];
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+                for (int r = 0; r < NH; ++r) {
+                    if (kk < KK) {
+                        const uint32_t x0 = __shfl_sync(kFull, pp[r][2 * kk], src0);
+                        const uint32_t y0 = __shfl_sync(kFull, pp[r][2 * kk + 1], src0);
+                        const uint32_t x1 = __shfl_sync(kFull, pp[r][2 * kk], src1);
+                        const uint32_t y1 = __shfl_sync(kFull, pp[r][2 * kk + 1], src1);
+                        const uint32_t u0 = hi_half ? y0 : x0;  // tokens 4cq, 4cq+1
+                        const uint32_t u1 = hi_half ? y1 : x1;  // tokens 4cq+2, 4cq+3
+                        bh[r][kk] = __byte_perm(u0, u1, 0x5410);
+                        bl[r][kk] = __byte_perm(u0, u1, 0x7632);
+                    } else {
+                        bh[r][kk] = 0u;
+                        bl[r][kk] = 0u;
+                    }
+                }
+            uint32_t vmask[2] = {kFull, kFull};
+            if constexpr (!FULL) {
+#pragma unroll
+                for (int kk = 0; kk < KK; ++kk) {
+                    const int t0 = 16 * kk + 4 * cq;
+                    vmask[kk] = (counts(t0) ? 0x000000ffu : 0u) |
+                                (counts(t0 + 1) ? 0x0000ff00u : 0u) |
+                                (counts(t0 + 2) ? 0x00ff0000u : 0u) |
+                                (counts(t0 + 3) ? 0xff000000u : 0u);
+                }
+            }
+#pragma unroll
+            for (int mp = 0; mp < MT / 2; ++mp) {
+                uint32_t w[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
+#pragma unroll
+                for (int kk = 0; kk < KK; ++kk) {
+                    ldsm_x4(PAIR ? vbase + kk * PAGE + (32 * mp + lane) * B
+                                 : vbase + (32 * mp + lane) * B + kk * 16,
+                            w[kk][0], w[kk][1], w[kk][2], w[kk][3]);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) w[kk][i] &= vmask[kk];
+                }
+                const uint32_t a0[4] = {w[0][0], w[0][1], w[1][0], w[1][1]};
+                const uint32_t a1[4] = {w[0][2], w[0][3], w[1][2], w[1][3]};
+#pragma unroll
+                for (int r = 0; r < NH; ++r) {
+                    mma_e4m3_16832(acc[2 * mp][r], a0, bh[r][0], bh[r][1]);
+                    mma_e4m3_16832(acc[2 * mp][r], a0, bl[r][0], bl[r][1]);
+                    mma_e4m3_16832(acc[2 * mp + 1][r], a1, bh[r][0], bh[r][1]);
+                    mma_e4m3_16832(acc[2 * mp + 1][r], a1, bl[r][0], bl[r][1]);
+                }
+            }
+        } else {
+        // ---------------- O^T += V^T P^T  (rows: head dim, cols: heads, k: tokens)
+        // Per 16-token k-tile, thread cq holds V for tokens 4cq..4cq+3 (one
+        // contiguous 4-token group per row), so k = 2cq,2cq+1 <-> tokens
+        // 4cq,4cq+1 and k = 2cq+8,2cq+9 <-> 4cq+2,4cq+3; P is regrouped to
+        // that order with quad shuffles.
+#pragma unroll
+        for (int kk = 0; kk < KK; ++kk) {
+            uint32_t pb0[NH], pb1[NH];
+#pragma unroll
+            for (int r = 0; r < NH; ++r) {
+                const uint32_t x0 = __shfl_sync(kFull, pp[r][2 * kk], src0);
+                const uint32_t y0 = __shfl_sync(kFull, pp[r][2 * kk + 1], src0);
+                const uint32_t x1 = __shfl_sync(kFull, pp[r][2 * kk], src1);
+                const uint32_t y1 = __shfl_sync(kFull, pp[r][2 * kk + 1], src1);
+                pb0[r] = hi_half ? y0 : x0;
+                pb1[r] = hi_half ? y1 : x1;
+            }
+            // Slots past the sequence end may hold anything (even NaN); their
+            // weights are 0, but 0 * NaN is NaN, so their V is zeroed.
+            uint32_t mlo = kFull, mhi = kFull;
+            if constexpr (!FULL) {
+                const int t0 = 16 * kk + 4 * cq;
+                mlo = (counts(t0) ? 0x0000ffffu : 0u) | (counts(t0 + 1) ? 0xffff0000u : 0u);
+                mhi = (counts(t0 + 2) ? 0x0000ffffu : 0u) | (counts(t0 + 3) ? 0xffff0000u : 0u);
+            }
+            if constexpr (!FP8) {
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    const uint32_t ra =
+                        PAIR ? vbase + kk * PAGE + (16 * mt + gq) * (B * 2) + cq * 8
+                             : vbase + (16 * mt + gq) * (B * 2) + kk * 32 + cq * 8;
+                    const uint2 va = lds64(ra);
+                    const uint2 vb = lds64(ra + 8 * (B * 2));
+                    uint32_t a[4] = {va.x, vb.x, va.y, vb.y};
+                    if constexpr (!FULL) {
+                        a[0] &= mlo;
+                        a[1] &= mlo;
+                        a[2] &= mhi;
+                        a[3] &= mhi;
+                    }
+#pragma unroll
+                    for (int r = 0; r < NH; ++r) mma_bf16_16816(acc[mt][r], a, pb0[r], pb1[r]);
+                }
+            } else {
+#pragma unroll
+                for (int mp = 0; mp < MT / 2; ++mp) {
+                    uint32_t w0, w1, w2, w3;
+                    // With pairs, k-tile kk is page kk's 16 tokens.
+                    ldsm_x4(PAIR ? vbase + kk * PAGE + (32 * mp + lane) * B
+                                 : vbase + (32 * mp + lane) * B + kk * 16,
+                            w0, w1, w2, w3);
+                    uint32_t a0[4] = {e4m3_lo_pair(w0), e4m3_lo_pair(w1), e4m3_hi_pair(w0),
+                                      e4m3_hi_pair(w1)};
+                    uint32_t a1[4] = {e4m3_lo_pair(w2), e4m3_lo_pair(w3), e4m3_hi_pair(w2),
+                                      e4m3_hi_pair(w3)};
+                    if constexpr (!FULL) {
+                        a0[0] &= mlo;
+                        a0[1] &= mlo;
+                        a0[2] &= mhi;
+                        a0[3] &= mhi;
+                        a1[0] &= mlo;
+                        a1[1] &= mlo;
+                        a1[2] &= mhi;
+                        a1[3] &= mhi;
+                    }
+#pragma unroll
+                    for (int r = 0; r < NH; ++r) {
+                        mma_f16_16816(acc[2 * mp][r], a0, pb0[r], pb1[r]);
+                        mma_f16_16816(acc[2 * mp + 1][r], a1, pb0[r], pb1[r]);
+                    }
+                }
+            }
+        }
+        }  // e4m3 MMAs or f16/bf16 MMAs
+    }
+};
+
 // The paired 8-row form with f16 MMAs is held to three CTAs per SM (170
 // registers), the residency of the other 8-row forms.
 template <int D, int B, bool FP8, int NH, int W, bool F8MMA>
@@ -481,393 +907,11 @@ __global__ void __launch_bounds__(W * 32,
         const int n_pro = n_my < NS ? n_my : NS;
         for (int i = 0; i < n_pro; ++i) issue(i);
 
-        // ---- Q fragments (A operand of S = Q K^T; rows = heads 8r + gq)
-        uint32_t qa[F8MMA ? 1 : KT][4];
-        uint32_t qa8[F8MMA ? K32 : 1][2][4];  // e4m3 MMAs: [k-step][hi, lo][regs]
-        float qk_mul = p.scale_log2;
-        float out_mul = 1.f;
-        if constexpr (F8MMA) {
-            // e4m3 operands: q is scaled by 2^e so that max|q| 2^e < 256, then
-            // split into hi + lo e4m3 codes (about 2^-8 relative together); both
-            // halves multiply the same K bytes, so one accumulator takes both.
-            // Natural d order: register i holds d = 32 jp + 16 (i >> 1) + 4 cq + 0..3.
-            float amax = 0.f;
+        WarpAttn<D, B, FP8, NH, F8MMA> wa(lane);
+        wa.load_q(qraw, p.scale_log2, k_scale, v_scale);
 #pragma unroll
-            for (int r = 0; r < 2; ++r)
-#pragma unroll
-                for (int kt = 0; kt < KT; ++kt) {
-                    const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
-                    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(w0)), fabsf(bf16_hi(w0))),
-                                             fmaxf(fabsf(bf16_lo(w1)), fabsf(bf16_hi(w1)))));
-                }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
-            int e = 0;
-            if (amax > 0.f && amax < INFINITY)
-                e = 7 - (static_cast<int>((__float_as_uint(amax) >> 23) & 0xff) - 127);
-            e = max(-100, min(100, e));
-            const float up = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
-            const float down = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
-#pragma unroll
-            for (int jp = 0; jp < K32; ++jp)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int r = i & 1, kt = 2 * jp + (i >> 1);
-                    if (r >= NH) {  // rows 8..15 unused: zero codes
-                        qa8[jp][0][i] = 0u;
-                        qa8[jp][1][i] = 0u;
-                        continue;
-                    }
-                    const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
-                    float unused;
-                    const uint32_t a = split_e4m3x2(bf16_lo(w0) * up, bf16_hi(w0) * up, &unused);
-                    const uint32_t b = split_e4m3x2(bf16_lo(w1) * up, bf16_hi(w1) * up, &unused);
-                    qa8[jp][0][i] = __byte_perm(a, b, 0x5410);  // hi codes of d .. d+3
-                    qa8[jp][1][i] = __byte_perm(a, b, 0x7632);  // lo codes
-                }
-            qk_mul = p.scale_log2 * k_scale * down;
-            out_mul = v_scale;
-        } else if constexpr (!FP8) {
-#pragma unroll
-            for (int r = 0; r < 2; ++r)
-#pragma unroll
-                for (int kt = 0; kt < KT; ++kt) {
-                    qa[kt][r] = qraw[r][kt][0];
-                    qa[kt][r + 2] = qraw[r][kt][1];
-                }
-        } else {
-            // f16 operands: q is scaled by 2^-e so that max|q| < 2^15 (f16 range);
-            // 2^e goes back into the logit multiplier.  Within each 16-wide chunk the
-            // k order is permuted to match the e4m3 byte order delivered by ldmatrix:
-            // k = 2c,2c+1 <-> d = 4c,4c+1 and k = 2c+8,2c+9 <-> d = 4c+2,4c+3.
-            float amax = 0.f;
-#pragma unroll
-            for (int r = 0; r < 2; ++r)
-#pragma unroll
-                for (int kt = 0; kt < KT; ++kt) {
-                    const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
-                    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(w0)), fabsf(bf16_hi(w0))),
-                                             fmaxf(fabsf(bf16_lo(w1)), fabsf(bf16_hi(w1)))));
-                }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
-            int ex = 0;
-            if (amax > 0.f && amax < INFINITY)
-                ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xff) - 127;
-            const int e = ex > 14 ? ex - 14 : 0;
-            const float down = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
-            const float up = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
-#pragma unroll
-            for (int r = 0; r < 2; ++r)
-#pragma unroll
-                for (int kt = 0; kt < KT; ++kt) {
-                    const uint32_t w0 = qraw[r][kt][0], w1 = qraw[r][kt][1];
-                    qa[kt][r] = pack_f16x2(bf16_lo(w0) * down, bf16_hi(w0) * down);
-                    qa[kt][r + 2] = pack_f16x2(bf16_lo(w1) * down, bf16_hi(w1) * down);
-                }
-            qk_mul = p.scale_log2 * k_scale * up;
-            out_mul = v_scale;
-        }
-
-        float m_run[NH], l_run[NH];
-        float acc[MT][NH][4];
-#pragma unroll
-        for (int r = 0; r < NH; ++r) {
-            m_run[r] = -INFINITY;
-            l_run[r] = 0.f;
-        }
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-            for (int r = 0; r < NH; ++r)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc[mt][r][e] = 0.f;
-
-        const int quad0 = lane & ~3;
-        const int src0 = quad0 | ((2 * cq) & 3);
-        const int src1 = quad0 | ((2 * cq + 1) & 3);
-        const bool hi_half = cq >= 2;
-
-        // One landed page: S = Q K^T, online softmax, O^T += V^T P^T.  FULL pages
-        // (every slot a token) skip all masking.
-        // `valid` (`valid2`): tokens of the stage's (second) page that count.
-        auto page = [&](auto full_tag, auto alibi_tag, const uint32_t kbase, const int valid,
-                        const int valid2, const int pos0) {
-            constexpr bool FULL = decltype(full_tag)::value;
-            constexpr bool ALIBI = decltype(alibi_tag)::value;
-            const uint32_t vbase = kbase + NPG * PAGE;
-            auto counts = [&](int tk) {  // token tk of the stage is part of the sequence
-                if constexpr (PAIR) return tk < B ? tk < valid : tk - B < valid2;
-                return tk < valid;
-            };
-
-            // ---------------- S = Q K^T  (rows: heads, cols: tokens)
-            float sc[NT][4];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
-            {
-                const int mi = lane >> 3, r8 = lane & 7;
-                if constexpr (!FP8) {
-#pragma unroll
-                    for (int kt = 0; kt < KT; ++kt)
-#pragma unroll
-                        for (int np = 0; np < NT / 2; ++np) {
-                            const int tok = 8 * (2 * np + (mi >> 1)) + r8;
-                            const int chunk = 2 * kt + (mi & 1);
-                            const uint32_t ka = PAIR ? kbase + np * PAGE + chunk * CHUNK +
-                                                           (tok & 15) * 16
-                                                     : kbase + chunk * CHUNK + tok * 16;
-                            uint32_t b0, b1, b2, b3;
-                            ldsm_x4(ka, b0, b1, b2, b3);
-                            mma_bf16_16816(sc[2 * np], qa[kt], b0, b1);
-                            mma_bf16_16816(sc[2 * np + 1], qa[kt], b2, b3);
-                        }
-                } else if constexpr (F8MMA) {
-                    // K bytes go into the MMA as they are: register = 4 e4m3 codes of
-                    // d = 4 cq..4 cq+3 of a 16-d chunk of one token.
-#pragma unroll
-                    for (int jp = 0; jp < K32; ++jp)
-#pragma unroll
-                        for (int np = 0; np < NT / 2; ++np) {
-                            const int tok = 8 * (2 * np + (mi & 1)) + r8;
-                            const int chunk = 2 * jp + (mi >> 1);
-                            const uint32_t ka = PAIR ? kbase + np * PAGE + chunk * CHUNK +
-                                                           (tok & 15) * 16
-                                                     : kbase + chunk * CHUNK + tok * 16;
-                            uint32_t w0, w1, w2, w3;
-                            ldsm_x4(ka, w0, w1, w2, w3);
-                            mma_e4m3_16832(sc[2 * np], qa8[jp][0], w0, w2);
-                            mma_e4m3_16832(sc[2 * np], qa8[jp][1], w0, w2);
-                            mma_e4m3_16832(sc[2 * np + 1], qa8[jp][0], w1, w3);
-                            mma_e4m3_16832(sc[2 * np + 1], qa8[jp][1], w1, w3);
-                        }
-                } else {
-#pragma unroll
-                    for (int jp = 0; jp < KT / 2; ++jp)
-#pragma unroll
-                        for (int np = 0; np < NT / 2; ++np) {
-                            const int tok = 8 * (2 * np + (mi & 1)) + r8;
-                            const int chunk = 2 * jp + (mi >> 1);
-                            // With pairs, tokens 16 np .. 16 np + 15 are page np's.
-                            const uint32_t ka = PAIR ? kbase + np * PAGE + chunk * CHUNK +
-                                                           (tok & 15) * 16
-                                                     : kbase + chunk * CHUNK + tok * 16;
-                            uint32_t w0, w1, w2, w3;
-                            ldsm_x4(ka, w0, w1, w2, w3);
-                            const uint32_t(&qlo)[4] = qa[2 * jp];
-                            const uint32_t(&qhi)[4] = qa[2 * jp + 1];
-                            mma_f16_16816(sc[2 * np], qlo, e4m3_lo_pair(w0), e4m3_hi_pair(w0));
-                            mma_f16_16816(sc[2 * np + 1], qlo, e4m3_lo_pair(w1), e4m3_hi_pair(w1));
-                            mma_f16_16816(sc[2 * np], qhi, e4m3_lo_pair(w2), e4m3_hi_pair(w2));
-                            mma_f16_16816(sc[2 * np + 1], qhi, e4m3_lo_pair(w3), e4m3_hi_pair(w3));
-                        }
-                }
-            }
-
-            // ---------------- online softmax (log2 domain), per head row
-            uint32_t pp[NH][NT];
-            float alpha[NH];
-            bool grew = false;
-#pragma unroll
-            for (int r = 0; r < NH; ++r) {
-                float v[NT][2];
-                float mx = -INFINITY;
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        float x = sc[nt][2 * r + e] * qk_mul;
-                        if constexpr (ALIBI)
-                            x = fmaf(slope2[r], static_cast<float>(pos0 + 8 * nt + 2 * cq + e), x);
-                        if constexpr (!FULL) {
-                            if (!counts(8 * nt + 2 * cq + e)) x = -INFINITY;
-                        }
-                        v[nt][e] = x;
-                        mx = fmaxf(mx, x);
-                    }
-                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-                const float m_new = fmaxf(m_run[r], mx);
-                const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-                grew |= m_new > m_run[r];
-                alpha[r] = fast_exp2(m_run[r] - m_use);
-                m_run[r] = m_new;
-                float ls = 0.f;
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    const float p0 = fast_exp2(v[nt][0] - m_use);
-                    const float p1 = fast_exp2(v[nt][1] - m_use);
-                    uint32_t w;
-                    if constexpr (F8MMA) {
-                        // weights x 256 as hi + lo e4m3 codes (hi pair | lo pair << 16);
-                        // the running sum uses the represented values, in the same x 256
-                        // units as the accumulator.
-                        float sum2;
-                        w = split_e4m3x2(p0 * 256.f, p1 * 256.f, &sum2);
-                        ls += sum2;
-                    } else if constexpr (!FP8) {
-                        w = pack_bf16x2(p0, p1);
-                        ls += bf16_lo(w) + bf16_hi(w);
-                    } else {
-                        w = pack_f16x2(p0, p1);
-                        ls += f16_lo(w) + f16_hi(w);
-                    }
-                    pp[r][nt] = w;
-                }
-                l_run[r] = l_run[r] * alpha[r] + ls;
-            }
-
-            // ---------------- rescale O^T columns (heads 8r + 2cq, 8r + 2cq + 1),
-            // only when some row maximum of the warp moved.
-            if (__any_sync(kFull, grew)) {
-#pragma unroll
-                for (int r = 0; r < NH; ++r) {
-                    const float a0 = __shfl_sync(kFull, alpha[r], 8 * cq);
-                    const float a1 = __shfl_sync(kFull, alpha[r], 8 * cq + 4);
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) {
-                        acc[mt][r][0] *= a0;
-                        acc[mt][r][1] *= a1;
-                        acc[mt][r][2] *= a0;
-                        acc[mt][r][3] *= a1;
-                    }
-                }
-            }
-
-            if constexpr (F8MMA) {
-                // O^T += V^T P^T with one 32-token e4m3 k-step per stage: tokens
-                // 16 kk + 4 cq .. +3 of each k-tile come from the same quad shuffles
-                // as below; V bytes go into the MMA as they are (with paired
-                // 16-token pages, k-tile kk is page kk).
-                uint32_t bh[NH][2], bl[NH][2];
-#pragma unroll
-                for (int kk = 0; kk < 2; ++kk)
-#pragma unroll
-                    for (int r = 0; r < NH; ++r) {
-                        if (kk < KK) {
-                            const uint32_t x0 = __shfl_sync(kFull, pp[r][2 * kk], src0);
-                            const uint32_t y0 = __shfl_sync(kFull, pp[r][2 * kk + 1], src0);
-                            const uint32_t x1 = __shfl_sync(kFull, pp[r][2 * kk], src1);
-                            const uint32_t y1 = __shfl_sync(kFull, pp[r][2 * kk + 1], src1);
-                            const uint32_t u0 = hi_half ? y0 : x0;  // tokens 4cq, 4cq+1
-                            const uint32_t u1 = hi_half ? y1 : x1;  // tokens 4cq+2, 4cq+3
-                            bh[r][kk] = __byte_perm(u0, u1, 0x5410);
-                            bl[r][kk] = __byte_perm(u0, u1, 0x7632);
-                        } else {
-                            bh[r][kk] = 0u;
-                            bl[r][kk] = 0u;
-                        }
-                    }
-                uint32_t vmask[2] = {kFull, kFull};
-                if constexpr (!FULL) {
-#pragma unroll
-                    for (int kk = 0; kk < KK; ++kk) {
-                        const int t0 = 16 * kk + 4 * cq;
-                        vmask[kk] = (counts(t0) ? 0x000000ffu : 0u) |
-                                    (counts(t0 + 1) ? 0x0000ff00u : 0u) |
-                                    (counts(t0 + 2) ? 0x00ff0000u : 0u) |
-                                    (counts(t0 + 3) ? 0xff000000u : 0u);
-                    }
-                }
-#pragma unroll
-                for (int mp = 0; mp < MT / 2; ++mp) {
-                    uint32_t w[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
-#pragma unroll
-                    for (int kk = 0; kk < KK; ++kk) {
-                        ldsm_x4(PAIR ? vbase + kk * PAGE + (32 * mp + lane) * B
-                                     : vbase + (32 * mp + lane) * B + kk * 16,
-                                w[kk][0], w[kk][1], w[kk][2], w[kk][3]);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) w[kk][i] &= vmask[kk];
-                    }
-                    const uint32_t a0[4] = {w[0][0], w[0][1], w[1][0], w[1][1]};
-                    const uint32_t a1[4] = {w[0][2], w[0][3], w[1][2], w[1][3]};
-#pragma unroll
-                    for (int r = 0; r < NH; ++r) {
-                        mma_e4m3_16832(acc[2 * mp][r], a0, bh[r][0], bh[r][1]);
-                        mma_e4m3_16832(acc[2 * mp][r], a0, bl[r][0], bl[r][1]);
-                        mma_e4m3_16832(acc[2 * mp + 1][r], a1, bh[r][0], bh[r][1]);
-                        mma_e4m3_16832(acc[2 * mp + 1][r], a1, bl[r][0], bl[r][1]);
-                    }
-                }
-            } else {
-            // ---------------- O^T += V^T P^T  (rows: head dim, cols: heads, k: tokens)
-            // Per 16-token k-tile, thread cq holds V for tokens 4cq..4cq+3 (one
-            // contiguous 4-token group per row), so k = 2cq,2cq+1 <-> tokens
-            // 4cq,4cq+1 and k = 2cq+8,2cq+9 <-> 4cq+2,4cq+3; P is regrouped to
-            // that order with quad shuffles.
-#pragma unroll
-            for (int kk = 0; kk < KK; ++kk) {
-                uint32_t pb0[NH], pb1[NH];
-#pragma unroll
-                for (int r = 0; r < NH; ++r) {
-                    const uint32_t x0 = __shfl_sync(kFull, pp[r][2 * kk], src0);
-                    const uint32_t y0 = __shfl_sync(kFull, pp[r][2 * kk + 1], src0);
-                    const uint32_t x1 = __shfl_sync(kFull, pp[r][2 * kk], src1);
-                    const uint32_t y1 = __shfl_sync(kFull, pp[r][2 * kk + 1], src1);
-                    pb0[r] = hi_half ? y0 : x0;
-                    pb1[r] = hi_half ? y1 : x1;
-                }
-                // Slots past the sequence end may hold anything (even NaN); their
-                // weights are 0, but 0 * NaN is NaN, so their V is zeroed.
-                uint32_t mlo = kFull, mhi = kFull;
-                if constexpr (!FULL) {
-                    const int t0 = 16 * kk + 4 * cq;
-                    mlo = (counts(t0) ? 0x0000ffffu : 0u) | (counts(t0 + 1) ? 0xffff0000u : 0u);
-                    mhi = (counts(t0 + 2) ? 0x0000ffffu : 0u) | (counts(t0 + 3) ? 0xffff0000u : 0u);
-                }
-                if constexpr (!FP8) {
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) {
-                        const uint32_t ra =
-                            PAIR ? vbase + kk * PAGE + (16 * mt + gq) * (B * 2) + cq * 8
-                                 : vbase + (16 * mt + gq) * (B * 2) + kk * 32 + cq * 8;
-                        const uint2 va = lds64(ra);
-                        const uint2 vb = lds64(ra + 8 * (B * 2));
-                        uint32_t a[4] = {va.x, vb.x, va.y, vb.y};
-                        if constexpr (!FULL) {
-                            a[0] &= mlo;
-                            a[1] &= mlo;
-                            a[2] &= mhi;
-                            a[3] &= mhi;
-                        }
-#pragma unroll
-                        for (int r = 0; r < NH; ++r) mma_bf16_16816(acc[mt][r], a, pb0[r], pb1[r]);
-                    }
-                } else {
-#pragma unroll
-                    for (int mp = 0; mp < MT / 2; ++mp) {
-                        uint32_t w0, w1, w2, w3;
-                        // With pairs, k-tile kk is page kk's 16 tokens.
-                        ldsm_x4(PAIR ? vbase + kk * PAGE + (32 * mp + lane) * B
-                                     : vbase + (32 * mp + lane) * B + kk * 16,
-                                w0, w1, w2, w3);
-                        uint32_t a0[4] = {e4m3_lo_pair(w0), e4m3_lo_pair(w1), e4m3_hi_pair(w0),
-                                          e4m3_hi_pair(w1)};
-                        uint32_t a1[4] = {e4m3_lo_pair(w2), e4m3_lo_pair(w3), e4m3_hi_pair(w2),
-                                          e4m3_hi_pair(w3)};
-                        if constexpr (!FULL) {
-                            a0[0] &= mlo;
-                            a0[1] &= mlo;
-                            a0[2] &= mhi;
-                            a0[3] &= mhi;
-                            a1[0] &= mlo;
-                            a1[1] &= mlo;
-                            a1[2] &= mhi;
-                            a1[3] &= mhi;
-                        }
-#pragma unroll
-                        for (int r = 0; r < NH; ++r) {
-                            mma_f16_16816(acc[2 * mp][r], a0, pb0[r], pb1[r]);
-                            mma_f16_16816(acc[2 * mp + 1][r], a1, pb0[r], pb1[r]);
-                        }
-                    }
-                }
-            }
-            }  // e4m3 MMAs or f16/bf16 MMAs
-        };
+        for (int r = 0; r < NH; ++r) wa.slope2[r] = slope2[r];
+        wa.reset();
 
         bool timed_out = false;
         int k = 0;
@@ -886,14 +930,14 @@ __global__ void __launch_bounds__(W * 32,
             const int pos0 = jg * B - (T - 1);  // ALiBi position of the stage's first slot
             if (!has_alibi) {
                 if (full)
-                    page(std::true_type{}, std::false_type{}, kbase, valid, valid2, pos0);
+                    wa.template page<true, false>(kbase, valid, valid2, pos0);
                 else
-                    page(std::false_type{}, std::false_type{}, kbase, valid, valid2, pos0);
+                    wa.template page<false, false>(kbase, valid, valid2, pos0);
             } else {
                 if (full)
-                    page(std::true_type{}, std::true_type{}, kbase, valid, valid2, pos0);
+                    wa.template page<true, true>(kbase, valid, valid2, pos0);
                 else
-                    page(std::false_type{}, std::true_type{}, kbase, valid, valid2, pos0);
+                    wa.template page<false, true>(kbase, valid, valid2, pos0);
             }
             __syncwarp();
             if (k + NS < n_my) issue(k + NS);
@@ -920,8 +964,8 @@ __global__ void __launch_bounds__(W * 32,
         // ---------------- merge the four warps' partial softmax states
 #pragma unroll
         for (int r = 0; r < NH; ++r) {
-            l_run[r] += __shfl_xor_sync(kFull, l_run[r], 1);
-            l_run[r] += __shfl_xor_sync(kFull, l_run[r], 2);
+            wa.l_run[r] += __shfl_xor_sync(kFull, wa.l_run[r], 1);
+            wa.l_run[r] += __shfl_xor_sync(kFull, wa.l_run[r], 2);
         }
         __syncthreads();  // every warp is done with its stages
         float* s_acc = reinterpret_cast<float*>(smem);
@@ -934,16 +978,16 @@ __global__ void __launch_bounds__(W * 32,
                 const int h = 8 * r + 2 * cq;
                 const int d = 16 * mt + gq;
                 float* base = s_acc + (warp * NH * 8 + h) * RS + d;
-                base[0] = acc[mt][r][0];
-                base[RS] = acc[mt][r][1];
-                base[8] = acc[mt][r][2];
-                base[RS + 8] = acc[mt][r][3];
+                base[0] = wa.acc[mt][r][0];
+                base[RS] = wa.acc[mt][r][1];
+                base[8] = wa.acc[mt][r][2];
+                base[RS + 8] = wa.acc[mt][r][3];
             }
         if (cq == 0) {
 #pragma unroll
             for (int r = 0; r < NH; ++r) {
-                s_m[warp * 16 + 8 * r + gq] = m_run[r];
-                s_l[warp * 16 + 8 * r + gq] = timed_out ? 0.f : l_run[r];
+                s_m[warp * 16 + 8 * r + gq] = wa.m_run[r];
+                s_l[warp * 16 + 8 * r + gq] = timed_out ? 0.f : wa.l_run[r];
             }
         }
         __syncthreads();
@@ -970,7 +1014,7 @@ __global__ void __launch_bounds__(W * 32,
                     O += wt * s_acc[(w * NH * 8 + h) * RS + d];
                 }
             }
-            const float o = L > 0.f ? (O / L) * out_mul : 0.f;
+            const float o = L > 0.f ? (O / L) * wa.out_mul : 0.f;
             const long long row = row_of(h);
             if (direct) {
                 p.out[row * D + d] = __float2bfloat16_rn(o);
@@ -1012,6 +1056,13 @@ struct CombineParams {
     int prefix_pages, prefix_parts, P_total;
     int balanced, Hk, G;
     const int* br_scan;  // balanced: per-sequence page prefix [S + 1], pages per CTA
+    // Dynamic schedule: every row is merged here from its units' slots --
+    // slot 0 (the unit's owner) plus one per helper, as the helper counters
+    // of the call that just ran (generation hdr[0] - 1) record them.
+    int dynamic;
+    int dyn_units_pre, dyn_k_pre, dyn_k_own, dyn_k_total;
+    const unsigned int* dyn_hdr;
+    const unsigned long long* dyn_uw;
 };
 
 // Log-sum-exp merge of the split-KV partials of one (sequence, q head) per
@@ -1024,6 +1075,9 @@ struct CombineParams {
 // (its last segment) unless the unit starts its range, every other one in its
 // slot 0 (its first segment).  A unit inside one CTA was written by the decode
 // kernel; a sequence with no pages gets a zero row here.
+// Dynamic schedule: a row's slots are those of its prefix unit (if a prefix
+// is declared) followed by those of its (sequence, kv head) unit; every row
+// is written here.
 // Partitions with an empty sum are skipped.
 template <int D>
 __global__ void __launch_bounds__(kThreads) pa_combine_kernel(const CombineParams p) {
@@ -1037,7 +1091,22 @@ __global__ void __launch_bounds__(kThreads) pa_combine_kernel(const CombineParam
     long long base = row * p.P_total;  // slot i is partial row base + i ...
     long long br_c0 = 0, br_off = 0, br_per = 1;
     int br_g = 0;
-    if (p.balanced) {
+    int dyn_n_pre = 0;
+    if (p.dynamic) {
+        const unsigned int gen = *p.dyn_hdr - 1u;
+        const int h = static_cast<int>(row - static_cast<long long>(s) * p.Hq);
+        const int kvh = h / p.G;
+        auto slots = [&](int u, int k) {
+            const unsigned long long w = p.dyn_uw[2 * u + 1];
+            const unsigned int helpers =
+                static_cast<unsigned int>(w >> 32) == gen ? static_cast<unsigned int>(w) : 0u;
+            return 1 + static_cast<int>(min(helpers, static_cast<unsigned int>(k - 1)));
+        };
+        if (p.prefix_pages > 0)
+            dyn_n_pre = slots(kvh + p.Hk * ((s * p.G + h % p.G) / 16), p.dyn_k_pre);
+        nps = dyn_n_pre + slots(p.dyn_units_pre + s * p.Hk + kvh, p.dyn_k_own);
+        base = row * p.dyn_k_total;
+    } else if (p.balanced) {
         const int h = static_cast<int>(row - static_cast<long long>(s) * p.Hq);
         const int c_s = __ldg(p.br_scan + s);
         const int n_s = __ldg(p.br_scan + s + 1) - c_s;
@@ -1066,6 +1135,7 @@ __global__ void __launch_bounds__(kThreads) pa_combine_kernel(const CombineParam
     }
     // ... or, balanced, slot 2 c + k of CTA c = c0 + i, row g of its G rows.
     auto slot_row = [&](int i) -> long long {
+        if (p.dynamic) return base + (i < dyn_n_pre ? i : p.dyn_k_pre + (i - dyn_n_pre));
         if (!p.balanced) return base + i;
         const long long c = br_c0 + i;
         const int k = (i == 0 && br_off != br_c0 * br_per) ? 1 : 0;

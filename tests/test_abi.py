@@ -249,3 +249,34 @@ def test_noalloc_reports_argument_errors_before_the_scratch_size(L, over):
 
 def test_noalloc_zero_sequences_is_a_no_op(L):
     assert _noalloc(L, num_seqs=0, out=None, query=None) == pa.PA_OK
+
+
+def test_dynamic_schedule_plan_and_workspace():
+    # One wave of CTAs; slots per row and unit kind from warps per unit; the
+    # workspace holds the header, 16 bytes of counters per unit (256-aligned),
+    # then the partials of every query row's slots.
+    for idx in (2, 3, 4, 5):
+        c = W.WORKLOADS[idx]
+        pref = c.shared_prefix_blocks
+        p = pa.plan(c.num_seqs, c.num_heads, c.num_kv_heads, c.head_size, c.block_size,
+                    c.max_seq_len, c.kv_dtype, num_sms=148, schedule="dynamic",
+                    shared_prefix_blocks=pref)
+        assert p["dynamic"] == 1 and p["balanced"] == 0 and p["partition_pages"] == 0
+        assert p["grid_ctas"] == 148 * 3
+        warps = p["grid_ctas"] * p["warps_per_cta"]
+        groups = -(-(c.num_seqs * c.group) // 16) if pref else 0
+        units = c.num_kv_heads * groups + c.num_seqs * c.num_kv_heads
+        k = min(64, 2 * -(-warps // units) + 2)
+        assert p["num_partitions"] == k and p["prefix_partitions"] == (k if pref else 0)
+        assert p["prefix_groups"] == groups
+        k_total = k * (2 if pref else 1)
+        expect = 256 + -(-units * 16 // 256) * 256 + c.num_seqs * c.num_heads * k_total * \
+            (c.head_size + 2) * 4
+        assert p["workspace_bytes"] == -(-expect // 256) * 256
+        assert p["smem_bytes"] == p["warps_per_cta"] * p["stages"] * (
+            2 * c.head_size * c.block_size * c.elem_bytes *
+            (2 if (c.block_size == 16 and (c.kv_dtype == "fp8_e4m3" or c.head_size == 64)) else 1)
+            + 24)
+    with pytest.raises(pa.PagedAttentionError):  # no forced partitions
+        pa.plan(64, 32, 8, 128, 16, 4096, "bf16", num_sms=148, schedule="dynamic",
+                partition_pages=8)
