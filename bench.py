@@ -213,7 +213,7 @@ def workload_config(idx: int, num_seqs: int = 0):
 
 def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, num_seqs=0,
              cascade=True, alibi=False, schedule="auto", min_region_ms=0.0,
-             min_clock_samples=12, extras=True):
+             min_clock_samples=12, extras=True, mha_cuda_cores=False):
     import torch
 
     import paged_kv_cache_471_b200 as pa
@@ -244,7 +244,8 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
         pa.decode(out, wl.query, wl.key_cache, wl.value_cache, cfg.num_kv_heads, cfg.scale,
                   wl.block_tables, wl.seq_lens, cfg.block_size, cfg.max_seq_len, cfg.kv_dtype,
                   wl.k_scale, wl.v_scale, workspace_tensor=ws, stream=stream,
-                  shared_prefix_blocks=prefix, alibi_slopes=slopes, schedule=schedule)
+                  shared_prefix_blocks=prefix, alibi_slopes=slopes, schedule=schedule,
+                  mha_cuda_cores=mha_cuda_cores)
 
     for _ in range(max(warmup, 3)):
         if flush:
@@ -341,7 +342,8 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
                                            cfg.num_kv_heads, cfg.scale, wl.block_tables,
                                            wl.seq_lens, cfg.block_size, cfg.max_seq_len,
                                            cfg.kv_dtype, wl.k_scale, wl.v_scale,
-                                           workspace_tensor=ws, stream=st, schedule=schedule)
+                                           workspace_tensor=ws, stream=st, schedule=schedule,
+                                           mha_cuda_cores=mha_cuda_cores)
             step_on(gs)  # warm on the capture stream
             gs.synchronize()
             with torch.cuda.graph(graph, stream=gs):
@@ -410,7 +412,7 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
                           cfg.scale, bt_d[b], sl_d[b], cfg.block_size, cfg.max_seq_len,
                           cfg.kv_dtype, wl.k_scale, wl.v_scale, workspace_tensor=ws,
                           stream=stream, shared_prefix_blocks=prefix, alibi_slopes=slopes,
-                          schedule=schedule)
+                          schedule=schedule, mha_cuda_cores=mha_cuda_cores)
                 ev_used[b].record(stream)
                 with torch.cuda.stream(down):
                     down.wait_event(ev_used[b])
@@ -711,6 +713,8 @@ def main(argv=None):
     ap.add_argument("--schedule", default="auto",
                     choices=["auto", "balanced", "partitioned", "dynamic"],
                     help="how CTAs share the work (pa_options.schedule)")
+    ap.add_argument("--mha-cuda-cores", action="store_true",
+                    help="q.K and P.V on the CUDA cores for one query head per kv head")
     ap.add_argument("--no-cascade", action="store_true",
                     help="do not declare a workload's shared prefix (plain per-sequence decode)")
     ap.add_argument("--no-per-config", action="store_true",
@@ -745,7 +749,7 @@ def main(argv=None):
     for idx in cfg_ids:
         r = time_gpu(idx, args.steps, args.warmup, device, want_e2e=not args.no_e2e, rank=rank,
                      num_seqs=args.num_seqs, cascade=not args.no_cascade, alibi=args.alibi,
-                     schedule=args.schedule)
+                     schedule=args.schedule, mha_cuda_cores=args.mha_cuda_cores)
         r["step_ms"] = reduce_max(r["step_ms"], device)
         if "e2e_ms" in r:
             r["e2e_ms"] = reduce_max(r["e2e_ms"], device)
@@ -758,7 +762,7 @@ def main(argv=None):
         # One GPU, one workload asked for: the line also carries every
         # workload's figures (each its own timed region of >= 0.3 s).
         if (ws == 1 and len(cfg_ids) == 1 and not args.no_per_config and not args.num_seqs
-                and not args.alibi and args.schedule == "auto"):
+                and not args.alibi and args.schedule == "auto" and not args.mha_cuda_cores):
             per = {}
             for j in (1, 2, 3, 4, 5):
                 rj = time_gpu(j, args.steps, args.warmup, device, want_e2e=False,

@@ -133,6 +133,11 @@ typedef enum pa_kv_dtype {
  *      partial wave, but every CTA then waits for the slowest SM; it pays
  *      where SMs stream at even rates (measured on e4m3 pages, ~1%).  Needs
  *      no shared prefix and no forced partition_pages (PA_ERR_UNSUPPORTED).
+ *  mha_cuda_cores: non-zero runs q.K^T and P.V of a bf16 cache with one query
+ *      head per kv head (num_heads == num_kv_heads, no shared prefix) as fp32
+ *      FMAs on the CUDA cores instead of tensor-core tiles, whose 16 rows would
+ *      hold that one head; the softmax weights then stay fp32.  Other batches
+ *      are not affected.  0 = tensor-core tiles for every batch.
  *  test_stall_copies: for testing the failure path only.  Non-zero makes every
  *      page's completion barrier wait for 16 bytes that no copy delivers and
  *      cuts each wait to ~20 ms, so the kernel takes its give-up path: it lets
@@ -150,6 +155,7 @@ typedef struct pa_options {
     int fp8_compute;
     int test_stall_copies;
     int schedule;
+    int mha_cuda_cores;
 } pa_options;
 
 /* pa_options.schedule values. */

@@ -51,7 +51,8 @@ class Options(ctypes.Structure):
     _fields_ = [("partition_pages", ctypes.c_int), ("num_sms", ctypes.c_int),
                 ("stages", ctypes.c_int), ("shared_prefix_blocks", ctypes.c_int),
                 ("alibi_slopes", ctypes.c_void_p), ("fp8_compute", ctypes.c_int),
-                ("test_stall_copies", ctypes.c_int), ("schedule", ctypes.c_int)]
+                ("test_stall_copies", ctypes.c_int), ("schedule", ctypes.c_int),
+                ("mha_cuda_cores", ctypes.c_int)]
 
 
 class Plan(ctypes.Structure):
@@ -149,16 +150,17 @@ SCHEDULES = {"auto": 0, "balanced": 1, "partitioned": 2, "dynamic": 3}
 
 
 def _opts(partition_pages=0, num_sms=0, stages=0, shared_prefix_blocks=0, alibi_ptr=None,
-          fp8_compute=False, test_stall_copies=False, schedule="auto"):
+          fp8_compute=False, test_stall_copies=False, schedule="auto", mha_cuda_cores=False):
     if schedule not in SCHEDULES:
         raise ValueError(f"schedule must be one of {sorted(SCHEDULES)}")
     if not partition_pages and not num_sms and not stages and not shared_prefix_blocks \
             and not alibi_ptr and not fp8_compute and not test_stall_copies \
-            and schedule == "auto":
+            and schedule == "auto" and not mha_cuda_cores:
         return None
     return ctypes.byref(Options(int(partition_pages), int(num_sms), int(stages),
                                 int(shared_prefix_blocks), alibi_ptr, int(bool(fp8_compute)),
-                                int(bool(test_stall_copies)), SCHEDULES[schedule]))
+                                int(bool(test_stall_copies)), SCHEDULES[schedule],
+                                int(bool(mha_cuda_cores))))
 
 
 def kv_dtype_code(kv_dtype) -> int:
@@ -226,7 +228,8 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
            seq_lens, block_size: int, max_seq_len: int, kv_dtype="bf16", k_scale=None,
            v_scale=None, workspace_tensor=None, partition_pages: int = 0, stream=None,
            stages: int = 0, shared_prefix_blocks: int = 0, alibi_slopes=None,
-           fp8_compute: bool = False, test_stall_copies: bool = False, schedule: str = "auto"):
+           fp8_compute: bool = False, test_stall_copies: bool = False, schedule: str = "auto",
+           mha_cuda_cores: bool = False):
     """Paged decode attention into ``out`` (bf16 [num_seqs, num_heads, head_size]).
 
     key_cache: [num_blocks, num_kv_heads, head_size/x, block_size, x];
@@ -236,8 +239,8 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
 
     The keyword options are those of pa_options in include/pagedattn.h:
     partition_pages, stages, shared_prefix_blocks, alibi_slopes ([num_heads]
-    fp32), fp8_compute, test_stall_copies, and schedule ("auto",
-    "partitioned", "balanced" or "dynamic").  workspace_tensor defaults to a cached
+    fp32), fp8_compute, test_stall_copies, schedule ("auto",
+    "partitioned", "balanced" or "dynamic") and mha_cuda_cores.  workspace_tensor defaults to a cached
     zeroed buffer per device; stream defaults to the current stream.
     """
     import torch
@@ -291,7 +294,7 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
                                 workspace_tensor.numel() * workspace_tensor.element_size(),
                                 st.cuda_stream,
                                 _opts(partition_pages, 0, stages, shared_prefix_blocks, alibi,
-                                      fp8_compute, test_stall_copies, schedule))
+                                      fp8_compute, test_stall_copies, schedule, mha_cuda_cores))
     _check(rc)
     return out
 

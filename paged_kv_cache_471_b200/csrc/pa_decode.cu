@@ -339,12 +339,18 @@ cudaError_t launch_pdl(void (*kern)(Params...), unsigned grid, unsigned block, s
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-template <int D, int B, bool FP8, int NH, bool F8MMA>
+// Forms with a CUDA-core variant for one query head per kv head: bf16 pages.
+template <int D, int B, bool FP8, bool F8MMA>
+constexpr bool has_scalar_form() {
+    return !FP8 && !F8MMA;
+}
+
+template <int D, int B, bool FP8, int NH, bool F8MMA, bool SC = false>
 cudaError_t launch_decode(const pa::DecodeParams& p, long long grid, size_t smem,
                           cudaStream_t st) {
     static std::atomic<int> done[kMaxDevices];
     constexpr int W = pa::decode_warps<D, B, FP8>();
-    auto kern = pa::pa_decode_kernel<D, B, FP8, NH, W, F8MMA>;
+    auto kern = pa::pa_decode_kernel<D, B, FP8, NH, W, F8MMA, SC>;
     if (smem > kMaxSmemPerCta - kStaticSmemReserve) return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem(kern, done);
     if (e != cudaSuccess) return e;
@@ -352,7 +358,12 @@ cudaError_t launch_decode(const pa::DecodeParams& p, long long grid, size_t smem
 }
 
 template <int D, int B, bool FP8, bool F8MMA>
-cudaError_t launch_nh(const pa::DecodeParams& p, long long grid, size_t smem, cudaStream_t st) {
+cudaError_t launch_nh(const pa::DecodeParams& p, bool sc, long long grid, size_t smem,
+                      cudaStream_t st) {
+    if constexpr (has_scalar_form<D, B, FP8, F8MMA>()) {
+        if (sc && p.G == 1 && p.prefix_pages == 0)
+            return launch_decode<D, B, FP8, 1, F8MMA, true>(p, grid, smem, st);
+    }
     // Shared-prefix units pack 16 query rows, so they need the 16-row form.
     return (p.G > 8 || p.prefix_pages > 0)
                ? launch_decode<D, B, FP8, 2, F8MMA>(p, grid, smem, st)
@@ -360,30 +371,30 @@ cudaError_t launch_nh(const pa::DecodeParams& p, long long grid, size_t smem, cu
 }
 
 template <int D, int B>
-cudaError_t launch_dtype(const pa::DecodeParams& p, bool fp8, bool f8mma, long long grid,
-                         size_t smem, cudaStream_t st) {
-    if (!fp8) return launch_nh<D, B, false, false>(p, grid, smem, st);
-    return f8mma ? launch_nh<D, B, true, true>(p, grid, smem, st)
-                 : launch_nh<D, B, true, false>(p, grid, smem, st);
+cudaError_t launch_dtype(const pa::DecodeParams& p, bool fp8, bool f8mma, bool sc,
+                         long long grid, size_t smem, cudaStream_t st) {
+    if (!fp8) return launch_nh<D, B, false, false>(p, sc, grid, smem, st);
+    return f8mma ? launch_nh<D, B, true, true>(p, sc, grid, smem, st)
+                 : launch_nh<D, B, true, false>(p, sc, grid, smem, st);
 }
 
-cudaError_t launch_any(const pa::DecodeParams& p, int D, int B, bool fp8, bool f8mma,
+cudaError_t launch_any(const pa::DecodeParams& p, int D, int B, bool fp8, bool f8mma, bool sc,
                        long long grid, size_t smem, cudaStream_t st) {
-    if (D == 64) return B == 16 ? launch_dtype<64, 16>(p, fp8, f8mma, grid, smem, st)
-                                : launch_dtype<64, 32>(p, fp8, f8mma, grid, smem, st);
-    return B == 16 ? launch_dtype<128, 16>(p, fp8, f8mma, grid, smem, st)
-                   : launch_dtype<128, 32>(p, fp8, f8mma, grid, smem, st);
+    if (D == 64) return B == 16 ? launch_dtype<64, 16>(p, fp8, f8mma, sc, grid, smem, st)
+                                : launch_dtype<64, 32>(p, fp8, f8mma, sc, grid, smem, st);
+    return B == 16 ? launch_dtype<128, 16>(p, fp8, f8mma, sc, grid, smem, st)
+                   : launch_dtype<128, 32>(p, fp8, f8mma, sc, grid, smem, st);
 }
 
 // The dynamic schedule's persistent grid: at most the CTAs that can be
 // resident at once (the planner's slots, bounded by the occupancy of this
 // kernel form), so that every warp runs from the start.
-template <int D, int B, bool FP8, int NH, bool F8MMA>
+template <int D, int B, bool FP8, int NH, bool F8MMA, bool SC = false>
 cudaError_t launch_dyn(const pa::DecodeParams& p, pa::DynParams t, long long grid, size_t smem,
                        cudaStream_t st) {
     static std::atomic<int> done[kMaxDevices];
     constexpr int W = pa::decode_warps<D, B, FP8>();
-    auto kern = pa::pa_decode_dyn_kernel<D, B, FP8, NH, W, F8MMA>;
+    auto kern = pa::pa_decode_dyn_kernel<D, B, FP8, NH, W, F8MMA, SC>;
     if (smem > kMaxSmemPerCta - kStaticSmemReserve) return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem(kern, done);
     if (e != cudaSuccess) return e;
@@ -399,26 +410,31 @@ cudaError_t launch_dyn(const pa::DecodeParams& p, pa::DynParams t, long long gri
 }
 
 template <int D, int B, bool FP8, bool F8MMA>
-cudaError_t launch_dyn_nh(const pa::DecodeParams& p, const pa::DynParams& t, long long grid,
-                          size_t smem, cudaStream_t st) {
+cudaError_t launch_dyn_nh(const pa::DecodeParams& p, const pa::DynParams& t, bool sc,
+                          long long grid, size_t smem, cudaStream_t st) {
+    if constexpr (has_scalar_form<D, B, FP8, F8MMA>()) {
+        if (sc && p.G == 1 && p.prefix_pages == 0)
+            return launch_dyn<D, B, FP8, 1, F8MMA, true>(p, t, grid, smem, st);
+    }
     return (p.G > 8 || p.prefix_pages > 0) ? launch_dyn<D, B, FP8, 2, F8MMA>(p, t, grid, smem, st)
                                            : launch_dyn<D, B, FP8, 1, F8MMA>(p, t, grid, smem, st);
 }
 
 template <int D, int B>
 cudaError_t launch_dyn_dtype(const pa::DecodeParams& p, const pa::DynParams& t, bool fp8,
-                             bool f8mma, long long grid, size_t smem, cudaStream_t st) {
-    if (!fp8) return launch_dyn_nh<D, B, false, false>(p, t, grid, smem, st);
-    return f8mma ? launch_dyn_nh<D, B, true, true>(p, t, grid, smem, st)
-                 : launch_dyn_nh<D, B, true, false>(p, t, grid, smem, st);
+                             bool f8mma, bool sc, long long grid, size_t smem, cudaStream_t st) {
+    if (!fp8) return launch_dyn_nh<D, B, false, false>(p, t, sc, grid, smem, st);
+    return f8mma ? launch_dyn_nh<D, B, true, true>(p, t, sc, grid, smem, st)
+                 : launch_dyn_nh<D, B, true, false>(p, t, sc, grid, smem, st);
 }
 
 cudaError_t launch_dyn_any(const pa::DecodeParams& p, const pa::DynParams& t, int D, int B,
-                           bool fp8, bool f8mma, long long grid, size_t smem, cudaStream_t st) {
-    if (D == 64) return B == 16 ? launch_dyn_dtype<64, 16>(p, t, fp8, f8mma, grid, smem, st)
-                                : launch_dyn_dtype<64, 32>(p, t, fp8, f8mma, grid, smem, st);
-    return B == 16 ? launch_dyn_dtype<128, 16>(p, t, fp8, f8mma, grid, smem, st)
-                   : launch_dyn_dtype<128, 32>(p, t, fp8, f8mma, grid, smem, st);
+                           bool fp8, bool f8mma, bool sc, long long grid, size_t smem,
+                           cudaStream_t st) {
+    if (D == 64) return B == 16 ? launch_dyn_dtype<64, 16>(p, t, fp8, f8mma, sc, grid, smem, st)
+                                : launch_dyn_dtype<64, 32>(p, t, fp8, f8mma, sc, grid, smem, st);
+    return B == 16 ? launch_dyn_dtype<128, 16>(p, t, fp8, f8mma, sc, grid, smem, st)
+                   : launch_dyn_dtype<128, 32>(p, t, fp8, f8mma, sc, grid, smem, st);
 }
 
 cudaError_t launch_combine(const pa::CombineParams& c, int D, cudaStream_t st) {
@@ -664,6 +680,7 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool f8mma = opts && opts->fp8_compute && kv_dtype == PA_KV_FP8_E4M3;
+    const bool sc = opts && opts->mha_cuda_cores;
     if (pl.dynamic) {
         // [header: status, ..., generation / unit cursor / warps finished at
         //  byte 64][unit counters, 16 bytes per unit][partials: rows x slots]
@@ -690,7 +707,7 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
         p.ws_m = dpart + drows * head_size;
         p.ws_l = p.ws_m + drows;
         cudaError_t e = launch_dyn_any(p, t, head_size, block_size, kv_dtype == PA_KV_FP8_E4M3,
-                                       f8mma, pl.grid_ctas, pl.smem_bytes, s);
+                                       f8mma, sc, pl.grid_ctas, pl.smem_bytes, s);
         if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
         pa::CombineParams c;
         std::memset(&c, 0, sizeof c);
@@ -717,7 +734,7 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
         if (e != cudaSuccess) return fail(PA_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
         return PA_OK;
     }
-    cudaError_t e = launch_any(p, head_size, block_size, kv_dtype == PA_KV_FP8_E4M3, f8mma,
+    cudaError_t e = launch_any(p, head_size, block_size, kv_dtype == PA_KV_FP8_E4M3, f8mma, sc,
                                pl.grid_ctas, pl.smem_bytes, s);
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
     if (pl.balanced || pl.num_partitions > 1 || p.prefix_pages > 0) {

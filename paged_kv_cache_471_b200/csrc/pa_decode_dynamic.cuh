@@ -127,17 +127,18 @@ __device__ __forceinline__ uint32_t tagged_add(unsigned long long* w, uint32_t g
     return 0xffffffffu;
 }
 
-template <int D, int B, bool FP8, int NH, int W, bool F8MMA>
+// SC: one query head per kv head on the CUDA cores (WarpAttnScalar).
+template <int D, int B, bool FP8, int NH, int W, bool F8MMA, bool SC = false>
 __global__ void __launch_bounds__(W * 32,
-                                  (pair_pages<D, B, FP8, F8MMA>() && !F8MMA && NH == 1) ? 3 : 1)
+                                  ((pair_pages<D, B, FP8, F8MMA>() && !F8MMA && NH == 1) || SC) ? 3
+                                                                                                : 1)
     pa_decode_dyn_kernel(const DecodeParams p, const __grid_constant__ DynParams t) {
     static_assert(!F8MMA || FP8, "e4m3 MMAs need e4m3 pages");
-    using WA = WarpAttn<D, B, FP8, NH, F8MMA>;
+    static_assert(!SC || (!FP8 && NH == 1), "the CUDA-core form takes bf16 pages and one head");
+    using WA = std::conditional_t<SC, WarpAttnScalar<D, B>, WarpAttn<D, B, FP8, NH, F8MMA>>;
     constexpr int PAGE = WA::PAGE;
     constexpr int NPG = WA::NPG;
     constexpr bool PAIR = WA::PAIR;
-    constexpr int KT = WA::KT;
-    constexpr int MT = WA::MT;
     constexpr int STAGE = 2 * PAGE * NPG;
 
     extern __shared__ __align__(128) uint8_t smem[];
@@ -396,74 +397,18 @@ __global__ void __launch_bounds__(W * 32,
     auto begin_unit = [&](int u, int slot) {
         cu = unit_ref<B>(p, t, u);
         cslot = slot;
-        uint32_t qraw[2][KT][2];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const long long qr = (r < NH) ? row_of(cu, 8 * r + gq) : -1;
-            const bool ok = qr >= 0;
-            const uint16_t* qrow = p.q + (ok ? qr : 0) * D;
-#pragma unroll
-            for (int kt = 0; kt < KT; ++kt) {
-                uint32_t w0 = 0, w1 = 0;
-                if (ok) {
-                    if constexpr (!FP8) {
-                        const unsigned int* qw = reinterpret_cast<const unsigned int*>(qrow);
-                        w0 = __ldg(qw + 8 * kt + cq);
-                        w1 = __ldg(qw + 8 * kt + 4 + cq);
-                    } else {
-                        const uint2 w =
-                            __ldg(reinterpret_cast<const uint2*>(qrow + 16 * kt + 4 * cq));
-                        w0 = w.x;
-                        w1 = w.y;
-                    }
-                }
-                qraw[r][kt][0] = w0;
-                qraw[r][kt][1] = w1;
-            }
-        }
-        wa.load_q(qraw, p.scale_log2, k_scale, v_scale);
-#pragma unroll
-        for (int r = 0; r < NH; ++r) {
-            const long long qr = row_of(cu, 8 * r + gq);
-            wa.slope2[r] =
-                (has_alibi && qr >= 0) ? __ldg(p.alibi + qr % p.Hq) * 1.4426950408889634f : 0.f;
-        }
+        auto rows = [&](int lr) { return row_of(cu, lr); };
+        wa.fetch_query(p.q, rows);
+        wa.set_alibi(p.alibi, p.Hq, rows);
+        wa.finish_query(p.scale_log2, k_scale, v_scale);
         wa.reset();
     };
 
     // The unit's partial for this warp's slot: o = acc / l (times the output
     // multiplier) and (max, sum); `dead` leaves an empty partial instead.
     auto finish_unit = [&](bool dead) {
-        const int rows_here = rows_of(cu);
-#pragma unroll
-        for (int hr = 0; hr < NH; ++hr) {
-            float l = wa.l_run[hr];
-            l += __shfl_xor_sync(kFull, l, 1);
-            l += __shfl_xor_sync(kFull, l, 2);
-            const float lh[2] = {__shfl_sync(kFull, l, 8 * cq), __shfl_sync(kFull, l, 8 * cq + 4)};
-            const float mh[2] = {__shfl_sync(kFull, wa.m_run[hr], 8 * cq),
-                                 __shfl_sync(kFull, wa.m_run[hr], 8 * cq + 4)};
-#pragma unroll
-            for (int e1 = 0; e1 < 2; ++e1) {
-                const int h = 8 * hr + 2 * cq + e1;
-                if (h >= rows_here) continue;
-                const long long prow = prow_of(row_of(cu, h), cu.pre, cslot);
-                const float L = dead ? 0.f : lh[e1];
-                const float inv = L > 0.f ? wa.out_mul / L : 0.f;
-                if (!dead) {
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                        for (int e2 = 0; e2 < 2; ++e2)
-                            p.ws_o[prow * D + 16 * mt + gq + 8 * e2] =
-                                wa.acc[mt][hr][e1 + 2 * e2] * inv;
-                }
-                if (gq == 0) {
-                    p.ws_m[prow] = mh[e1];
-                    p.ws_l[prow] = L;
-                }
-            }
-        }
+        wa.write_partial(p.ws_o, p.ws_m, p.ws_l, rows_of(cu),
+                         [&](int h) { return prow_of(row_of(cu, h), cu.pre, cslot); }, dead);
     };
 
     // ------------------------------------------------------------ the ring

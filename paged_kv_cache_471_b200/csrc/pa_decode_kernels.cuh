@@ -164,6 +164,53 @@ struct WarpAttn {
         hi_half = cq >= 2;
     }
 
+    uint32_t qraw[2][KT][2];  // raw query words until finish_query
+
+    // Start loading the query rows row_of(8r + gq) (-1: none) in the order
+    // the fragments use them; finish_query turns them into MMA operands.
+    template <class RowFn>
+    __device__ __forceinline__ void fetch_query(const uint16_t* q, RowFn row_of) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const long long qr = (r < NH) ? row_of(8 * r + gq) : -1;
+            const bool ok = qr >= 0;
+            const uint16_t* qrow = q + (ok ? qr : 0) * D;
+#pragma unroll
+            for (int kt = 0; kt < KT; ++kt) {
+                uint32_t w0 = 0, w1 = 0;
+                if (ok) {
+                    if constexpr (!FP8) {
+                        const unsigned int* qw = reinterpret_cast<const unsigned int*>(qrow);
+                        w0 = __ldg(qw + 8 * kt + cq);
+                        w1 = __ldg(qw + 8 * kt + 4 + cq);
+                    } else {
+                        const uint2 w =
+                            __ldg(reinterpret_cast<const uint2*>(qrow + 16 * kt + 4 * cq));
+                        w0 = w.x;
+                        w1 = w.y;
+                    }
+                }
+                qraw[r][kt][0] = w0;
+                qraw[r][kt][1] = w1;
+            }
+        }
+    }
+
+    __device__ __forceinline__ void finish_query(float scale_log2, float k_scale, float v_scale) {
+        load_q(qraw, scale_log2, k_scale, v_scale);
+    }
+
+    // ALiBi: the logit of token t gains slope * (t - (T - 1)); slopes of rows
+    // row_of(8r + gq), kept in log2 units (0 without ALiBi).
+    template <class RowFn>
+    __device__ __forceinline__ void set_alibi(const float* alibi, int Hq, RowFn row_of) {
+#pragma unroll
+        for (int r = 0; r < NH; ++r) {
+            const long long qr = row_of(8 * r + gq);
+            slope2[r] = (alibi && qr >= 0) ? __ldg(alibi + qr % Hq) * 1.4426950408889634f : 0.f;
+        }
+    }
+
     // Q fragments (A operand of S = Q K^T; rows = heads 8r + gq) from the raw
     // bf16 query words of rows 8r + gq, in the order the fragments use, and
     // the logit multiplier (log2 domain) and output multiplier that go with them.
@@ -252,6 +299,76 @@ struct WarpAttn {
                 }
             qk_mul = scale_log2 * k_scale * up;
             out_mul = v_scale;
+        }
+    }
+
+    // Sum each row's l over its quad, so every thread of a quad holds its
+    // row's total (before the state leaves the warp).
+    __device__ __forceinline__ void reduce_l() {
+#pragma unroll
+        for (int r = 0; r < NH; ++r) {
+            l_run[r] += __shfl_xor_sync(kFull, l_run[r], 1);
+            l_run[r] += __shfl_xor_sync(kFull, l_run[r], 2);
+        }
+    }
+
+    // This warp's state for the CTA's merge (after reduce_l): row h of the
+    // accumulator at acc_rows[h * rs + d], each row's max and sum at m16[h]
+    // and l16[h] (sum 0 when zero_l).
+    __device__ __forceinline__ void store_merge(float* acc_rows, int rs, float* m16, float* l16,
+                                                bool zero_l) const {
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int r = 0; r < NH; ++r) {
+                float* base = acc_rows + (8 * r + 2 * cq) * rs + 16 * mt + gq;
+                base[0] = acc[mt][r][0];
+                base[rs] = acc[mt][r][1];
+                base[8] = acc[mt][r][2];
+                base[rs + 8] = acc[mt][r][3];
+            }
+        if (cq == 0) {
+#pragma unroll
+            for (int r = 0; r < NH; ++r) {
+                m16[8 * r + gq] = m_run[r];
+                l16[8 * r + gq] = zero_l ? 0.f : l_run[r];
+            }
+        }
+    }
+
+    // This warp's state as a partial of each of its first `rows` rows:
+    // o = acc / l times the output multiplier at ws_o[prow(h) * D + d], and
+    // (max, sum) at ws_m / ws_l[prow(h)]; `dead` writes only an empty sum.
+    template <class RowFn>
+    __device__ __forceinline__ void write_partial(float* ws_o, float* ws_m, float* ws_l, int rows,
+                                                  RowFn prow, bool dead) const {
+#pragma unroll
+        for (int hr = 0; hr < NH; ++hr) {
+            float l = l_run[hr];
+            l += __shfl_xor_sync(kFull, l, 1);
+            l += __shfl_xor_sync(kFull, l, 2);
+            const float lh[2] = {__shfl_sync(kFull, l, 8 * cq), __shfl_sync(kFull, l, 8 * cq + 4)};
+            const float mh[2] = {__shfl_sync(kFull, m_run[hr], 8 * cq),
+                                 __shfl_sync(kFull, m_run[hr], 8 * cq + 4)};
+#pragma unroll
+            for (int e1 = 0; e1 < 2; ++e1) {
+                const int h = 8 * hr + 2 * cq + e1;
+                if (h >= rows) continue;
+                const long long pr = prow(h);
+                const float L = dead ? 0.f : lh[e1];
+                const float inv = L > 0.f ? out_mul / L : 0.f;
+                if (!dead) {
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                        for (int e2 = 0; e2 < 2; ++e2)
+                            ws_o[pr * D + 16 * mt + gq + 8 * e2] = acc[mt][hr][e1 + 2 * e2] * inv;
+                }
+                if (gq == 0) {
+                    ws_m[pr] = mh[e1];
+                    ws_l[pr] = L;
+                }
+            }
         }
     }
 
@@ -551,13 +668,229 @@ struct WarpAttn {
     }
 };
 
+// One query head per kv head (MHA), bf16 pages: the same contract as
+// WarpAttn, with q.K and P.V on the CUDA cores instead of tensor-core tiles
+// whose 16 rows would hold one real head.  A stage holds BT = 16 or 32
+// tokens (two 16-token pages of head size 64 are paired):
+//   * q.K: lane l takes head dims [part DL, (part + 1) DL), part = l / 8,
+//     DL = D / 4, and tokens l % 8 + 8 j, reading each token's 16-byte
+//     column groups of the K page (8 consecutive head dims); the 8 lanes of
+//     a shared-memory phase read 8 different tokens, so 8 different banks.
+//     Two xor shuffles add the four parts;
+//   * softmax in fp32 over the stage's tokens with xor shuffles;
+//   * P.V: the weights go through the first bytes of the stage's (already
+//     read) K page and come back as broadcast float4 loads; lane l owns head
+//     dims l + 32 i and reads its V rows' 16-byte pieces in an order that
+//     keeps the 8 lanes of a phase on distinct banks.
+// The weights stay fp32 (not rounded to bf16 as the MMA operands are).
+template <int D, int B>
+struct WarpAttnScalar {
+    static constexpr bool PAIR = pair_pages<D, B, false, false>();
+    static constexpr int NPG = PAIR ? 2 : 1;  // logical pages per stage
+    static constexpr int BT = B * NPG;        // tokens per stage
+    static constexpr int PAGE = D * B * 2;    // one bf16 K (or V) page of one kv head
+    static constexpr int CHUNK = B * 16;      // bytes of one 16-byte column group of a K page
+    static constexpr int DL = D / 4;          // head dims per lane in q.K
+    static constexpr int TJ = BT / 8;         // tokens per lane in q.K
+    static constexpr int DV = D / 32;         // head dims per lane in P.V
+
+    int lane, tl, part;
+    uint4 qw[DL / 8];  // raw query words until finish_query
+    float q[DL];
+    float qk_mul, out_mul;
+    float slope2[1];
+    float m_run[1], l_run[1];
+    float acc[DV];
+
+    __device__ __forceinline__ explicit WarpAttnScalar(int lane_) {
+        lane = lane_;
+        tl = lane & 7;
+        part = lane >> 3;
+    }
+
+    template <class RowFn>
+    __device__ __forceinline__ void fetch_query(const uint16_t* qp, RowFn row_of) {
+        const long long qr = row_of(0);
+        const uint4* src = reinterpret_cast<const uint4*>(qp + (qr >= 0 ? qr : 0) * D + part * DL);
+#pragma unroll
+        for (int c = 0; c < DL / 8; ++c) qw[c] = qr >= 0 ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    }
+
+    __device__ __forceinline__ void finish_query(float scale_log2, float, float) {
+#pragma unroll
+        for (int c = 0; c < DL / 8; ++c) {
+            const uint32_t w[4] = {qw[c].x, qw[c].y, qw[c].z, qw[c].w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                q[8 * c + 2 * k] = bf16_lo(w[k]);
+                q[8 * c + 2 * k + 1] = bf16_hi(w[k]);
+            }
+        }
+        qk_mul = scale_log2;
+        out_mul = 1.f;
+    }
+
+    template <class RowFn>
+    __device__ __forceinline__ void set_alibi(const float* alibi, int Hq, RowFn row_of) {
+        const long long qr = row_of(0);
+        slope2[0] = (alibi && qr >= 0) ? __ldg(alibi + qr % Hq) * 1.4426950408889634f : 0.f;
+    }
+
+    __device__ __forceinline__ void reset() {
+        m_run[0] = -INFINITY;
+        l_run[0] = 0.f;
+#pragma unroll
+        for (int i = 0; i < DV; ++i) acc[i] = 0.f;
+    }
+
+    // Every lane holds the row's sum already.
+    __device__ __forceinline__ void reduce_l() {}
+
+    __device__ __forceinline__ void store_merge(float* acc_rows, int, float* m16, float* l16,
+                                                bool zero_l) const {
+#pragma unroll
+        for (int i = 0; i < DV; ++i) acc_rows[lane + 32 * i] = acc[i];
+        if (lane == 0) {
+            m16[0] = m_run[0];
+            l16[0] = zero_l ? 0.f : l_run[0];
+        }
+    }
+
+    template <class RowFn>
+    __device__ __forceinline__ void write_partial(float* ws_o, float* ws_m, float* ws_l, int rows,
+                                                  RowFn prow, bool dead) const {
+        if (rows < 1) return;
+        const long long pr = prow(0);
+        const float L = dead ? 0.f : l_run[0];
+        const float inv = L > 0.f ? out_mul / L : 0.f;
+        if (!dead) {
+#pragma unroll
+            for (int i = 0; i < DV; ++i) ws_o[pr * D + lane + 32 * i] = acc[i] * inv;
+        }
+        if (lane == 0) {
+            ws_m[pr] = m_run[0];
+            ws_l[pr] = L;
+        }
+    }
+
+    template <bool FULL, bool ALIBI>
+    __device__ __forceinline__ void page(const uint32_t kbase, const int valid, const int valid2,
+                                         const int pos0) {
+        const uint32_t vbase = kbase + NPG * PAGE;
+        // ---------------- logits of tokens tl + 8 j (this lane's quarter of the head dims)
+        float x[TJ];
+#pragma unroll
+        for (int j = 0; j < TJ; ++j) {
+            const int tok = tl + 8 * j;
+            const int pg = PAIR ? tok / B : 0;
+            const uint32_t kp = kbase + pg * PAGE + (tok % B) * 16 + part * (DL / 8) * CHUNK;
+            float sc = 0.f;
+#pragma unroll
+            for (int c = 0; c < DL / 8; ++c) {
+                const uint4 w = lds128(kp + c * CHUNK);
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    sc = fmaf(q[8 * c + 2 * k], bf16_lo(ww[k]), sc);
+                    sc = fmaf(q[8 * c + 2 * k + 1], bf16_hi(ww[k]), sc);
+                }
+            }
+            sc += __shfl_xor_sync(kFull, sc, 8);
+            sc += __shfl_xor_sync(kFull, sc, 16);
+            float v = sc * qk_mul;
+            if constexpr (ALIBI) v = fmaf(slope2[0], static_cast<float>(pos0 + tok), v);
+            if constexpr (!FULL) {
+                const bool counts = PAIR ? (tok < B ? tok < valid : tok - B < valid2) : tok < valid;
+                if (!counts) v = -INFINITY;
+            }
+            x[j] = v;
+        }
+        // ---------------- online softmax over the stage's tokens
+        float mx = x[0];
+#pragma unroll
+        for (int j = 1; j < TJ; ++j) mx = fmaxf(mx, x[j]);
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+        const float m_new = fmaxf(m_run[0], mx);
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        const bool grew = m_new > m_run[0];
+        const float alpha = fast_exp2(m_run[0] - m_use);
+        m_run[0] = m_new;
+        float pw[TJ];
+        float ls = 0.f;
+#pragma unroll
+        for (int j = 0; j < TJ; ++j) {
+            pw[j] = fast_exp2(x[j] - m_use);
+            ls += pw[j];
+        }
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) ls += __shfl_xor_sync(kFull, ls, o);
+        l_run[0] = l_run[0] * alpha + ls;
+        if (grew) {
+#pragma unroll
+            for (int i = 0; i < DV; ++i) acc[i] *= alpha;
+        }
+        // ---------------- weights to every lane through the stage's K page
+        __syncwarp();  // every lane has read its K words
+        if (part == 0) {
+#pragma unroll
+            for (int j = 0; j < TJ; ++j) sts32(kbase + 4 * (tl + 8 * j), __float_as_uint(pw[j]));
+        }
+        __syncwarp();
+        float pv[BT];
+#pragma unroll
+        for (int c = 0; c < BT / 4; ++c) {
+            const uint4 w = lds128(kbase + 16 * c);
+            pv[4 * c] = __uint_as_float(w.x);
+            pv[4 * c + 1] = __uint_as_float(w.y);
+            pv[4 * c + 2] = __uint_as_float(w.z);
+            pv[4 * c + 3] = __uint_as_float(w.w);
+        }
+        // ---------------- O += V P for head dims lane + 32 i
+        // A V row of one page is PIECES 16-byte pieces of 8 tokens.  Lanes of
+        // one 8-lane shared-memory phase start on different pieces (rot), so
+        // their loads land on distinct banks; the piece index is then a
+        // run-time value, and each weight is picked from the pieces' weights.
+        constexpr int PIECES = B * 2 / 16;
+        const int rot = PIECES == 2 ? (lane >> 2) & 1 : (lane >> 1) & 3;
+#pragma unroll
+        for (int pgv = 0; pgv < NPG; ++pgv) {
+            const int cnt = FULL ? B : (pgv == 0 ? valid : valid2);
+#pragma unroll
+            for (int i = 0; i < DV; ++i) {
+                const uint32_t row = vbase + pgv * PAGE + (lane + 32 * i) * (B * 2);
+#pragma unroll
+                for (int hh = 0; hh < PIECES; ++hh) {
+                    const int h = (hh + rot) % PIECES;
+                    const uint4 w = lds128(row + 16 * h);
+                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        float pj = pv[pgv * B + j];
+#pragma unroll
+                        for (int hc = 1; hc < PIECES; ++hc)
+                            pj = (h == hc) ? pv[pgv * B + 8 * hc + j] : pj;
+                        float v = (j & 1) ? bf16_hi(ww[j >> 1]) : bf16_lo(ww[j >> 1]);
+                        if constexpr (!FULL) v = 8 * h + j < cnt ? v : 0.f;  // slots past the end may hold NaN
+                        acc[i] = fmaf(pj, v, acc[i]);
+                    }
+                }
+            }
+        }
+    }
+};
+
 // The paired 8-row form with f16 MMAs is held to three CTAs per SM (170
 // registers), the residency of the other 8-row forms.
-template <int D, int B, bool FP8, int NH, int W, bool F8MMA>
+// SC: one query head per kv head on the CUDA cores (WarpAttnScalar).
+template <int D, int B, bool FP8, int NH, int W, bool F8MMA, bool SC = false>
 __global__ void __launch_bounds__(W * 32,
-                                  (pair_pages<D, B, FP8, F8MMA>() && !F8MMA && NH == 1) ? 3 : 1)
+                                  ((pair_pages<D, B, FP8, F8MMA>() && !F8MMA && NH == 1) || SC) ? 3
+                                                                                                : 1)
     pa_decode_kernel(const DecodeParams p) {
     static_assert(!F8MMA || FP8, "e4m3 MMAs need e4m3 pages");
+    static_assert(!SC || (!FP8 && NH == 1), "the CUDA-core form takes bf16 pages and one head");
+    using WA = std::conditional_t<SC, WarpAttnScalar<D, B>, WarpAttn<D, B, FP8, NH, F8MMA>>;
     constexpr int ELEM = FP8 ? 1 : 2;
     constexpr int K32 = D / 32;  // 32-wide k-steps over the head dim (e4m3 MMA)
     constexpr int PAGE = D * B * ELEM;  // one K (or V) page of one kv head
@@ -765,46 +1098,16 @@ __global__ void __launch_bounds__(W * 32,
         int win_b = load_win(32, 0);
         int win_a2 = PAIR ? load_win(0, 1) : -1;
         int win_b2 = PAIR ? load_win(32, 1) : -1;
-        // Raw query words of rows 8r + gq, in the order the fragments use.
-        uint32_t qraw[2][KT][2];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const long long qr = (r < NH) ? row_of(8 * r + gq) : -1;
-            const bool ok = qr >= 0;
-            const uint16_t* qrow = p.q + (ok ? qr : 0) * D;
-#pragma unroll
-            for (int kt = 0; kt < KT; ++kt) {
-                uint32_t w0 = 0, w1 = 0;
-                if (ok) {
-                    if constexpr (!FP8) {
-                        const unsigned int* qw = reinterpret_cast<const unsigned int*>(qrow);
-                        w0 = __ldg(qw + 8 * kt + cq);
-                        w1 = __ldg(qw + 8 * kt + 4 + cq);
-                    } else {
-                        const uint2 w =
-                            __ldg(reinterpret_cast<const uint2*>(qrow + 16 * kt + 4 * cq));
-                        w0 = w.x;
-                        w1 = w.y;
-                    }
-                }
-                qraw[r][kt][0] = w0;
-                qraw[r][kt][1] = w1;
-            }
-        }
+        // The query rows, as MMA operands (or CUDA-core registers) later.
+        WA wa(lane);
+        wa.fetch_query(p.q, row_of);
         float k_scale = 1.f, v_scale = 1.f;
         if constexpr (FP8) {
             k_scale = __ldg(p.k_scale);
             v_scale = __ldg(p.v_scale);
         }
-        // ALiBi: logit of token t gains slope * (t - (T - 1)); kept in log2 units.
         const bool has_alibi = p.alibi != nullptr;
-        float slope2[NH];
-#pragma unroll
-        for (int r = 0; r < NH; ++r) {
-            const long long qr = row_of(8 * r + gq);
-            slope2[r] =
-                (has_alibi && qr >= 0) ? __ldg(p.alibi + qr % p.Hq) * 1.4426950408889634f : 0.f;
-        }
+        wa.set_alibi(p.alibi, p.Hq, row_of);
 
         // ---- sequence length, with the device-side range checks
         int T, nb;
@@ -907,10 +1210,7 @@ __global__ void __launch_bounds__(W * 32,
         const int n_pro = n_my < NS ? n_my : NS;
         for (int i = 0; i < n_pro; ++i) issue(i);
 
-        WarpAttn<D, B, FP8, NH, F8MMA> wa(lane);
-        wa.load_q(qraw, p.scale_log2, k_scale, v_scale);
-#pragma unroll
-        for (int r = 0; r < NH; ++r) wa.slope2[r] = slope2[r];
+        wa.finish_query(p.scale_log2, k_scale, v_scale);
         wa.reset();
 
         bool timed_out = false;
@@ -962,34 +1262,13 @@ __global__ void __launch_bounds__(W * 32,
         }
 
         // ---------------- merge the four warps' partial softmax states
-#pragma unroll
-        for (int r = 0; r < NH; ++r) {
-            wa.l_run[r] += __shfl_xor_sync(kFull, wa.l_run[r], 1);
-            wa.l_run[r] += __shfl_xor_sync(kFull, wa.l_run[r], 2);
-        }
+        wa.reduce_l();
         __syncthreads();  // every warp is done with its stages
         float* s_acc = reinterpret_cast<float*>(smem);
         float* s_m = s_acc + W * NH * 8 * RS;
         float* s_l = s_m + W * 16;
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-            for (int r = 0; r < NH; ++r) {
-                const int h = 8 * r + 2 * cq;
-                const int d = 16 * mt + gq;
-                float* base = s_acc + (warp * NH * 8 + h) * RS + d;
-                base[0] = wa.acc[mt][r][0];
-                base[RS] = wa.acc[mt][r][1];
-                base[8] = wa.acc[mt][r][2];
-                base[RS + 8] = wa.acc[mt][r][3];
-            }
-        if (cq == 0) {
-#pragma unroll
-            for (int r = 0; r < NH; ++r) {
-                s_m[warp * 16 + 8 * r + gq] = wa.m_run[r];
-                s_l[warp * 16 + 8 * r + gq] = timed_out ? 0.f : wa.l_run[r];
-            }
-        }
+        wa.store_merge(s_acc + warp * NH * 8 * RS, RS, s_m + warp * 16, s_l + warp * 16,
+                       timed_out);
         __syncthreads();
 
         const int rows_here = pre ? min(16, rows_total - rg * 16) : p.G;
