@@ -213,7 +213,7 @@ def workload_config(idx: int, num_seqs: int = 0):
 
 def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, num_seqs=0,
              cascade=True, alibi=False, schedule="auto", min_region_ms=0.0,
-             min_clock_samples=12, extras=True, mha_cuda_cores=False):
+             min_clock_samples=12, extras=True, mha_cuda_cores=False, fp8_compute=False):
     import torch
 
     import paged_kv_cache_471_b200 as pa
@@ -231,8 +231,10 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
                                for i in range(cfg.num_heads)], dtype=torch.float32, device=device)
     if prefix and schedule == "balanced":
         schedule = "auto"  # balanced ranges do not take a shared prefix
+    fp8_compute = fp8_compute and cfg.kv_dtype == W.FP8_E4M3
     plan = pa.plan(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_size, cfg.block_size,
-                   cfg.max_seq_len, cfg.kv_dtype, shared_prefix_blocks=prefix, schedule=schedule)
+                   cfg.max_seq_len, cfg.kv_dtype, shared_prefix_blocks=prefix, schedule=schedule,
+                   fp8_compute=fp8_compute)
     ws = torch.zeros(plan["workspace_bytes"], dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
     alg_bytes = bytes_of(wl)
@@ -245,7 +247,7 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
                   wl.block_tables, wl.seq_lens, cfg.block_size, cfg.max_seq_len, cfg.kv_dtype,
                   wl.k_scale, wl.v_scale, workspace_tensor=ws, stream=stream,
                   shared_prefix_blocks=prefix, alibi_slopes=slopes, schedule=schedule,
-                  mha_cuda_cores=mha_cuda_cores)
+                  mha_cuda_cores=mha_cuda_cores, fp8_compute=fp8_compute)
 
     for _ in range(max(warmup, 3)):
         if flush:
@@ -343,7 +345,7 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
                                            wl.seq_lens, cfg.block_size, cfg.max_seq_len,
                                            cfg.kv_dtype, wl.k_scale, wl.v_scale,
                                            workspace_tensor=ws, stream=st, schedule=schedule,
-                                           mha_cuda_cores=mha_cuda_cores)
+                                           mha_cuda_cores=mha_cuda_cores, fp8_compute=fp8_compute)
             step_on(gs)  # warm on the capture stream
             gs.synchronize()
             with torch.cuda.graph(graph, stream=gs):
@@ -371,7 +373,9 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
                steps=steps, clocks=clocks, status=status,
                launches_per_step=1 + (plan["num_partitions"] > 1 or prefix > 0
                                       or plan["balanced"] == 1 or plan["dynamic"] == 1),
-               shared_prefix_blocks=prefix, alibi=alibi, extra=extra)
+               shared_prefix_blocks=prefix, alibi=alibi, extra=extra,
+               options={"schedule": schedule, "mha_cuda_cores": bool(mha_cuda_cores),
+                        "fp8_compute": bool(fp8_compute)})
 
     if want_e2e:
         # End to end through the public call, as a serving loop runs it: every
@@ -412,7 +416,7 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
                           cfg.scale, bt_d[b], sl_d[b], cfg.block_size, cfg.max_seq_len,
                           cfg.kv_dtype, wl.k_scale, wl.v_scale, workspace_tensor=ws,
                           stream=stream, shared_prefix_blocks=prefix, alibi_slopes=slopes,
-                          schedule=schedule, mha_cuda_cores=mha_cuda_cores)
+                          schedule=schedule, mha_cuda_cores=mha_cuda_cores, fp8_compute=fp8_compute)
                 ev_used[b].record(stream)
                 with torch.cuda.stream(down):
                     down.wait_event(ev_used[b])
@@ -540,6 +544,7 @@ def result_line(idx, r, n_gpus, steps, warmup, cpu=None):
         "plan": r["plan"],
         "shared_prefix_blocks_declared": r["shared_prefix_blocks"],
         "alibi": r["alibi"],
+        "options": r["options"],
         **({"small_workload": {
             **r["extra"],
             "warm_l2_back_to_back_gbs": round(r["alg_bytes"] / (r["extra"]["warm_l2_back_to_back_ms_per_call"] * 1e-3) / 1e9, 2),
@@ -713,6 +718,8 @@ def main(argv=None):
     ap.add_argument("--schedule", default="auto",
                     choices=["auto", "balanced", "partitioned", "dynamic"],
                     help="how CTAs share the work (pa_options.schedule)")
+    ap.add_argument("--fp8-compute", action="store_true",
+                    help="e4m3 x e4m3 tensor-core products for an FP8 cache (pa_options.fp8_compute)")
     ap.add_argument("--mha-cuda-cores", action="store_true",
                     help="q.K and P.V on the CUDA cores for one query head per kv head")
     ap.add_argument("--no-cascade", action="store_true",
@@ -749,7 +756,8 @@ def main(argv=None):
     for idx in cfg_ids:
         r = time_gpu(idx, args.steps, args.warmup, device, want_e2e=not args.no_e2e, rank=rank,
                      num_seqs=args.num_seqs, cascade=not args.no_cascade, alibi=args.alibi,
-                     schedule=args.schedule, mha_cuda_cores=args.mha_cuda_cores)
+                     schedule=args.schedule, mha_cuda_cores=args.mha_cuda_cores,
+                     fp8_compute=args.fp8_compute)
         r["step_ms"] = reduce_max(r["step_ms"], device)
         if "e2e_ms" in r:
             r["e2e_ms"] = reduce_max(r["e2e_ms"], device)
@@ -762,7 +770,8 @@ def main(argv=None):
         # One GPU, one workload asked for: the line also carries every
         # workload's figures (each its own timed region of >= 0.3 s).
         if (ws == 1 and len(cfg_ids) == 1 and not args.no_per_config and not args.num_seqs
-                and not args.alibi and args.schedule == "auto" and not args.mha_cuda_cores):
+                and not args.alibi and args.schedule == "auto" and not args.mha_cuda_cores
+                and not args.fp8_compute):
             per = {}
             for j in (1, 2, 3, 4, 5):
                 rj = time_gpu(j, args.steps, args.warmup, device, want_e2e=False,

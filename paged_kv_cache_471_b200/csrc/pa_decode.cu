@@ -161,8 +161,10 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         const long long n_units = units_pre + units;
         if (n_units >= (1ll << 30) || static_cast<long long>(num_seqs) * num_heads >= (1ll << 31))
             return fail(PA_ERR_INVALID_ARG, "%s", "batch too large for the dynamic schedule");
+        // Slots per unit: enough that the last units can take every warp as a
+        // helper (twice the warps per unit, plus 8).
         const long long warps = slots * W;
-        long long kslots = n_units > 0 ? 2 * ((warps + n_units - 1) / n_units) + 2 : 2;
+        long long kslots = n_units > 0 ? (2 * warps + n_units - 1) / n_units + 8 : 2;
         if (kslots > kMaxDynSlots) kslots = kMaxDynSlots;
         const long long k_total = (cascade ? 2 : 1) * kslots;
         const size_t dsmem = static_cast<size_t>(W) * ns * (stage + 8 + 16);

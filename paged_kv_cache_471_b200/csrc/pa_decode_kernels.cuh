@@ -1432,15 +1432,35 @@ __global__ void __launch_bounds__(kThreads) pa_combine_kernel(const CombineParam
 #pragma unroll
     for (int i = 0; i < PER; ++i) a[i] = 0.f;
     float L = 0.f;
-    for (int i = 0; i < nps; ++i) {
-        const long long r = slot_row(i);
-        const float l = p.ws_l[r];
-        if (!(l > 0.f)) continue;
-        const float wt = exp2f(p.ws_m[r] - M) * l;
-        L += wt;
-        const float* o = p.ws_o + r * D;
+    // Slots in groups of 32: each lane loads one slot's (max, sum) and forms
+    // its weight, then the group's partial rows are read with the weights
+    // broadcast.  Every row is loaded (an empty slot's may hold anything) and
+    // an empty slot's contribution is dropped by a select, so the loads of
+    // consecutive slots are independent and several are in flight at once.
+    for (int i0 = 0; i0 < nps; i0 += 32) {
+        const int n = min(32, nps - i0);
+        float wt = 0.f;
+        long long rl = 0;
+        if (lane < n) {
+            rl = slot_row(i0 + lane);
+            const float l = p.ws_l[rl];
+            if (l > 0.f) wt = exp2f(p.ws_m[rl] - M) * l;
+        }
+        float wsum = wt;
 #pragma unroll
-        for (int j = 0; j < PER; ++j) a[j] += wt * o[lane + 32 * j];
+        for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(kFull, wsum, o);
+        L += wsum;
+#pragma unroll 4
+        for (int k = 0; k < n; ++k) {
+            const float w = __shfl_sync(kFull, wt, k);
+            const long long r = __shfl_sync(kFull, rl, k);
+            const float* o = p.ws_o + r * D;
+#pragma unroll
+            for (int j = 0; j < PER; ++j) {
+                const float v = o[lane + 32 * j];
+                a[j] += w > 0.f ? w * v : 0.f;
+            }
+        }
     }
 #pragma unroll
     for (int j = 0; j < PER; ++j)

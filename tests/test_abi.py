@@ -266,7 +266,7 @@ def test_dynamic_schedule_plan_and_workspace():
         warps = p["grid_ctas"] * p["warps_per_cta"]
         groups = -(-(c.num_seqs * c.group) // 16) if pref else 0
         units = c.num_kv_heads * groups + c.num_seqs * c.num_kv_heads
-        k = min(64, 2 * -(-warps // units) + 2)
+        k = min(64, -(-2 * warps // units) + 8)
         assert p["num_partitions"] == k and p["prefix_partitions"] == (k if pref else 0)
         assert p["prefix_groups"] == groups
         k_total = k * (2 if pref else 1)
