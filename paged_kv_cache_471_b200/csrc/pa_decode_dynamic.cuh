@@ -16,7 +16,7 @@
 // head, group of 16 query rows) when a prefix is declared.  Each unit has a
 // page counter in the workspace.  A warp takes the next unit from a cursor
 // as its owner (partial slot 0), then claims ranges of its pages from the
-// unit's counter -- each range a few ring stages, fewer as the unit runs out
+// unit's counter -- each range a quarter of the pages left, 4 to 32 ring stages
 // -- and accumulates every page it reads in registers.  When its unit is
 // exhausted it takes the next unit from the cursor; once the cursor has
 // handed out every unit, it joins the unit with the most pages left as a
@@ -211,30 +211,41 @@ __global__ void __launch_bounds__(W * 32,
     size_t ihead = 0;
     int ra = 0, rn = 0, ri = 0;  // current range: pages ra .. ra + NPG * rn of the unit, next stage ri
     int win_a = -1, win_a2 = -1;  // block ids of the current range: lane l <-> stage l
+    int win_n = -1, win_n2 = -1;  // ... and of the next range, once loaded
     int nv = 0, nstep = 0;         // the next range's claim (count before it, pages)
+    int nv_b = 0;                  // its count, once read
     bool n_claimed = false;        // a next-range claim is in flight
+    bool n_loaded = false;         // the next range's block ids are in win_n
     bool cursor_done = false, exhausted = false;
     uint32_t valid_mask = 0;  // bit NPG * stage (+ 1): that page had a legal block id
 
     auto claim_step = [&](int left) {
-        int st = left / 8;
+        int st = left / 4;
         st = max(t.step_min, min(t.step_max, st));
         return (st + NPG - 1) / NPG * NPG;
     };
-    auto load_window = [&](int a, int n_stages) {
-        const int j = iu.j_base + a + NPG * lane;
+    // Block ids of range [v, v + step) of the current unit: lane l <-> stage l.
+    auto load_window = [&](int v, int step, int& w1, int& w2) {
+        const int n_stages = (min(v + step, iu.n) - v + NPG - 1) / NPG;
+        const int j = iu.j_base + v + NPG * lane;
         const int jend = iu.j_base + iu.n;
-        win_a = (lane < n_stages && j < jend) ? __ldg(ibt + j) : -1;
-        if constexpr (PAIR) win_a2 = (lane < n_stages && j + 1 < jend) ? __ldg(ibt + j + 1) : -1;
+        w1 = (lane < n_stages && j < jend) ? __ldg(ibt + j) : -1;
+        if constexpr (PAIR) w2 = (lane < n_stages && j + 1 < jend) ? __ldg(ibt + j + 1) : -1;
     };
     // Start issuing range [v, v + step) of the current unit (clipped to it);
-    // false when the unit has no pages there.
-    auto start_range = [&](int v, int step) -> bool {
+    // false when the unit has no pages there.  `preloaded`: its block ids are
+    // in win_n already.
+    auto start_range = [&](int v, int step, bool preloaded) -> bool {
         if (v >= iu.n) return false;
         ra = v;
         rn = (min(v + step, iu.n) - v + NPG - 1) / NPG;
         ri = 0;
-        load_window(ra, rn);
+        if (preloaded) {
+            win_a = win_n;
+            win_a2 = win_n2;
+        } else {
+            load_window(ra, step, win_a, win_a2);
+        }
         // Claim the range after this one now; its count is read when this
         // range runs out, so the atomic's latency is hidden.
         nstep = claim_step(iu.n - (v + step));
@@ -243,6 +254,7 @@ __global__ void __launch_bounds__(W * 32,
             nv = static_cast<int>(static_cast<uint32_t>(w));
         }
         n_claimed = true;
+        n_loaded = false;
         return true;
     };
     // Join unit u with slot `slot`: claim its first range.  A unit with no
@@ -270,7 +282,7 @@ __global__ void __launch_bounds__(W * 32,
             if (lane == 0) atomicOr(p.status, kDevTimeout);
             v = static_cast<uint32_t>(iu.n);
         }
-        if (!start_range(static_cast<int>(v), step)) {
+        if (!start_range(static_cast<int>(v), step, false)) {
             empty_partial(iu, slot);
             iu.u = -1;
             return false;
@@ -340,8 +352,8 @@ __global__ void __launch_bounds__(W * 32,
             bool ok = false;
             if (iu.u >= 0 && n_claimed) {  // the current unit's next range
                 n_claimed = false;
-                const int v = __shfl_sync(kFull, nv, 0);
-                ok = start_range(v, nstep);
+                const int v = n_loaded ? nv_b : __shfl_sync(kFull, nv, 0);
+                ok = start_range(v, nstep, n_loaded);
             }
             if (!ok) {
                 iu.u = -1;
@@ -352,6 +364,14 @@ __global__ void __launch_bounds__(W * 32,
             }
         }
         const int i = ri++;
+        // With the second stage of a range (the first, for a one-stage range)
+        // the next range's claim has returned: read its block ids now, so
+        // they are in registers when this range runs out.
+        if (n_claimed && !n_loaded && (i == 1 || rn == 1)) {
+            nv_b = __shfl_sync(kFull, nv, 0);
+            if (nv_b < iu.n) load_window(nv_b, nstep, win_n, win_n2);
+            n_loaded = true;
+        }
         const int jg = iu.j_base + ra + NPG * i;  // the stage's first page in the row
         const int pb = __shfl_sync(kFull, win_a, i);
         const int pb2 = PAIR ? __shfl_sync(kFull, win_a2, i) : -1;

@@ -36,7 +36,7 @@ class Model:
         self.slots = {}     # (unit, slot) -> (warp, pages read)
 
     def step(self, left):
-        st = max(self.step_min, min(self.step_max, left // 8))
+        st = max(self.step_min, min(self.step_max, left // 4))
         return st
 
     def warp(self, w):

@@ -49,7 +49,10 @@ def test_pa_decode_symbol_through_ctypes(idx):
     ctypes in the pages' argument order with a caller-allocated workspace;
     config 5 reduced is split by the planner, so the combine runs too."""
     import ctypes
-    cfg = REDUCED[idx].replace(shared_prefix_blocks=0)
+    cfg = REDUCED[idx]
+    if cfg.shared_prefix_blocks:  # same sizes, no prefix declared: a pool for it
+        cfg = W.reduced(idx, num_seqs=cfg.num_seqs, seq_len_hi=cfg.seq_len_hi,
+                        seq_len_lo=cfg.seq_len_lo, shared_prefix_blocks=0)
     wl = W.make_workload(cfg, DEV)
     L = pa.lib()
     code = pa.kv_dtype_code(cfg.kv_dtype)
