@@ -177,10 +177,11 @@ typedef struct pa_plan {
     int prefix_groups;      /* 16-query-row groups per kv head streaming the prefix     */
     int balanced;           /* 1: balanced page ranges (num_partitions and
                                partition_pages are then 0), 0: fixed partitions        */
-    int dynamic;            /* 1: the dynamic schedule; num_partitions and
-                               prefix_partitions are then the partial slots per query
-                               row of a (sequence, kv head) unit and of a prefix unit,
-                               partition_pages is 0, grid_ctas an upper bound          */
+    int dynamic;            /* > 0: the dynamic schedule, with this many owner warps
+                               per unit; num_partitions and prefix_partitions are then
+                               the partial slots per query row of a (sequence, kv head)
+                               unit and of a prefix unit, partition_pages is 0,
+                               grid_ctas an upper bound; 0: another schedule            */
 } pa_plan;
 
 /*

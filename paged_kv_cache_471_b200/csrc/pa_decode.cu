@@ -161,10 +161,14 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         const long long n_units = units_pre + units;
         if (n_units >= (1ll << 30) || static_cast<long long>(num_seqs) * num_heads >= (1ll << 31))
             return fail(PA_ERR_INVALID_ARG, "%s", "batch too large for the dynamic schedule");
-        // Slots per unit: enough that the last units can take every warp as a
-        // helper (twice the warps per unit, plus 8).
+        // Owners per unit: four when the batch has at least half as many units
+        // as warps (the four warps of a CTA per unit of the partitioned
+        // schedule), else one.  Slots per unit: the owners', and enough
+        // helpers that the last units can take every warp (twice the warps
+        // per unit, plus 8).
         const long long warps = slots * W;
-        long long kslots = n_units > 0 ? (2 * warps + n_units - 1) / n_units + 8 : 2;
+        const long long owners = 2 * n_units >= warps ? 4 : 1;
+        long long kslots = n_units > 0 ? owners + (2 * warps + n_units - 1) / n_units + 8 : 2;
         if (kslots > kMaxDynSlots) kslots = kMaxDynSlots;
         const long long k_total = (cascade ? 2 : 1) * kslots;
         const size_t dsmem = static_cast<size_t>(W) * ns * (stage + 8 + 16);
@@ -185,7 +189,7 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         pl->prefix_partitions = cascade ? static_cast<int>(kslots) : 0;
         pl->prefix_groups = static_cast<int>(groups);
         pl->balanced = 0;
-        pl->dynamic = 1;
+        pl->dynamic = static_cast<int>(owners);
         return PA_OK;
     }
     const bool br_fits = !cascade && !forced_pp && num_seqs > 0 &&
@@ -693,6 +697,7 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
         std::memset(&t, 0, sizeof t);
         t.units_pre = num_kv_heads * pl.prefix_groups;
         t.units = t.units_pre + num_seqs * num_kv_heads;
+        t.owners = pl.dynamic;
         t.k_pre = pl.prefix_partitions;
         t.k_own = pl.num_partitions;
         t.k_total = t.k_pre + t.k_own;
@@ -727,6 +732,7 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
         c.G = num_heads / num_kv_heads;
         c.dynamic = 1;
         c.dyn_units_pre = t.units_pre;
+        c.dyn_owners = t.owners;
         c.dyn_k_pre = t.k_pre;
         c.dyn_k_own = t.k_own;
         c.dyn_k_total = t.k_total;

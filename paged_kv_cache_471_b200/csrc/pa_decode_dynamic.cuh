@@ -14,13 +14,14 @@
 //
 // Units are (sequence, kv head) pairs, after the shared-prefix units (kv
 // head, group of 16 query rows) when a prefix is declared.  Each unit has a
-// page counter in the workspace.  A warp takes the next unit from a cursor
-// as its owner (partial slot 0), then claims ranges of its pages from the
-// unit's counter -- each range a quarter of the pages left, 4 to 32 ring stages
-// -- and accumulates every page it reads in registers.  When its unit is
-// exhausted it takes the next unit from the cursor; once the cursor has
-// handed out every unit, it joins the unit with the most pages left as a
-// helper (partial slot 1, 2, ...; at most K slots per unit), until no unit
+// page counter in the workspace.  A cursor hands every unit to `owners`
+// warps (partial slots 0 .. owners - 1): four for a batch with at least
+// half as many units as warps, as the four warps of a CTA share a unit in
+// pa_decode_kernel, else one.  A warp claims ranges of its unit's pages from
+// the unit's counter -- each range a quarter of the pages left, 4 to 32
+// ring stages -- and accumulates every page it reads in registers.  When its unit is exhausted it takes the next cursor entry; once
+// the cursor is spent, it joins as a helper (the next slots; at most K slots
+// per unit) the unit with the most pages left per warp on it, until no unit
 // has pages worth joining for.  Each (warp, unit) pair writes one fp32
 // partial (o = acc / l, max, sum) and pa_combine_kernel merges a row's
 // slots.  So a row has as many partials as warps read its unit: one for most
@@ -54,6 +55,7 @@ constexpr int kDynHeaderWord = 16;  // first of the dynamic schedule's header wo
 struct DynParams {
     int units_pre;    // shared-prefix units (0 without a prefix), numbered first
     int units;        // units_pre + num_seqs * num_kv_heads
+    int owners;       // warps the cursor hands each unit to (slots 0 .. owners - 1)
     int k_pre, k_own;  // partial slots per row of a prefix / per-sequence unit
     int k_total;       // k_pre + k_own: slots per query row (prefix slots first)
     int total_warps;   // warps of the grid
@@ -264,7 +266,7 @@ __global__ void __launch_bounds__(W * 32,
         islot = slot;
         ibt = p.bt + (iu.pre ? 0 : (long long)iu.s * p.max_blocks);
         ihead = static_cast<size_t>(iu.kvh) * PAGE;
-        if (slot == 0 && !iu.pre && iu.kvh == 0) {  // the owner checks the sequence once
+        if (slot == 0 && !iu.pre && iu.kvh == 0) {  // the first owner checks the sequence once
             if (iu.bad && lane == 0) atomicOr(p.status, iu.bad);
             if (cascade && iu.s > 0) {
                 // The declared prefix must be the same physical blocks as row 0's.
@@ -292,54 +294,70 @@ __global__ void __launch_bounds__(W * 32,
         if ((lane >> 1) < rows_of(iu) && qr >= 0) prefetch_l2(p.q + qr * D + (lane & 1) * (D / 2));
         return true;
     };
-    // The unit to help: the one with the most pages left among those probed
-    // (remaining >= two minimum claims), with a free helper slot.
+    // The unit to help: among the units probed with at least two minimum
+    // claims of pages left, the one with the most pages left per warp already
+    // on it (owner plus helpers), so that warps looking at the same time
+    // spread over the units instead of piling onto one; it must have a free
+    // helper slot.  Gives up after four probes that find nothing worth
+    // joining, or 16 tries in all.
     auto help = [&]() -> bool {
-        for (int attempt = 0; attempt < 4; ++attempt) {
+        int empty = 0;
+        for (int attempt = 0; attempt < 16; ++attempt) {
             const unsigned int h = (static_cast<unsigned int>(gw) * 2654435761u) ^ (attempt * 40503u);
-            int best_u = -1, best_left = 2 * t.step_min - 1;
+            int best_u = -1;
+            float best_score = 0.f;
             for (int k = 0; k < t.probe_rounds; ++k) {
                 const int u = static_cast<int>((h + static_cast<unsigned int>(lane + 32 * k)) %
                                                static_cast<unsigned int>(t.units));
                 const UnitRef r = unit_ref<B>(p, t, u);
-                const int used = static_cast<int>(tagged_count(
-                    *reinterpret_cast<volatile unsigned long long*>(t.uw + 2 * u), gen));
+                const volatile unsigned long long* w =
+                    reinterpret_cast<volatile unsigned long long*>(t.uw + 2 * u);
+                const int used = static_cast<int>(tagged_count(w[0], gen));
+                const int helpers = static_cast<int>(tagged_count(w[1], gen));
                 const int left = r.n - used;
-                if (left > best_left) {
-                    best_left = left;
-                    best_u = u;
+                const int k_max = u < t.units_pre ? t.k_pre : t.k_own;
+                if (left >= 2 * t.step_min && t.owners + helpers < k_max) {
+                    const float score = static_cast<float>(left) / static_cast<float>(2 + helpers);
+                    if (score > best_score) {
+                        best_score = score;
+                        best_u = u;
+                    }
                 }
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
-                const int ol = __shfl_xor_sync(kFull, best_left, o);
+                const float os = __shfl_xor_sync(kFull, best_score, o);
                 const int ou = __shfl_xor_sync(kFull, best_u, o);
-                if (ol > best_left || (ol == best_left && ou > best_u)) {
-                    best_left = ol;
+                if (os > best_score || (os == best_score && ou > best_u)) {
+                    best_score = os;
                     best_u = ou;
                 }
             }
-            if (best_u < 0) return false;  // nothing worth joining
+            if (best_u < 0) {  // nothing worth joining among these units
+                if (++empty == 4) return false;
+                continue;
+            }
             const int k_max = best_u < t.units_pre ? t.k_pre : t.k_own;
             uint32_t hs = 0;
             if (lane == 0) hs = tagged_add(t.uw + 2 * best_u + 1, gen, 1u);
             hs = __shfl_sync(kFull, hs, 0);
-            if (hs == 0xffffffffu || static_cast<int>(hs) + 1 >= k_max) continue;  // no slot
-            if (join(best_u, static_cast<int>(hs) + 1)) return true;
+            if (hs == 0xffffffffu || t.owners + static_cast<int>(hs) >= k_max) continue;  // no slot
+            if (join(best_u, t.owners + static_cast<int>(hs))) return true;
         }
         return false;
     };
-    // The next unit: from the cursor while it lasts, then one to help.
+    // The next unit: from the cursor while it lasts (entry e is owner slot
+    // e % owners of unit e / owners), then one to help.
     auto next_unit = [&]() -> bool {
         while (!cursor_done) {
-            unsigned int u = 0;
-            if (lane == 0) u = atomicAdd(t.hdr + 1, 1u);
-            u = __shfl_sync(kFull, u, 0);
-            if (u >= static_cast<unsigned int>(t.units)) {
+            unsigned int e = 0;
+            if (lane == 0) e = atomicAdd(t.hdr + 1, 1u);
+            e = __shfl_sync(kFull, e, 0);
+            if (e >= static_cast<unsigned int>(t.units) * static_cast<unsigned int>(t.owners)) {
                 cursor_done = true;
                 break;
             }
-            if (join(static_cast<int>(u), 0)) return true;
+            if (join(static_cast<int>(e / t.owners), static_cast<int>(e % t.owners))) return true;
         }
         return help();
     };

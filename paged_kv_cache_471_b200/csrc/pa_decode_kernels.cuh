@@ -1336,10 +1336,10 @@ struct CombineParams {
     int balanced, Hk, G;
     const int* br_scan;  // balanced: per-sequence page prefix [S + 1], pages per CTA
     // Dynamic schedule: every row is merged here from its units' slots --
-    // slot 0 (the unit's owner) plus one per helper, as the helper counters
-    // of the call that just ran (generation hdr[0] - 1) record them.
+    // the owners' slots plus one per helper, as the helper counters of the
+    // call that just ran (generation hdr[0] - 1) record them.
     int dynamic;
-    int dyn_units_pre, dyn_k_pre, dyn_k_own, dyn_k_total;
+    int dyn_units_pre, dyn_owners, dyn_k_pre, dyn_k_own, dyn_k_total;
     const unsigned int* dyn_hdr;
     const unsigned long long* dyn_uw;
 };
@@ -1379,7 +1379,8 @@ __global__ void __launch_bounds__(kThreads) pa_combine_kernel(const CombineParam
             const unsigned long long w = p.dyn_uw[2 * u + 1];
             const unsigned int helpers =
                 static_cast<unsigned int>(w >> 32) == gen ? static_cast<unsigned int>(w) : 0u;
-            return 1 + static_cast<int>(min(helpers, static_cast<unsigned int>(k - 1)));
+            return p.dyn_owners +
+                   static_cast<int>(min(helpers, static_cast<unsigned int>(k - p.dyn_owners)));
         };
         if (p.prefix_pages > 0)
             dyn_n_pre = slots(kvh + p.Hk * ((s * p.G + h % p.G) / 16), p.dyn_k_pre);

@@ -261,12 +261,14 @@ def test_dynamic_schedule_plan_and_workspace():
         p = pa.plan(c.num_seqs, c.num_heads, c.num_kv_heads, c.head_size, c.block_size,
                     c.max_seq_len, c.kv_dtype, num_sms=148, schedule="dynamic",
                     shared_prefix_blocks=pref)
-        assert p["dynamic"] == 1 and p["balanced"] == 0 and p["partition_pages"] == 0
+        assert p["balanced"] == 0 and p["partition_pages"] == 0
         assert p["grid_ctas"] == 148 * 3
         warps = p["grid_ctas"] * p["warps_per_cta"]
         groups = -(-(c.num_seqs * c.group) // 16) if pref else 0
         units = c.num_kv_heads * groups + c.num_seqs * c.num_kv_heads
-        k = min(64, -(-2 * warps // units) + 8)
+        owners = 4 if 2 * units >= warps else 1
+        assert p["dynamic"] == owners
+        k = min(64, owners + -(-2 * warps // units) + 8)
         assert p["num_partitions"] == k and p["prefix_partitions"] == (k if pref else 0)
         assert p["prefix_groups"] == groups
         k_total = k * (2 if pref else 1)

@@ -1,13 +1,17 @@
 """The dynamic schedule's claiming protocol, on the CPU.
 
 The decode kernel's warps claim work through counters in the workspace: a
-cursor hands each unit to one owner (partial slot 0); a unit's page counter
+cursor hands each unit to its owners (partial slots 0 .. owners - 1: four
+for a batch with at least half as many units as warps, else one); a unit's
+page counter
 hands out ranges of its pages, and each warp claims its next range while it
-issues the current one; once the cursor is spent, warps join the unit with
-the most pages left (at least two minimum claims) as helpers, taking slot
-1 + (helper counter), and only if that slot is below the unit's limit K;
+issues the current one; once the cursor is spent, warps join as helpers the
+unit with the most pages left (at least two minimum claims) per warp on it,
+taking slot owners + (helper counter), and only if that slot is below the
+unit's limit K;
 a warp that joins a unit with no pages left writes an empty partial.  The
-combine then reads slots 0 .. min(helpers, K - 1) of each unit.
+combine then reads slots 0 .. owners + min(helpers, K - owners) - 1 of each
+unit.
 
 The protocol is written out here from that description, run with warps
 interleaved at random (the order in which their atomics land), and checked:
@@ -22,11 +26,12 @@ import pytest
 
 
 class Model:
-    def __init__(self, pages, warps, k, step_min=4, step_max=32, seed=0):
+    def __init__(self, pages, warps, k, owners=1, step_min=4, step_max=32, seed=0):
         self.n = list(pages)
         self.U = len(pages)
         self.W = warps
         self.K = k
+        self.O = owners
         self.step_min, self.step_max = step_min, step_max
         self.rng = random.Random(seed)
         self.cursor = 0
@@ -42,39 +47,48 @@ class Model:
     def warp(self, w):
         """A generator: each yield is one atomic of this warp."""
         cursor_done = False
-        attempts = 0  # failed helper attempts since the last join (the kernel gives up at 4)
+        attempts = 0  # failed helper attempts since the last join (the kernel gives up at 16)
+        empty = 0     # of them, probes that found nothing (the kernel gives up at 4)
         while True:
             joined = None
             while not cursor_done:
-                u = self.cursor
+                e = self.cursor
                 self.cursor += 1
                 yield
-                if u >= self.U:
+                if e >= self.U * self.O:
                     cursor_done = True
                     break
-                joined = (u, 0)
+                joined = (e // self.O, e % self.O)
                 break
             if joined is None:
-                best, best_left = None, 2 * self.step_min - 1
+                best, best_score = None, 0.0
                 probe = list(range(self.U))
                 self.rng.shuffle(probe)
                 for u in probe[:256]:
                     left = self.n[u] - self.page_ctr[u]
-                    if left > best_left:
-                        best, best_left = u, left
+                    if left >= 2 * self.step_min and self.O + self.helpers[u] < self.K:
+                        score = left / (2 + self.helpers[u])
+                        if score > best_score:
+                            best, best_score = u, score
                 yield
                 if best is None:
-                    return
+                    empty += 1
+                    if empty == 4:
+                        return
+                    attempts += 1
+                    if attempts == 16:
+                        return
+                    continue
                 hs = self.helpers[best]
                 self.helpers[best] += 1
                 yield
-                if hs + 1 >= self.K:
+                if self.O + hs >= self.K:
                     attempts += 1
-                    if attempts == 4:
+                    if attempts == 16:
                         return
                     continue  # no slot: probe again
-                joined = (best, hs + 1)
-            attempts = 0
+                joined = (best, self.O + hs)
+            attempts = empty = 0
             u, slot = joined
             assert (u, slot) not in self.slots
             mine = []
@@ -113,6 +127,7 @@ CASES = [
     ("ragged, empty units", [0, 5, 130, 4096, 1, 0, 77, 900, 33], 48, None),
     ("more units than warps", [64] * 100, 16, None),
     ("slot limit binds", [2000] * 3, 64, 4),
+    ("four owners per unit", [256] * 30 + [70] * 10, 48, None),
 ]
 
 
@@ -120,16 +135,17 @@ CASES = [
 @pytest.mark.parametrize("seed", range(5))
 def test_every_page_once_and_every_read_slot_written(name, pages, warps, k, seed):
     units = len(pages)
+    owners = 4 if 2 * units >= warps else 1
     if k is None:
-        k = min(64, -(-2 * warps // units) + 8)
-    m = Model(pages, warps, k, seed=seed)
+        k = min(64, owners + -(-2 * warps // units) + 8)
+    m = Model(pages, warps, k, owners=owners, seed=seed)
     m.run()
     # every page of every unit read exactly once
     want = {(u, j) for u, n in enumerate(pages) for j in range(n)}
     assert set(m.read) == want
     # the combine's slots of each unit are exactly the written ones
     for u in range(units):
-        count = 1 + min(m.helpers[u], k - 1)
+        count = owners + min(m.helpers[u], k - owners)
         written = {s for (uu, s) in m.slots if uu == u}
         assert written == set(range(count)), (u, written, count)
     # pages of a slot belong to that slot's unit and warp
