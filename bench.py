@@ -60,14 +60,20 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# The device code of the default decode path: pa_decode_kernel, pa_combine_kernel
+# and the page body they share.  (The dynamic schedule's kernel lives in its own
+# header and does not change what these kernels read or write.)
+KERNEL_SOURCES = ("pa_decode_kernels.cuh", "pa_ptx.cuh")
+
+
 def kernel_source_hash() -> str:
-    """Hash of the device code: the .cuh kernel headers with comments and
-    whitespace removed (host-side ABI code does not change what the kernels
-    read or write, and neither do comments)."""
+    """Hash of the default path's device code: its kernel headers with
+    comments and whitespace removed (host-side ABI code does not change what
+    the kernels read or write, and neither do comments)."""
     import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_471_b200", "csrc")
-    for name in sorted(n for n in os.listdir(csrc) if n.endswith(".cuh")):
+    for name in KERNEL_SOURCES:
         with open(os.path.join(csrc, name), encoding="utf-8") as f:
             text = f.read()
         text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
