@@ -382,10 +382,11 @@ __global__ void __launch_bounds__(W * 32,
             }
         }
         const int i = ri++;
-        // With the second stage of a range (the first, for a one-stage range)
-        // the next range's claim has returned: read its block ids now, so
-        // they are in registers when this range runs out.
-        if (n_claimed && !n_loaded && (i == 1 || rn == 1)) {
+        // Halfway through a range the next range's claim (an atomic issued
+        // when this range started) has long returned: read it and load its
+        // block ids now, so they are in registers when this range runs out.
+        // (Reading it sooner would stall the warp on the atomic's latency.)
+        if (n_claimed && !n_loaded && i == rn / 2) {
             nv_b = __shfl_sync(kFull, nv, 0);
             if (nv_b < iu.n) load_window(nv_b, nstep, win_n, win_n2);
             n_loaded = true;
