@@ -220,7 +220,7 @@ def workload_config(idx: int, num_seqs: int = 0):
 def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, num_seqs=0,
              cascade=True, alibi=False, schedule="auto", min_region_ms=0.0,
              min_clock_samples=12, extras=True, mha_cuda_cores=False, fp8_compute=False,
-             partition_pages=0):
+             partition_pages=0, stages=0):
     import torch
 
     import paged_kv_cache_471_b200 as pa
@@ -241,7 +241,7 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
     fp8_compute = fp8_compute and cfg.kv_dtype == W.FP8_E4M3
     plan = pa.plan(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_size, cfg.block_size,
                    cfg.max_seq_len, cfg.kv_dtype, shared_prefix_blocks=prefix, schedule=schedule,
-                   fp8_compute=fp8_compute, partition_pages=partition_pages)
+                   fp8_compute=fp8_compute, partition_pages=partition_pages, stages=stages)
     ws = torch.zeros(plan["workspace_bytes"], dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
     alg_bytes = bytes_of(wl)
@@ -255,7 +255,7 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
                   wl.k_scale, wl.v_scale, workspace_tensor=ws, stream=stream,
                   shared_prefix_blocks=prefix, alibi_slopes=slopes, schedule=schedule,
                   mha_cuda_cores=mha_cuda_cores, fp8_compute=fp8_compute,
-                  partition_pages=partition_pages)
+                  partition_pages=partition_pages, stages=stages)
 
     for _ in range(max(warmup, 3)):
         if flush:
@@ -354,7 +354,7 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
                                            cfg.kv_dtype, wl.k_scale, wl.v_scale,
                                            workspace_tensor=ws, stream=st, schedule=schedule,
                                            mha_cuda_cores=mha_cuda_cores, fp8_compute=fp8_compute,
-                  partition_pages=partition_pages)
+                  partition_pages=partition_pages, stages=stages)
             step_on(gs)  # warm on the capture stream
             gs.synchronize()
             with torch.cuda.graph(graph, stream=gs):
@@ -384,7 +384,8 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
                                       or plan["balanced"] == 1 or plan["dynamic"] > 0),
                shared_prefix_blocks=prefix, alibi=alibi, extra=extra,
                options={"schedule": schedule, "mha_cuda_cores": bool(mha_cuda_cores),
-                        "fp8_compute": bool(fp8_compute), "partition_pages": partition_pages})
+                        "fp8_compute": bool(fp8_compute), "partition_pages": partition_pages,
+                        "stages": stages})
 
     if want_e2e:
         # End to end through the public call, as a serving loop runs it: every
@@ -426,7 +427,7 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
                           cfg.kv_dtype, wl.k_scale, wl.v_scale, workspace_tensor=ws,
                           stream=stream, shared_prefix_blocks=prefix, alibi_slopes=slopes,
                           schedule=schedule, mha_cuda_cores=mha_cuda_cores, fp8_compute=fp8_compute,
-                  partition_pages=partition_pages)
+                  partition_pages=partition_pages, stages=stages)
                 ev_used[b].record(stream)
                 with torch.cuda.stream(down):
                     down.wait_event(ev_used[b])
@@ -728,6 +729,8 @@ def main(argv=None):
     ap.add_argument("--schedule", default="auto",
                     choices=["auto", "balanced", "partitioned", "dynamic"],
                     help="how CTAs share the work (pa_options.schedule)")
+    ap.add_argument("--stages", type=int, default=0,
+                    help="force this many page buffers per warp (pa_options.stages)")
     ap.add_argument("--partition-pages", type=int, default=0,
                     help="force split-KV partitions of this many blocks (pa_options.partition_pages)")
     ap.add_argument("--fp8-compute", action="store_true",
@@ -769,7 +772,8 @@ def main(argv=None):
         r = time_gpu(idx, args.steps, args.warmup, device, want_e2e=not args.no_e2e, rank=rank,
                      num_seqs=args.num_seqs, cascade=not args.no_cascade, alibi=args.alibi,
                      schedule=args.schedule, mha_cuda_cores=args.mha_cuda_cores,
-                     fp8_compute=args.fp8_compute, partition_pages=args.partition_pages)
+                     fp8_compute=args.fp8_compute, partition_pages=args.partition_pages,
+                     stages=args.stages)
         r["step_ms"] = reduce_max(r["step_ms"], device)
         if "e2e_ms" in r:
             r["e2e_ms"] = reduce_max(r["e2e_ms"], device)
@@ -783,7 +787,7 @@ def main(argv=None):
         # workload's figures (each its own timed region of >= 0.3 s).
         if (ws == 1 and len(cfg_ids) == 1 and not args.no_per_config and not args.num_seqs
                 and not args.alibi and args.schedule == "auto" and not args.mha_cuda_cores
-                and not args.fp8_compute and not args.partition_pages):
+                and not args.fp8_compute and not args.partition_pages and not args.stages):
             per = {}
             for j in (1, 2, 3, 4, 5):
                 rj = time_gpu(j, args.steps, args.warmup, device, want_e2e=False,
