@@ -1344,6 +1344,101 @@ struct CombineParams {
     const unsigned long long* dyn_uw;
 };
 
+// The merge of one row of the partitioned schedule whose slots fit in a
+// warp (at most 32): every load it needs -- the sequence length, each slot's
+// (max, sum), one slot per lane, and the partial rows of the first 16 slots,
+// D / 32 consecutive head dims per lane -- is issued before any of them is
+// used, so a row costs one memory round trip (a second one for slots
+// 16..31).  Slots past the row's count (and an empty slot's row) may hold
+// anything; their weight is 0 and a select drops them.
+template <int D>
+__device__ __forceinline__ void combine_row_fast(const CombineParams& p, long long row, int s,
+                                                 int lane) {
+    constexpr int V = D / 32;  // head dims per lane: 4 * lane .. (D = 128) or 2 * lane ..
+    constexpr int KO = 16;     // partial rows loaded up front
+    const int np = p.P_total;
+    const long long base = row * np;
+    const int T0 = __ldg(p.seq_lens + s);
+    float l = 0.f, m = -INFINITY;
+    if (lane < np) {
+        l = p.ws_l[base + lane];
+        m = p.ws_m[base + lane];
+    }
+    auto load_row = [&](int i, float (&v)[V]) {
+        const float* src = p.ws_o + (base + i) * D + V * lane;
+        if constexpr (V == 4) {
+            const float4 x = *reinterpret_cast<const float4*>(src);
+            v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+        } else {
+            const float2 x = *reinterpret_cast<const float2*>(src);
+            v[0] = x.x; v[1] = x.y;
+        }
+    };
+    float o[KO][V];
+#pragma unroll
+    for (int i = 0; i < KO; ++i) {
+        if (i < np) {
+            load_row(i, o[i]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < V; ++j) o[i][j] = 0.f;
+        }
+    }
+    // The row's slots: the prefix partitions, then the sequence's own.
+    const int T = max(0, min(T0, p.max_blocks * p.B));
+    const int nb = (T + p.B - 1) / p.B;
+    int nps;
+    if (p.prefix_pages > 0) {
+        const int own = nb > p.prefix_pages ? (nb - p.prefix_pages + p.PP - 1) / p.PP : 0;
+        nps = p.prefix_parts + min(p.P, own);
+    } else {
+        nps = min(p.P, (nb + p.PP - 1) / p.PP);
+        if (nps <= 1) return;  // one partition: the decode kernel wrote the row
+    }
+    const bool live = lane < nps && l > 0.f;
+    float M = live ? m : -INFINITY;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
+    const float wt = live ? exp2f(m - M) * l : 0.f;
+    float L = wt;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(kFull, L, off);
+    float a[V];
+#pragma unroll
+    for (int j = 0; j < V; ++j) a[j] = 0.f;
+#pragma unroll
+    for (int i = 0; i < KO; ++i) {
+        const float w = __shfl_sync(kFull, wt, i);
+#pragma unroll
+        for (int j = 0; j < V; ++j) a[j] += w > 0.f ? w * o[i][j] : 0.f;
+    }
+    for (int i0 = KO; i0 < nps; i0 += 8) {
+        float q[8][V];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (i0 + i < nps) {
+                load_row(i0 + i, q[i]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < V; ++j) q[i][j] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float w = __shfl_sync(kFull, wt, (i0 + i) & 31);
+#pragma unroll
+            for (int j = 0; j < V; ++j) a[j] += (i0 + i < nps && w > 0.f) ? w * q[i][j] : 0.f;
+        }
+    }
+    __nv_bfloat16* dst = p.out + row * D + V * lane;
+#pragma unroll
+    for (int j = 0; j < V; j += 2) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(L > 0.f ? a[j] / L : 0.f,
+                                                       L > 0.f ? a[j + 1] / L : 0.f);
+        *reinterpret_cast<__nv_bfloat162*>(dst + j) = h;
+    }
+}
+
 // Log-sum-exp merge of the split-KV partials of one (sequence, q head) per
 // warp:  M = max_p m_p;  w_p = l_p 2^(m_p - M);  out = sum_p w_p o_p / sum_p w_p.
 // Without a shared prefix, rows whose sequence fits in one partition were
@@ -1366,6 +1461,10 @@ __global__ void __launch_bounds__(kThreads) pa_combine_kernel(const CombineParam
     const long long row = (long long)blockIdx.x * kWarps + warp;
     if (row >= (long long)p.S * p.Hq) return;
     const int s = static_cast<int>(row / p.Hq);
+    if (!p.dynamic && !p.balanced && p.P_total <= 32) {
+        combine_row_fast<D>(p, row, s, lane);
+        return;
+    }
     int nps;
     long long base = row * p.P_total;  // slot i is partial row base + i ...
     long long br_c0 = 0, br_off = 0, br_per = 1;
