@@ -152,8 +152,6 @@ __global__ void __launch_bounds__(W * 32,
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int gq = lane >> 2;
-    const int cq = lane & 3;
     const int gw = blockIdx.x * W + warp;  // this warp's number in the grid
 
     // Shared memory: per-warp page stages, then the mbarriers, then each

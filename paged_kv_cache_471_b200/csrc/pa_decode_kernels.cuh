@@ -892,7 +892,6 @@ __global__ void __launch_bounds__(W * 32,
     static_assert(!SC || (!FP8 && NH == 1), "the CUDA-core form takes bf16 pages and one head");
     using WA = std::conditional_t<SC, WarpAttnScalar<D, B>, WarpAttn<D, B, FP8, NH, F8MMA>>;
     constexpr int ELEM = FP8 ? 1 : 2;
-    constexpr int K32 = D / 32;  // 32-wide k-steps over the head dim (e4m3 MMA)
     constexpr int PAGE = D * B * ELEM;  // one K (or V) page of one kv head
     // Small pages go in pairs (pair_pages): a stage holds two
     // consecutive logical blocks of the unit (K a, K b, V a, V b), so a warp
@@ -900,13 +899,7 @@ __global__ void __launch_bounds__(W * 32,
     // the page code covers 32 tokens.
     constexpr bool PAIR = pair_pages<D, B, FP8, F8MMA>();
     constexpr int NPG = PAIR ? 2 : 1;  // logical pages per stage
-    constexpr int BT = B * NPG;        // tokens per stage
     constexpr int STAGE = 2 * PAGE * NPG;
-    constexpr int NT = BT / 8;  // 8-token n-tiles per stage (QK)
-    constexpr int KT = D / 16;  // 16-wide k-tiles over the head dim (QK)
-    constexpr int MT = D / 16;  // 16-row m-tiles over the head dim (PV)
-    constexpr int KK = BT / 16; // 16-token k-tiles per stage (PV)
-    constexpr int CHUNK = B * 16;  // bytes of one 16-byte column group of a K page
     constexpr int RS = D + 4;      // padded row stride of the merge buffer
 
     extern __shared__ __align__(128) uint8_t smem[];
@@ -920,8 +913,6 @@ __global__ void __launch_bounds__(W * 32,
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int gq = lane >> 2;  // fragment row group
-    const int cq = lane & 3;   // thread in quad
 
     // ---------------- this CTA's work: one unit, or a balanced page range
     bool pre = false;  // a shared-prefix unit
