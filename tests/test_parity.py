@@ -43,6 +43,36 @@ def test_reduced_workloads(idx, partition_pages):
     assert pa.read_status(device=DEV) == 0
 
 
+# Partition sizes that put a row's slot count (prefix partitions plus the
+# sequence's own) in each regime of the combine: at most 16 (one batch of
+# partial rows), 17..32 (a second batch), exactly 32, and more than 32 (the
+# slots read 32 at a time).
+SLOT_REGIMES = {
+    3: [(9, "<=16"), (5, "17..32"), (4, ">32")],
+    5: [(64, "<=16"), (8, "17..32"), (5, "32"), (4, ">32")],
+}
+
+
+@pytest.mark.parametrize("idx", sorted(SLOT_REGIMES))
+def test_combine_slot_count_regimes(idx):
+    cfg = REDUCED[idx]
+    wl = W.make_workload(cfg, DEV)
+    ref = run_oracle(wl)
+    for pp, regime in SLOT_REGIMES[idx]:
+        plan = pa.plan(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_size,
+                       cfg.block_size, cfg.max_seq_len, cfg.kv_dtype,
+                       shared_prefix_blocks=cfg.shared_prefix_blocks, partition_pages=pp)
+        slots = plan["num_partitions"] + plan["prefix_partitions"]
+        ok = {"<=16": slots <= 16, "17..32": 16 < slots < 32, "32": slots == 32,
+              ">32": slots > 32}[regime]
+        assert ok, (pp, regime, slots)
+        out = torch.full_like(wl.query, float("nan"))
+        run_gpu(wl, out=out, partition_pages=pp, shared_prefix_blocks=cfg.shared_prefix_blocks)
+        torch.cuda.synchronize()
+        compare(out, ref, cfg.kv_dtype, f"cfg{idx} pp={pp} ({slots} slots)")
+        assert pa.read_status(device=DEV) == 0
+
+
 @pytest.mark.parametrize("idx", [1, 3, 4, 5])
 def test_pa_decode_symbol_through_ctypes(idx):
     """The boundary call itself, pa_decode (no options), called through
