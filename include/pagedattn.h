@@ -84,6 +84,10 @@ typedef enum pa_kv_dtype {
 
 /* Bytes at the start of the workspace reserved for the status word. */
 #define PA_WORKSPACE_HEADER_BYTES 256
+/* After the header, in any workspace larger than the header: the split
+ * tail's per-unit CTA counts (at most 512 units), zero between calls; every
+ * plan's partials start after them. */
+#define PA_WORKSPACE_TAIL_COUNTER_BYTES 2048
 
 /*
  * Tuning knobs; pass NULL for the planner's defaults.
@@ -126,7 +130,11 @@ typedef enum pa_kv_dtype {
  *  schedule: how CTAs share the work.  PA_SCHEDULE_AUTO (0) and
  *      PA_SCHEDULE_PARTITIONED: one CTA per (sequence, kv head, partition), as
  *      many waves as that takes; the hardware hands units to SMs as they free
- *      up.  PA_SCHEDULE_BALANCED: one wave of CTAs (grid_ctas = resident CTA
+ *      up.  Under PA_SCHEDULE_AUTO, when units are not split and fill two or
+ *      three waves of CTA slots, the units of the last, partial wave are cut
+ *      into partitions whose CTAs follow every whole unit's (the split tail,
+ *      pa_plan.tail_units); PA_SCHEDULE_PARTITIONED leaves them whole.
+ *      PA_SCHEDULE_BALANCED: one wave of CTAs (grid_ctas = resident CTA
  *      slots), each taking an equal contiguous share of all (sequence, kv
  *      head, page) work; units cut at a share's ends are merged by the
  *      combine kernel, which then runs on every call.  That removes the last
@@ -182,6 +190,12 @@ typedef struct pa_plan {
                                the partial slots per query row of a (sequence, kv head)
                                unit and of a prefix unit, partition_pages is 0,
                                grid_ctas an upper bound; 0: another schedule            */
+    long long tail_units;     /* split tail: units of the last, partial wave of whole
+                                 units, each cut into tail_partitions partitions of
+                                 tail_partition_pages blocks whose CTAs follow every
+                                 whole unit's (PA_SCHEDULE_AUTO only); 0: none          */
+    int tail_partitions;
+    int tail_partition_pages;
 } pa_plan;
 
 /*
@@ -195,9 +209,12 @@ pa_status pa_plan_decode(pa_plan* plan, int num_seqs, int num_heads, int num_kv_
 /*
  * Workspace bytes pa_decode needs (>= PA_WORKSPACE_HEADER_BYTES), or 0 when the
  * sizes are invalid.  Layout: a 256-byte header whose first uint32 is the
- * status word, then (when P > 1 or a shared prefix is declared) per (seq,
- * query head, partition) an fp32 partial output [head_size], and fp32 running
- * max (log2 domain) and sum.  Under PA_SCHEDULE_BALANCED, after the header:
+ * status word; when the plan needs more, PA_WORKSPACE_TAIL_COUNTER_BYTES of
+ * split-tail counts, then (when P > 1 or a shared prefix is declared) per
+ * (seq, query head, partition) an fp32 partial output [head_size], and fp32
+ * running max (log2 domain) and sum -- or, with a split tail
+ * (pa_plan.tail_units > 0), the same per (tail unit, query head of its
+ * group, tail partition).  Under PA_SCHEDULE_BALANCED, after the counts:
  * the per-sequence page prefix and the pages per CTA (num_seqs + 2 ints,
  * padded to 256 bytes), then two slots of G query rows per CTA, each an fp32
  * partial [head_size] with its max and sum.  The sizes depend on the options

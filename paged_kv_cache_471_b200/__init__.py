@@ -35,6 +35,7 @@ PA_DEV_WAIT_TIMEOUT = 0x4
 PA_DEV_PREFIX_MISMATCH = 0x8
 
 WORKSPACE_HEADER_BYTES = 256
+WORKSPACE_TAIL_COUNTER_BYTES = 2048  # after the header when the plan needs more
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 _KV = {"bf16": PA_KV_BF16, "auto": PA_KV_BF16, "fp8": PA_KV_FP8_E4M3, "fp8_e4m3": PA_KV_FP8_E4M3,
@@ -61,7 +62,8 @@ class Plan(ctypes.Structure):
                 ("grid_ctas", ctypes.c_longlong), ("smem_bytes", ctypes.c_size_t),
                 ("workspace_bytes", ctypes.c_size_t), ("prefix_partitions", ctypes.c_int),
                 ("prefix_groups", ctypes.c_int), ("balanced", ctypes.c_int),
-                ("dynamic", ctypes.c_int)]
+                ("dynamic", ctypes.c_int), ("tail_units", ctypes.c_longlong),
+                ("tail_partitions", ctypes.c_int), ("tail_partition_pages", ctypes.c_int)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}
@@ -229,7 +231,7 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
            v_scale=None, workspace_tensor=None, partition_pages: int = 0, stream=None,
            stages: int = 0, shared_prefix_blocks: int = 0, alibi_slopes=None,
            fp8_compute: bool = False, test_stall_copies: bool = False, schedule: str = "auto",
-           mha_cuda_cores: bool = False):
+           mha_cuda_cores: bool = False, num_sms: int = 0):
     """Paged decode attention into ``out`` (bf16 [num_seqs, num_heads, head_size]).
 
     key_cache: [num_blocks, num_kv_heads, head_size/x, block_size, x];
@@ -240,8 +242,10 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
     The keyword options are those of pa_options in include/pagedattn.h:
     partition_pages, stages, shared_prefix_blocks, alibi_slopes ([num_heads]
     fp32), fp8_compute, test_stall_copies, schedule ("auto",
-    "partitioned", "balanced" or "dynamic") and mha_cuda_cores.  workspace_tensor defaults to a cached
-    zeroed buffer per device; stream defaults to the current stream.
+    "partitioned", "balanced" or "dynamic"), mha_cuda_cores and num_sms (plan
+    as if the GPU had that many SMs; 0 = the device's count).  workspace_tensor
+    defaults to a cached zeroed buffer per device; stream defaults to the
+    current stream.
     """
     import torch
     code = kv_dtype_code(kv_dtype)
@@ -285,7 +289,7 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
             need = workspace_size(S, Hq, num_kv_heads, D, block_size, max_seq_len, code,
                                   partition_pages, shared_prefix_blocks=shared_prefix_blocks,
                                   fp8_compute=fp8_compute and code == PA_KV_FP8_E4M3,
-                                  schedule=schedule, stages=stages)
+                                  schedule=schedule, stages=stages, num_sms=num_sms)
             workspace_tensor = workspace(need, dev)
         ws = _ptr(workspace_tensor, "workspace", None, dev)
         rc = lib().pa_decode_ex(*args_ptrs, S, Hq, int(num_kv_heads), D, float(scale), bt,
@@ -293,7 +297,7 @@ def decode(out, query, key_cache, value_cache, num_kv_heads: int, scale: float, 
                                 int(num_blocks), code, ks, vs, ws,
                                 workspace_tensor.numel() * workspace_tensor.element_size(),
                                 st.cuda_stream,
-                                _opts(partition_pages, 0, stages, shared_prefix_blocks, alibi,
+                                _opts(partition_pages, num_sms, stages, shared_prefix_blocks, alibi,
                                       fp8_compute, test_stall_copies, schedule, mha_cuda_cores))
     _check(rc)
     return out

@@ -98,6 +98,16 @@ struct DecodeParams {
     // pages per CTA in br_scan[0 .. S + 1] for the combine.
     int balanced;
     int* br_scan;
+    // Split tail (the partitioned schedule where units are not split): the
+    // first n_full per-sequence units run whole; each remaining unit is cut
+    // into tail_P partitions of tail_PP pages, whose CTAs come after every
+    // whole unit's.  Tail unit t = unit - n_full writes its partials at rows
+    // (t * G + g) * tail_P + part of ws_o / ws_m / ws_l and counts its CTAs
+    // in tail_cnt[t]; the last of them merges the unit's rows into out and
+    // sets the count back to 0 (counts are 0 between calls).
+    long long n_full;
+    int tail_P, tail_PP;
+    unsigned int* tail_cnt;
 };
 
 // Bytes of shared memory the final merge needs (it overlays the page stages).
@@ -917,6 +927,7 @@ __global__ void __launch_bounds__(W * 32,
     // ---------------- this CTA's work: one unit, or a balanced page range
     bool pre = false;  // a shared-prefix unit
     int kvh = 0, s = 0, part = 0, rg = 0;
+    long long tail_t = -1;  // unit of the split tail, or -1
     long long bx = 0, bx_first = 0, bx_end = 0;  // balanced: pages [bx, bx_end) still to do
     int bj = 0, bn = 0;                          // balanced: page in the unit, pages of the unit
     const int t_cap = p.max_blocks * B;
@@ -1000,10 +1011,20 @@ __global__ void __launch_bounds__(W * 32,
             part = static_cast<int>(unit / ((long long)p.Hk * p.prefix_groups));
             s = 0;
         } else {
-            const long long u = unit - p.prefix_units;
+            long long u = unit - p.prefix_units;
+            if (p.tail_P > 0 && u >= p.n_full) {
+                // A partition of a split-tail unit (all of them follow the
+                // whole units, partition-major).
+                const long long n_tail = static_cast<long long>(p.Hk) * p.S - p.n_full;
+                const long long t = u - p.n_full;
+                tail_t = t % n_tail;
+                part = static_cast<int>(t / n_tail);
+                u = p.n_full + tail_t;
+            } else {
+                part = static_cast<int>(u / ((long long)p.Hk * p.S));
+            }
             kvh = static_cast<int>(u % p.Hk);
             s = static_cast<int>((u / p.Hk) % p.S);
-            part = static_cast<int>(u / ((long long)p.Hk * p.S));
             if (p.longest_first) {
                 // The unit's sequence index is a rank: find the sequence with
                 // that rank among all lengths, longest first, so that the
@@ -1059,7 +1080,9 @@ __global__ void __launch_bounds__(W * 32,
     for (;;) {  // one segment per pass (a single pass unless balanced)
         const bool cascade = p.prefix_pages > 0;
         const int pg0 = pre ? 0 : p.prefix_pages;  // first page of this unit's page range
-        const int j0 = p.balanced ? bj : pg0 + part * p.PP;
+        const int PPu = tail_t >= 0 ? p.tail_PP : p.PP;  // the unit's partition size and count
+        const int Pu = tail_t >= 0 ? p.tail_P : p.P;
+        const int j0 = p.balanced ? bj : pg0 + part * PPu;
         const long long row0 = (long long)s * p.Hq + (long long)kvh * p.G;  // first q head row
         const int rows_total = p.S * p.G;  // query rows of one kv head (prefix units)
 
@@ -1079,7 +1102,7 @@ __global__ void __launch_bounds__(W * 32,
         // Block-table window: lane l holds the id of this warp's page (wbase + l).
         const int32_t* btrow = p.bt + (long long)s * p.max_blocks;
         const int jcap = p.balanced ? min(bn, p.max_blocks)
-                                    : min(j0 + p.PP, pre ? p.prefix_pages : p.max_blocks);
+                                    : min(j0 + PPu, pre ? p.prefix_pages : p.max_blocks);
         // (A stage's first page; with pairs, `off` = 1 reads its second.)
         auto load_win = [&](int base, int off) -> int {
             const int j = j0 + NPG * (warp + W * (base + lane)) + off;
@@ -1111,7 +1134,7 @@ __global__ void __launch_bounds__(W * 32,
             if (T < 0) { T = 0; bad = kDevSeqLen; }
             if (T > t_cap) { T = t_cap; bad = kDevSeqLen; }
             nb = (T + B - 1) / B;
-            const int covered = p.balanced ? nb : pg0 + p.P * p.PP;
+            const int covered = p.balanced ? nb : pg0 + Pu * PPu;
             if (nb > covered) { nb = covered; T = nb * B; bad = kDevSeqLen; }
             if (cascade && T < p.prefix_pages * B) bad |= kDevPrefix;
             if (bad && part == 0 && kvh == 0 && j0 == pg0 && threadIdx.x == 0)
@@ -1128,15 +1151,54 @@ __global__ void __launch_bounds__(W * 32,
         // Balanced: the segment ends with the unit or with the CTA's range.
         const int j1 = p.balanced
                            ? static_cast<int>(min(static_cast<long long>(nb), j0 + (bx_end - bx)))
-                           : min(nb, j0 + p.PP);
+                           : min(nb, j0 + PPu);
         const bool direct = !cascade && (p.balanced ? (j0 == 0 && j1 == nb)
-                                                    : ((p.P == 1) || (nb <= p.PP)));
+                                                    : ((Pu == 1) || (nb <= PPu)));
+
+        // Split tail: once this CTA's partial rows are stored (or it had no
+        // pages), count it in; the unit's last CTA merges the partials of its
+        // partitions that have pages (log-sum-exp, as pa_combine_kernel does)
+        // into out, unless one partition held the whole sequence and wrote out
+        // itself, and leaves the count at 0 for the next call.
+        auto tail_arrive = [&]() {
+            __threadfence();  // this thread's partial stores before the count
+            __syncthreads();
+            int last = 0;
+            if (threadIdx.x == 0)
+                last = atomicAdd(p.tail_cnt + tail_t, 1u) == static_cast<unsigned>(p.tail_P - 1);
+            if (!__syncthreads_or(last)) return;
+            __threadfence();
+            const int nps = min(p.tail_P, (nb + p.tail_PP - 1) / p.tail_PP);
+            if (nps > 1) {
+                const long long base = tail_t * p.G * p.tail_P;
+                for (int idx = threadIdx.x; idx < p.G * D; idx += (W * 32)) {
+                    const int g = idx / D;
+                    const int d = idx - g * D;
+                    const long long r0 = base + static_cast<long long>(g) * p.tail_P;
+                    float M = -INFINITY;
+                    for (int i = 0; i < nps; ++i)
+                        if (__ldcg(p.ws_l + r0 + i) > 0.f) M = fmaxf(M, __ldcg(p.ws_m + r0 + i));
+                    float L = 0.f, O = 0.f;
+                    for (int i = 0; i < nps; ++i) {
+                        const float l = __ldcg(p.ws_l + r0 + i);
+                        if (l > 0.f) {
+                            const float w = exp2f(__ldcg(p.ws_m + r0 + i) - M) * l;
+                            L += w;
+                            O += w * __ldcg(p.ws_o + (r0 + i) * D + d);
+                        }
+                    }
+                    p.out[(row0 + g) * D + d] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
+                }
+            }
+            if (threadIdx.x == 0) p.tail_cnt[tail_t] = 0u;
+        };
 
         if (j0 >= j1) {
             if (!cascade && part == 0) {  // empty sequence: defined as a zero output row
                 for (int i = threadIdx.x; i < p.G * D; i += (W * 32))
                     p.out[row0 * D + i] = __float2bfloat16_rn(0.f);
             }
+            if (tail_t >= 0) tail_arrive();
             return;
         }
 
@@ -1289,7 +1351,9 @@ __global__ void __launch_bounds__(W * 32,
             if (direct) {
                 p.out[row * D + d] = __float2bfloat16_rn(o);
             } else {
-                const long long prow = p.balanced ? br_row0 + h : row * p.P_total + slot;
+                const long long prow = p.balanced     ? br_row0 + h
+                                       : tail_t >= 0 ? (tail_t * p.G + h) * p.tail_P + part
+                                                     : row * p.P_total + slot;
                 p.ws_o[prow * D + d] = o;
                 if (d == 0) {
                     p.ws_m[prow] = M;
@@ -1297,6 +1361,7 @@ __global__ void __launch_bounds__(W * 32,
                 }
             }
         }
+        if (tail_t >= 0) tail_arrive();
 
         // ---------------- next segment (balanced ranges only)
         if (!p.balanced) break;
@@ -1335,21 +1400,26 @@ struct CombineParams {
     const unsigned long long* dyn_uw;
 };
 
-// The merge of one row of the partitioned schedule whose slots fit in a
-// warp (at most 32): every load it needs -- the sequence length, each slot's
-// (max, sum), one slot per lane, and the partial rows of the first 16 slots,
-// D / 32 consecutive head dims per lane -- is issued before any of them is
-// used, so a row costs one memory round trip (a second one for slots
-// 16..31).  Slots past the row's count (and an empty slot's row) may hold
-// anything; their weight is 0 and a select drops them.
-template <int D>
-__device__ __forceinline__ void combine_row_fast(const CombineParams& p, long long row, int s,
-                                                 int lane) {
+// What a row's merge needs once its slots' loads are in flight: how many
+// slots it has (< 0: nothing to do, the decode kernel wrote the row) and
+// which row of out it writes.
+struct SlotRow {
+    int nps;
+    long long out_row;
+};
+
+// The merge of one row whose slots fit in a warp (at most 32), at partial
+// rows base .. base + np - 1: every load it needs -- each slot's (max, sum),
+// one slot per lane, the partial rows of the first 16 slots (D / 32
+// consecutive head dims per lane), and whatever row_info reads -- is issued
+// before any of them is used, so a row costs one memory round trip (a second
+// one for slots 16..31).  Slots past the row's count (and an empty slot's
+// row) may hold anything; their weight is 0 and a select drops them.
+template <int D, class RowInfo>
+__device__ __forceinline__ void merge_slots(const CombineParams& p, long long base, int np,
+                                            int lane, RowInfo row_info) {
     constexpr int V = D / 32;  // head dims per lane: 4 * lane .. (D = 128) or 2 * lane ..
     constexpr int KO = 16;     // partial rows loaded up front
-    const int np = p.P_total;
-    const long long base = row * np;
-    const int T0 = __ldg(p.seq_lens + s);
     float l = 0.f, m = -INFINITY;
     if (lane < np) {
         l = p.ws_l[base + lane];
@@ -1375,17 +1445,9 @@ __device__ __forceinline__ void combine_row_fast(const CombineParams& p, long lo
             for (int j = 0; j < V; ++j) o[i][j] = 0.f;
         }
     }
-    // The row's slots: the prefix partitions, then the sequence's own.
-    const int T = max(0, min(T0, p.max_blocks * p.B));
-    const int nb = (T + p.B - 1) / p.B;
-    int nps;
-    if (p.prefix_pages > 0) {
-        const int own = nb > p.prefix_pages ? (nb - p.prefix_pages + p.PP - 1) / p.PP : 0;
-        nps = p.prefix_parts + min(p.P, own);
-    } else {
-        nps = min(p.P, (nb + p.PP - 1) / p.PP);
-        if (nps <= 1) return;  // one partition: the decode kernel wrote the row
-    }
+    const SlotRow r = row_info();
+    if (r.nps < 0) return;
+    const int nps = r.nps;
     const bool live = lane < nps && l > 0.f;
     float M = live ? m : -INFINITY;
 #pragma unroll
@@ -1421,7 +1483,7 @@ __device__ __forceinline__ void combine_row_fast(const CombineParams& p, long lo
             for (int j = 0; j < V; ++j) a[j] += (i0 + i < nps && w > 0.f) ? w * q[i][j] : 0.f;
         }
     }
-    __nv_bfloat16* dst = p.out + row * D + V * lane;
+    __nv_bfloat16* dst = p.out + r.out_row * D + V * lane;
 #pragma unroll
     for (int j = 0; j < V; j += 2) {
         const __nv_bfloat162 h = __floats2bfloat162_rn(L > 0.f ? a[j] / L : 0.f,
@@ -1449,11 +1511,26 @@ __global__ void __launch_bounds__(kThreads) pa_combine_kernel(const CombineParam
     grid_dep_wait();  // the decode grid's partials are complete and visible
     grid_dep_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    auto slots_of = [&](int seq, int parts, int pages) {  // non-empty partitions
+        const int T = max(0, min(p.seq_lens[seq], p.max_blocks * p.B));
+        const int nb = (T + p.B - 1) / p.B;
+        return min(parts, (nb + pages - 1) / pages);
+    };
     const long long row = (long long)blockIdx.x * kWarps + warp;
     if (row >= (long long)p.S * p.Hq) return;
     const int s = static_cast<int>(row / p.Hq);
     if (!p.dynamic && !p.balanced && p.P_total <= 32) {
-        combine_row_fast<D>(p, row, s, lane);
+        // The row's slots: the prefix partitions, then the sequence's own.
+        merge_slots<D>(p, row * p.P_total, p.P_total, lane, [&]() -> SlotRow {
+            if (p.prefix_pages > 0) {
+                const int T = max(0, min(p.seq_lens[s], p.max_blocks * p.B));
+                const int nb = (T + p.B - 1) / p.B;
+                const int own = nb > p.prefix_pages ? (nb - p.prefix_pages + p.PP - 1) / p.PP : 0;
+                return {p.prefix_parts + min(p.P, own), row};
+            }
+            const int n = slots_of(s, p.P, p.PP);
+            return {n <= 1 ? -1 : n, row};  // one partition: the decode kernel wrote the row
+        });
         return;
     }
     int nps;

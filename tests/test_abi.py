@@ -98,8 +98,53 @@ def test_zero_sequences_is_a_no_op(L):
 
 
 def test_workspace_size_header_only_without_split():
-    n = pa.workspace_size(64, 32, 32, 128, 16, 4096, "bf16", num_sms=148)
+    n = pa.workspace_size(64, 32, 32, 128, 16, 4096, "bf16", num_sms=148,
+                          schedule="partitioned")
     assert n == pa.WORKSPACE_HEADER_BYTES
+
+
+def test_split_tail_plan_and_workspace():
+    """Whole units in two or three waves: the last wave's units (units mod CTA
+    slots) are cut into 4 partitions whose CTAs follow the whole units; the
+    workspace holds, after the header and the split-tail counts, their
+    partials ((D + 2) floats per row and partition), 256-byte aligned."""
+    S, Hq, Hk, D, B, T = 32, 32, 32, 128, 16, 8192
+    p = pa.plan(S, Hq, Hk, D, B, T, "bf16", num_sms=148)
+    units, slots = S * Hk, 3 * 148
+    tail = units % slots
+    assert (p["num_partitions"], p["tail_units"], p["tail_partitions"]) == (1, tail, 4)
+    assert p["tail_partition_pages"] == -(-(T // B) // 4)
+    assert p["grid_ctas"] == units - tail + 4 * tail
+    body0 = pa.WORKSPACE_HEADER_BYTES + pa.WORKSPACE_TAIL_COUNTER_BYTES
+    body = tail * (Hq // Hk) * 4 * (D + 2) * 4
+    assert p["workspace_bytes"] == body0 + -(-body // 256) * 256
+    assert pa.workspace_size(S, Hq, Hk, D, B, T, "bf16", num_sms=148) == p["workspace_bytes"]
+    # GQA: G rows per tail unit
+    q = pa.plan(128, 32, 8, 128, 16, 16384, "fp8_e4m3", num_sms=148)
+    tail = (128 * 8) % slots
+    assert (q["tail_units"], q["tail_partitions"], q["tail_partition_pages"]) == (tail, 4, 256)
+    body = tail * 4 * 4 * (128 + 2) * 4
+    assert q["workspace_bytes"] == body0 + -(-body // 256) * 256
+
+
+def test_split_tail_only_where_it_applies():
+    base = dict(num_sms=148)
+    # 1024 units (2.3 waves of 444 CTA slots) get one
+    assert pa.plan(32, 32, 32, 128, 16, 4096, "bf16", **base)["tail_units"] == 1024 % 444
+    # the partitioned schedule, forced partitions, a shared prefix, fewer than
+    # two or four and more waves of units, or units filling whole waves: none
+    assert pa.plan(32, 32, 32, 128, 16, 4096, "bf16", schedule="partitioned",
+                   **base)["tail_units"] == 0
+    assert pa.plan(32, 32, 32, 128, 16, 4096, "bf16", partition_pages=64,
+                   **base)["tail_units"] == 0
+    assert pa.plan(32, 32, 32, 128, 16, 4096, "bf16", shared_prefix_blocks=16,
+                   **base)["tail_units"] == 0
+    assert pa.plan(16, 32, 32, 128, 16, 4096, "bf16", **base)["tail_units"] == 0
+    assert pa.plan(64, 32, 32, 128, 16, 4096, "bf16", **base)["tail_units"] == 0  # 4.6 waves
+    assert pa.plan(111, 12, 3, 128, 16, 4096, "bf16", num_sms=37)["tail_units"] == 0  # 3 x 111
+    # tail partitions of fewer than 16 pages are not made
+    assert pa.plan(32, 32, 32, 128, 16, 960, "bf16", **base)["tail_units"] == 0
+    assert pa.plan(32, 32, 32, 128, 16, 1024, "bf16", **base)["tail_units"] > 0
 
 
 def test_balanced_workspace_layout():
@@ -109,7 +154,7 @@ def test_balanced_workspace_layout():
     assert p["balanced"] == 1 and p["num_partitions"] == 0 and p["grid_ctas"] == 3 * 148
     scan = -(-(64 + 2) * 4 // 256) * 256
     rows = 2 * p["grid_ctas"] * 4
-    expect = -(-(256 + scan + rows * 130 * 4) // 256) * 256
+    expect = -(-(256 + 2048 + scan + rows * 130 * 4) // 256) * 256
     assert p["workspace_bytes"] == expect
 
 
@@ -123,9 +168,12 @@ def test_planner_on_the_five_workloads():
     p1, p2, p3, p4, p5 = (_plan(i) for i in range(1, 6))
     assert all(p["balanced"] == 0 for p in (p1, p2, p3, p4, p5))
     assert p1["num_partitions"] == 1 and p1["partition_pages"] == 16
-    assert p2["num_partitions"] == 1 and p2["grid_ctas"] == 64 * 32
+    # whole units; in two or three waves, the last wave's units in 4 partitions
+    assert p2["num_partitions"] == 1 and p2["grid_ctas"] == 64 * 32 and p2["tail_units"] == 0
     assert p3["num_partitions"] == 1  # two waves of units; longest-first order
-    assert p4["num_partitions"] == 1 and p4["grid_ctas"] == 256 * 8
+    assert p3["tail_units"] == 128 * 8 % 444
+    assert p4["num_partitions"] == 1 and p4["grid_ctas"] == 256 * 8 and p4["tail_units"] == 0
+    assert p1["tail_units"] == 0 and p5["tail_units"] == 0
     assert p5["num_partitions"] >= 4  # 64 (seq, kv head) units cannot fill 148 SMs
     # balanced ranges on request: one wave of CTAs
     q2, q3, q4 = (_plan(i, schedule="balanced") for i in (2, 3, 4))
@@ -138,7 +186,7 @@ def test_planner_on_the_five_workloads():
     assert p5["num_partitions"] * p5["partition_pages"] >= c5.max_blocks_per_seq
     ws = pa.workspace_size(c5.num_seqs, c5.num_heads, c5.num_kv_heads, 128, 32, c5.max_seq_len,
                            num_sms=148)
-    assert ws >= 256 + 8 * 32 * p5["num_partitions"] * 130 * 4
+    assert ws >= 256 + 2048 + 8 * 32 * p5["num_partitions"] * 130 * 4
 
 
 def test_planner_splits_between_one_and_two_waves():
@@ -146,11 +194,13 @@ def test_planner_splits_between_one_and_two_waves():
     # last wave of 68 full-length units would run alone.
     p = pa.plan(64, 32, 8, 128, 16, 16384, "bf16", num_sms=148)
     assert p["num_partitions"] >= 2
-    # 1024 units (more than two waves) are not split.
+    # 1024 units (more than two waves) are not split, apart from the split
+    # tail under the auto schedule, which the partitioned schedule leaves out.
     p = pa.plan(128, 32, 8, 128, 16, 16384, "bf16", num_sms=148)
-    assert p["num_partitions"] == 1
-    assert pa.plan(128, 32, 8, 128, 16, 16384, "bf16", num_sms=148,
-                   schedule="partitioned") == p
+    assert p["num_partitions"] == 1 and p["tail_units"] == 1024 % 444
+    q = pa.plan(128, 32, 8, 128, 16, 16384, "bf16", num_sms=148, schedule="partitioned")
+    assert q["num_partitions"] == 1 and q["tail_units"] == 0
+    assert q["grid_ctas"] == 1024 and p["grid_ctas"] == 1024 + 3 * p["tail_units"]
 
 
 def test_balanced_schedule_limits():
@@ -272,7 +322,7 @@ def test_dynamic_schedule_plan_and_workspace():
         assert p["num_partitions"] == k and p["prefix_partitions"] == (k if pref else 0)
         assert p["prefix_groups"] == groups
         k_total = k * (2 if pref else 1)
-        expect = 256 + -(-units * 16 // 256) * 256 + c.num_seqs * c.num_heads * k_total * \
+        expect = 256 + 2048 + -(-units * 16 // 256) * 256 + c.num_seqs * c.num_heads * k_total * \
             (c.head_size + 2) * 4
         assert p["workspace_bytes"] == -(-expect // 256) * 256
         assert p["smem_bytes"] == p["warps_per_cta"] * p["stages"] * (
