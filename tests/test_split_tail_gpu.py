@@ -227,3 +227,27 @@ def test_workspace_shared_with_split_and_unsplit_plans():
         torch.cuda.synchronize()
         assert not _tail_counts(ws).any()
         compare(out, ref, cfg.kv_dtype, f"shared workspace pp={pp}")
+
+
+def test_wait_give_up_path_with_a_tail():
+    """With test_stall_copies every page wait gives up after ~20 ms: every
+    tail CTA still counts in once, so the call ends with the counts at 0,
+    a finite output and PA_DEV_WAIT_TIMEOUT set; a normal call on the same
+    workspace afterwards is correct."""
+    T = 64 * 16
+    sms = 16
+    lens = [T, 5, 0, 17 * 16, T - 3, 33, 16 * 16, T] * 5
+    cfg = _mixed(16, lens, seed=55)
+    wl = W.make_workload(cfg, DEV, seq_lens=lens)
+    assert _plan(cfg, sms)["tail_units"] > 0
+    ws = _ws(cfg, sms)
+    out = torch.full_like(wl.query, float("nan"))
+    run_gpu(wl, out=out, ws=ws, num_sms=sms, test_stall_copies=True)
+    torch.cuda.synchronize()
+    assert pa.read_status(ws, clear=True) & pa.PA_DEV_WAIT_TIMEOUT
+    assert torch.isfinite(out.float()).all()
+    assert not _tail_counts(ws).any()
+    good = run_gpu(wl, ws=ws, num_sms=sms)
+    torch.cuda.synchronize()
+    assert pa.read_status(ws) == 0
+    compare(good, run_oracle(wl), cfg.kv_dtype, "split tail after a give-up")
