@@ -380,8 +380,7 @@ def time_gpu(idx: int, steps: int, warmup: int, device, want_e2e=True, rank=0, n
     res = dict(cfg=cfg, wl=wl, plan=plan, alg_bytes=alg_bytes, kern_ms=kern_ms,
                region_ms=region_ms, step_ms=step_ms, local_step_ms=local_step_ms, flush=flush,
                steps=steps, clocks=clocks, status=status,
-               launches_per_step=1 + (plan["num_partitions"] > 1 or prefix > 0
-                                      or plan["balanced"] == 1 or plan["dynamic"] > 0),
+               launches_per_step=1 + plan["combine"],
                shared_prefix_blocks=prefix, alibi=alibi, extra=extra,
                options={"schedule": schedule, "mha_cuda_cores": bool(mha_cuda_cores),
                         "fp8_compute": bool(fp8_compute), "partition_pages": partition_pages,

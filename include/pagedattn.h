@@ -85,9 +85,9 @@ typedef enum pa_kv_dtype {
 /* Bytes at the start of the workspace reserved for the status word. */
 #define PA_WORKSPACE_HEADER_BYTES 256
 /* After the header, in any workspace larger than the header: the split
- * tail's per-unit CTA counts (at most 512 units), zero between calls; every
+ * tail's per-unit CTA counts (at most 1024 units), zero between calls; every
  * plan's partials start after them. */
-#define PA_WORKSPACE_TAIL_COUNTER_BYTES 2048
+#define PA_WORKSPACE_MERGE_COUNT_BYTES 4096
 
 /*
  * Tuning knobs; pass NULL for the planner's defaults.
@@ -196,6 +196,11 @@ typedef struct pa_plan {
                                  whole unit's (PA_SCHEDULE_AUTO only); 0: none          */
     int tail_partitions;
     int tail_partition_pages;
+    int combine;              /* 1: a pa_combine_kernel launch follows the decode
+                                 (split partitions, a shared prefix, balanced and
+                                 dynamic schedules); 0: none -- whole units, or a
+                                 split tail, whose units' last CTAs merge their
+                                 rows inside the decode kernel                  */
 } pa_plan;
 
 /*
@@ -209,8 +214,8 @@ pa_status pa_plan_decode(pa_plan* plan, int num_seqs, int num_heads, int num_kv_
 /*
  * Workspace bytes pa_decode needs (>= PA_WORKSPACE_HEADER_BYTES), or 0 when the
  * sizes are invalid.  Layout: a 256-byte header whose first uint32 is the
- * status word; when the plan needs more, PA_WORKSPACE_TAIL_COUNTER_BYTES of
- * split-tail counts, then (when P > 1 or a shared prefix is declared) per
+ * status word; when the plan needs more, PA_WORKSPACE_MERGE_COUNT_BYTES of
+ * merge counts, then (when P > 1 or a shared prefix is declared) per
  * (seq, query head, partition) an fp32 partial output [head_size], and fp32
  * running max (log2 domain) and sum -- or, with a split tail
  * (pa_plan.tail_units > 0), the same per (tail unit, query head of its

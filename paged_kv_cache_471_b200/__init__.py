@@ -35,7 +35,7 @@ PA_DEV_WAIT_TIMEOUT = 0x4
 PA_DEV_PREFIX_MISMATCH = 0x8
 
 WORKSPACE_HEADER_BYTES = 256
-WORKSPACE_TAIL_COUNTER_BYTES = 2048  # after the header when the plan needs more
+WORKSPACE_MERGE_COUNT_BYTES = 4096  # after the header when the plan needs more
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 _KV = {"bf16": PA_KV_BF16, "auto": PA_KV_BF16, "fp8": PA_KV_FP8_E4M3, "fp8_e4m3": PA_KV_FP8_E4M3,
@@ -63,7 +63,8 @@ class Plan(ctypes.Structure):
                 ("workspace_bytes", ctypes.c_size_t), ("prefix_partitions", ctypes.c_int),
                 ("prefix_groups", ctypes.c_int), ("balanced", ctypes.c_int),
                 ("dynamic", ctypes.c_int), ("tail_units", ctypes.c_longlong),
-                ("tail_partitions", ctypes.c_int), ("tail_partition_pages", ctypes.c_int)]
+                ("tail_partitions", ctypes.c_int), ("tail_partition_pages", ctypes.c_int),
+                ("combine", ctypes.c_int)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}

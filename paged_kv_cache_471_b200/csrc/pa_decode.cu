@@ -28,11 +28,12 @@ constexpr unsigned long long kTestWaitLimitNs = 20000000ull;  // with test_stall
 constexpr long long kLongPartitionPages = 256;
 // Split tail: partitions per unit of the last, partial wave of whole units.
 constexpr int kTailParts = 4;
-// Workspace layout: the header (status word, dynamic-schedule words), then a
-// region of split-tail counters that only the split tail touches (they are 0
-// between calls), then the plan's partials (or page scan, or unit counters).
-constexpr long long kMaxTailUnits = PA_WORKSPACE_TAIL_COUNTER_BYTES / sizeof(unsigned int);
-constexpr size_t kBodyOffset = PA_WORKSPACE_HEADER_BYTES + PA_WORKSPACE_TAIL_COUNTER_BYTES;
+// Workspace layout: the header (status word, dynamic-schedule words), then
+// the split tail's per-unit merge counts, which nothing else touches (they
+// are 0 between calls), then the plan's partials (or page scan, or unit
+// counters).
+constexpr long long kMergeCounts = PA_WORKSPACE_MERGE_COUNT_BYTES / sizeof(unsigned int);
+constexpr size_t kBodyOffset = PA_WORKSPACE_HEADER_BYTES + PA_WORKSPACE_MERGE_COUNT_BYTES;
 constexpr int kDefaultStages = 2;
 constexpr int kMaxShortStages = 4;
 constexpr size_t kShortStagesSmem = 96 * 1024;  // keep >= 2 CTAs per SM
@@ -159,6 +160,7 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
     pl->tail_units = 0;
     pl->tail_partitions = 0;
     pl->tail_partition_pages = 0;
+    pl->combine = 0;
     if (schedule == PA_SCHEDULE_DYNAMIC) {
         // Persistent warps claiming pages (pa_decode_dynamic.cuh): one wave of
         // CTAs; per query row, a slot per warp that read its unit (at most
@@ -200,6 +202,7 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         pl->prefix_groups = static_cast<int>(groups);
         pl->balanced = 0;
         pl->dynamic = static_cast<int>(owners);
+        pl->combine = 1;
         return PA_OK;
     }
     const bool br_fits = !cascade && !forced_pp && num_seqs > 0 &&
@@ -226,6 +229,7 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         pl->prefix_partitions = 0;
         pl->prefix_groups = 0;
         pl->balanced = 1;
+        pl->combine = 1;
         return PA_OK;
     }
     long long pp;
@@ -290,7 +294,7 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
     if (whole_units && !cascade && schedule == PA_SCHEDULE_AUTO && units < 4 * slots) {
         const long long r = units % slots;
         const long long tpp = (pages_max + kTailParts - 1) / kTailParts;
-        if (r > 0 && r <= kMaxTailUnits && tpp >= kMinPartitionPages) {
+        if (r > 0 && r <= kMergeCounts && tpp >= kMinPartitionPages) {
             tail_units = r;
             tail_P = kTailParts;
             tail_PP = static_cast<int>(tpp);
@@ -329,6 +333,11 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
     pl->tail_units = tail_units;
     pl->tail_partitions = tail_P;
     pl->tail_partition_pages = tail_PP;
+    // Split partials are merged by the combine kernel (merging them in the
+    // decode kernel, by each unit's last CTA, measured slower on B200: -1.7%
+    // on the long-context workload, -3.9% on a 100 us call); the split tail's
+    // are merged in the kernel.
+    pl->combine = (P > 1 || cascade) ? 1 : 0;
     pl->smem_bytes = smem;
     pl->workspace_bytes = ws;
     pl->prefix_partitions = static_cast<int>(p_pre);
@@ -702,7 +711,9 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
     p.n_full = static_cast<long long>(num_seqs) * num_kv_heads - pl.tail_units;
     p.tail_P = pl.tail_partitions;
     p.tail_PP = pl.tail_partition_pages;
-    p.tail_cnt = reinterpret_cast<unsigned int*>(ws + PA_WORKSPACE_HEADER_BYTES);
+    p.merge_cnt = pl.tail_partitions > 0
+                      ? reinterpret_cast<unsigned int*>(ws + PA_WORKSPACE_HEADER_BYTES)
+                      : nullptr;
     p.S = num_seqs;
     p.Hq = num_heads;
     p.Hk = num_kv_heads;
@@ -789,7 +800,7 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
     cudaError_t e = launch_any(p, head_size, block_size, kv_dtype == PA_KV_FP8_E4M3, f8mma, sc,
                                pl.grid_ctas, pl.smem_bytes, s);
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
-    if (pl.balanced || pl.num_partitions > 1 || p.prefix_pages > 0) {
+    if (pl.combine) {
         pa::CombineParams c;
         std::memset(&c, 0, sizeof c);
         c.out = p.out;

@@ -102,12 +102,13 @@ struct DecodeParams {
     // first n_full per-sequence units run whole; each remaining unit is cut
     // into tail_P partitions of tail_PP pages, whose CTAs come after every
     // whole unit's.  Tail unit t = unit - n_full writes its partials at rows
-    // (t * G + g) * tail_P + part of ws_o / ws_m / ws_l and counts its CTAs
-    // in tail_cnt[t]; the last of them merges the unit's rows into out and
-    // sets the count back to 0 (counts are 0 between calls).
+    // (t * G + g) * tail_P + part of ws_o / ws_m / ws_l.
     long long n_full;
     int tail_P, tail_PP;
-    unsigned int* tail_cnt;
+    // The split tail's merge counts: each CTA of tail unit t counts itself in
+    // at merge_cnt[t]; the unit's last CTA merges its rows into out and sets
+    // the count back to 0 (counts are 0 between calls).
+    unsigned int* merge_cnt;
 };
 
 // Bytes of shared memory the final merge needs (it overlays the page stages).
@@ -890,6 +891,101 @@ struct WarpAttnScalar {
     }
 };
 
+// What a row's merge needs once its slots' loads are in flight: how many
+// slots it has (< 0: nothing to do, the decode kernel wrote the row) and
+// which row of out it writes.
+struct SlotRow {
+    int nps;
+    long long out_row;
+};
+
+// The merge of one row whose slots fit in a warp (at most 32), at partial
+// rows base .. base + np - 1: every load it needs -- each slot's (max, sum),
+// one slot per lane, the partial rows of the first 16 slots (D / 32
+// consecutive head dims per lane), and whatever row_info reads -- is issued
+// before any of them is used, so a row costs one memory round trip (a second
+// one for slots 16..31).  Slots past the row's count (and an empty slot's
+// row) may hold anything; their weight is 0 and a select drops them.  The
+// partials are read through L2 (other CTAs of the same kernel may have just
+// written them).
+template <int D, class RowInfo>
+__device__ __forceinline__ void merge_slots(const float* ws_o, const float* ws_m,
+                                            const float* ws_l, __nv_bfloat16* out,
+                                            long long base, int np, int lane, RowInfo row_info) {
+    constexpr int V = D / 32;  // head dims per lane: 4 * lane .. (D = 128) or 2 * lane ..
+    constexpr int KO = 16;     // partial rows loaded up front
+    float l = 0.f, m = -INFINITY;
+    if (lane < np) {
+        l = __ldcg(ws_l + base + lane);
+        m = __ldcg(ws_m + base + lane);
+    }
+    auto load_row = [&](int i, float (&v)[V]) {
+        const float* src = ws_o + (base + i) * D + V * lane;
+        if constexpr (V == 4) {
+            const float4 x = __ldcg(reinterpret_cast<const float4*>(src));
+            v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+        } else {
+            const float2 x = __ldcg(reinterpret_cast<const float2*>(src));
+            v[0] = x.x; v[1] = x.y;
+        }
+    };
+    float o[KO][V];
+#pragma unroll
+    for (int i = 0; i < KO; ++i) {
+        if (i < np) {
+            load_row(i, o[i]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < V; ++j) o[i][j] = 0.f;
+        }
+    }
+    const SlotRow r = row_info();
+    if (r.nps < 0) return;
+    const int nps = r.nps;
+    const bool live = lane < nps && l > 0.f;
+    float M = live ? m : -INFINITY;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
+    const float wt = live ? exp2f(m - M) * l : 0.f;
+    float L = wt;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(kFull, L, off);
+    float a[V];
+#pragma unroll
+    for (int j = 0; j < V; ++j) a[j] = 0.f;
+#pragma unroll
+    for (int i = 0; i < KO; ++i) {
+        const float w = __shfl_sync(kFull, wt, i);
+#pragma unroll
+        for (int j = 0; j < V; ++j) a[j] += w > 0.f ? w * o[i][j] : 0.f;
+    }
+    for (int i0 = KO; i0 < nps; i0 += 8) {
+        float q[8][V];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (i0 + i < nps) {
+                load_row(i0 + i, q[i]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < V; ++j) q[i][j] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float w = __shfl_sync(kFull, wt, (i0 + i) & 31);
+#pragma unroll
+            for (int j = 0; j < V; ++j) a[j] += (i0 + i < nps && w > 0.f) ? w * q[i][j] : 0.f;
+        }
+    }
+    __nv_bfloat16* dst = out + r.out_row * D + V * lane;
+#pragma unroll
+    for (int j = 0; j < V; j += 2) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(L > 0.f ? a[j] / L : 0.f,
+                                                       L > 0.f ? a[j + 1] / L : 0.f);
+        *reinterpret_cast<__nv_bfloat162*>(dst + j) = h;
+    }
+}
+
 // The paired 8-row form with f16 MMAs is held to three CTAs per SM (170
 // registers), the residency of the other 8-row forms.
 // SC: one query head per kv head on the CUDA cores (WarpAttnScalar).
@@ -1156,41 +1252,25 @@ __global__ void __launch_bounds__(W * 32,
                                                     : ((Pu == 1) || (nb <= PPu)));
 
         // Split tail: once this CTA's partial rows are stored (or it had no
-        // pages), count it in; the unit's last CTA merges the partials of its
-        // partitions that have pages (log-sum-exp, as pa_combine_kernel does)
-        // into out, unless one partition held the whole sequence and wrote out
-        // itself, and leaves the count at 0 for the next call.
+        // pages), it counts itself in on its unit; the unit's last CTA merges
+        // the partials of its partitions that have pages (a warp per row, as
+        // pa_combine_kernel does) into out -- unless one partition held the
+        // whole sequence and wrote out itself -- and leaves the count at 0.
         auto tail_arrive = [&]() {
             __threadfence();  // this thread's partial stores before the count
             __syncthreads();
             int last = 0;
             if (threadIdx.x == 0)
-                last = atomicAdd(p.tail_cnt + tail_t, 1u) == static_cast<unsigned>(p.tail_P - 1);
+                last = atomicAdd(p.merge_cnt + tail_t, 1u) == static_cast<unsigned>(p.tail_P - 1);
             if (!__syncthreads_or(last)) return;
-            __threadfence();
+            __threadfence();  // the other partitions' partials before reading them
+            if (threadIdx.x == 0) p.merge_cnt[tail_t] = 0u;  // all of the unit's CTAs are in
             const int nps = min(p.tail_P, (nb + p.tail_PP - 1) / p.tail_PP);
-            if (nps > 1) {
-                const long long base = tail_t * p.G * p.tail_P;
-                for (int idx = threadIdx.x; idx < p.G * D; idx += (W * 32)) {
-                    const int g = idx / D;
-                    const int d = idx - g * D;
-                    const long long r0 = base + static_cast<long long>(g) * p.tail_P;
-                    float M = -INFINITY;
-                    for (int i = 0; i < nps; ++i)
-                        if (__ldcg(p.ws_l + r0 + i) > 0.f) M = fmaxf(M, __ldcg(p.ws_m + r0 + i));
-                    float L = 0.f, O = 0.f;
-                    for (int i = 0; i < nps; ++i) {
-                        const float l = __ldcg(p.ws_l + r0 + i);
-                        if (l > 0.f) {
-                            const float w = exp2f(__ldcg(p.ws_m + r0 + i) - M) * l;
-                            L += w;
-                            O += w * __ldcg(p.ws_o + (r0 + i) * D + d);
-                        }
-                    }
-                    p.out[(row0 + g) * D + d] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
-                }
-            }
-            if (threadIdx.x == 0) p.tail_cnt[tail_t] = 0u;
+            if (nps <= 1) return;
+            const long long prow0 = tail_t * p.G * p.tail_P;
+            for (int g = warp; g < p.G; g += W)
+                merge_slots<D>(p.ws_o, p.ws_m, p.ws_l, p.out, prow0 + g * p.tail_P, p.tail_P,
+                               lane, [&]() -> SlotRow { return {nps, row0 + g}; });
         };
 
         if (j0 >= j1) {
@@ -1400,98 +1480,6 @@ struct CombineParams {
     const unsigned long long* dyn_uw;
 };
 
-// What a row's merge needs once its slots' loads are in flight: how many
-// slots it has (< 0: nothing to do, the decode kernel wrote the row) and
-// which row of out it writes.
-struct SlotRow {
-    int nps;
-    long long out_row;
-};
-
-// The merge of one row whose slots fit in a warp (at most 32), at partial
-// rows base .. base + np - 1: every load it needs -- each slot's (max, sum),
-// one slot per lane, the partial rows of the first 16 slots (D / 32
-// consecutive head dims per lane), and whatever row_info reads -- is issued
-// before any of them is used, so a row costs one memory round trip (a second
-// one for slots 16..31).  Slots past the row's count (and an empty slot's
-// row) may hold anything; their weight is 0 and a select drops them.
-template <int D, class RowInfo>
-__device__ __forceinline__ void merge_slots(const CombineParams& p, long long base, int np,
-                                            int lane, RowInfo row_info) {
-    constexpr int V = D / 32;  // head dims per lane: 4 * lane .. (D = 128) or 2 * lane ..
-    constexpr int KO = 16;     // partial rows loaded up front
-    float l = 0.f, m = -INFINITY;
-    if (lane < np) {
-        l = p.ws_l[base + lane];
-        m = p.ws_m[base + lane];
-    }
-    auto load_row = [&](int i, float (&v)[V]) {
-        const float* src = p.ws_o + (base + i) * D + V * lane;
-        if constexpr (V == 4) {
-            const float4 x = *reinterpret_cast<const float4*>(src);
-            v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
-        } else {
-            const float2 x = *reinterpret_cast<const float2*>(src);
-            v[0] = x.x; v[1] = x.y;
-        }
-    };
-    float o[KO][V];
-#pragma unroll
-    for (int i = 0; i < KO; ++i) {
-        if (i < np) {
-            load_row(i, o[i]);
-        } else {
-#pragma unroll
-            for (int j = 0; j < V; ++j) o[i][j] = 0.f;
-        }
-    }
-    const SlotRow r = row_info();
-    if (r.nps < 0) return;
-    const int nps = r.nps;
-    const bool live = lane < nps && l > 0.f;
-    float M = live ? m : -INFINITY;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
-    const float wt = live ? exp2f(m - M) * l : 0.f;
-    float L = wt;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(kFull, L, off);
-    float a[V];
-#pragma unroll
-    for (int j = 0; j < V; ++j) a[j] = 0.f;
-#pragma unroll
-    for (int i = 0; i < KO; ++i) {
-        const float w = __shfl_sync(kFull, wt, i);
-#pragma unroll
-        for (int j = 0; j < V; ++j) a[j] += w > 0.f ? w * o[i][j] : 0.f;
-    }
-    for (int i0 = KO; i0 < nps; i0 += 8) {
-        float q[8][V];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            if (i0 + i < nps) {
-                load_row(i0 + i, q[i]);
-            } else {
-#pragma unroll
-                for (int j = 0; j < V; ++j) q[i][j] = 0.f;
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float w = __shfl_sync(kFull, wt, (i0 + i) & 31);
-#pragma unroll
-            for (int j = 0; j < V; ++j) a[j] += (i0 + i < nps && w > 0.f) ? w * q[i][j] : 0.f;
-        }
-    }
-    __nv_bfloat16* dst = p.out + r.out_row * D + V * lane;
-#pragma unroll
-    for (int j = 0; j < V; j += 2) {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(L > 0.f ? a[j] / L : 0.f,
-                                                       L > 0.f ? a[j + 1] / L : 0.f);
-        *reinterpret_cast<__nv_bfloat162*>(dst + j) = h;
-    }
-}
-
 // Log-sum-exp merge of the split-KV partials of one (sequence, q head) per
 // warp:  M = max_p m_p;  w_p = l_p 2^(m_p - M);  out = sum_p w_p o_p / sum_p w_p.
 // Without a shared prefix, rows whose sequence fits in one partition were
@@ -1521,7 +1509,8 @@ __global__ void __launch_bounds__(kThreads) pa_combine_kernel(const CombineParam
     const int s = static_cast<int>(row / p.Hq);
     if (!p.dynamic && !p.balanced && p.P_total <= 32) {
         // The row's slots: the prefix partitions, then the sequence's own.
-        merge_slots<D>(p, row * p.P_total, p.P_total, lane, [&]() -> SlotRow {
+        merge_slots<D>(p.ws_o, p.ws_m, p.ws_l, p.out, row * p.P_total, p.P_total, lane,
+                       [&]() -> SlotRow {
             if (p.prefix_pages > 0) {
                 const int T = max(0, min(p.seq_lens[s], p.max_blocks * p.B));
                 const int nb = (T + p.B - 1) / p.B;

@@ -115,7 +115,7 @@ def test_split_tail_plan_and_workspace():
     assert (p["num_partitions"], p["tail_units"], p["tail_partitions"]) == (1, tail, 4)
     assert p["tail_partition_pages"] == -(-(T // B) // 4)
     assert p["grid_ctas"] == units - tail + 4 * tail
-    body0 = pa.WORKSPACE_HEADER_BYTES + pa.WORKSPACE_TAIL_COUNTER_BYTES
+    body0 = pa.WORKSPACE_HEADER_BYTES + pa.WORKSPACE_MERGE_COUNT_BYTES
     body = tail * (Hq // Hk) * 4 * (D + 2) * 4
     assert p["workspace_bytes"] == body0 + -(-body // 256) * 256
     assert pa.workspace_size(S, Hq, Hk, D, B, T, "bf16", num_sms=148) == p["workspace_bytes"]
@@ -147,6 +147,23 @@ def test_split_tail_only_where_it_applies():
     assert pa.plan(32, 32, 32, 128, 16, 1024, "bf16", **base)["tail_units"] > 0
 
 
+def test_where_the_split_partials_are_merged():
+    """By the combine kernel for split partitions, a shared prefix and the
+    balanced and dynamic schedules; a split tail's inside the decode kernel
+    (no combine launch); whole units need no merge."""
+    base = dict(num_sms=148)
+    assert pa.plan(8, 32, 8, 128, 32, 131072, "bf16", shared_prefix_blocks=1024,
+                   **base)["combine"] == 1
+    assert pa.plan(64, 32, 16, 128, 16, 4096, "bf16", partition_pages=64,
+                   **base)["combine"] == 1
+    assert pa.plan(32, 32, 32, 128, 16, 8192, "bf16", **base)["combine"] == 0  # split tail
+    assert pa.plan(64, 32, 32, 128, 16, 4096, "bf16", **base)["combine"] == 0  # whole units
+    assert pa.plan(64, 32, 8, 128, 16, 4096, "bf16", schedule="balanced",
+                   **base)["combine"] == 1
+    assert pa.plan(64, 32, 8, 128, 16, 4096, "bf16", schedule="dynamic",
+                   **base)["combine"] == 1
+
+
 def test_balanced_workspace_layout():
     # header, the per-sequence page scan (S + 2 ints, 256-byte aligned), then
     # two slots of G rows of (D + 2) floats per CTA slot.
@@ -154,7 +171,7 @@ def test_balanced_workspace_layout():
     assert p["balanced"] == 1 and p["num_partitions"] == 0 and p["grid_ctas"] == 3 * 148
     scan = -(-(64 + 2) * 4 // 256) * 256
     rows = 2 * p["grid_ctas"] * 4
-    expect = -(-(256 + 2048 + scan + rows * 130 * 4) // 256) * 256
+    expect = -(-(256 + 4096 + scan + rows * 130 * 4) // 256) * 256
     assert p["workspace_bytes"] == expect
 
 
@@ -186,7 +203,7 @@ def test_planner_on_the_five_workloads():
     assert p5["num_partitions"] * p5["partition_pages"] >= c5.max_blocks_per_seq
     ws = pa.workspace_size(c5.num_seqs, c5.num_heads, c5.num_kv_heads, 128, 32, c5.max_seq_len,
                            num_sms=148)
-    assert ws >= 256 + 2048 + 8 * 32 * p5["num_partitions"] * 130 * 4
+    assert ws >= 256 + 4096 + 8 * 32 * p5["num_partitions"] * 130 * 4
 
 
 def test_planner_splits_between_one_and_two_waves():
@@ -322,7 +339,7 @@ def test_dynamic_schedule_plan_and_workspace():
         assert p["num_partitions"] == k and p["prefix_partitions"] == (k if pref else 0)
         assert p["prefix_groups"] == groups
         k_total = k * (2 if pref else 1)
-        expect = 256 + 2048 + -(-units * 16 // 256) * 256 + c.num_seqs * c.num_heads * k_total * \
+        expect = 256 + 4096 + -(-units * 16 // 256) * 256 + c.num_seqs * c.num_heads * k_total * \
             (c.head_size + 2) * 4
         assert p["workspace_bytes"] == -(-expect // 256) * 256
         assert p["smem_bytes"] == p["warps_per_cta"] * p["stages"] * (

@@ -180,6 +180,13 @@ def test_back_to_back_calls_sharing_a_workspace():
     for i, o in enumerate(outs):
         assert torch.equal(o, alone[i % 2]), f"call {i}"
     compare(alone[1], run_oracle(wb), c.kv_dtype, "second batch")
+    _merge_counts_are_zero(ws)
+
+
+def _merge_counts_are_zero(ws):
+    """The in-kernel merge leaves every unit's count at 0 after a call."""
+    lo = pa.WORKSPACE_HEADER_BYTES
+    assert not ws[lo:lo + pa.WORKSPACE_MERGE_COUNT_BYTES].any()
 
 
 def test_calls_captured_in_a_cuda_graph():
@@ -208,6 +215,7 @@ def test_calls_captured_in_a_cuda_graph():
         torch.cuda.synchronize()
         for i, o in enumerate(outs):
             assert torch.equal(o, alone[i % 2]), f"graph call {i}"
+        _merge_counts_are_zero(ws)
     del graph
 
 
@@ -245,6 +253,8 @@ def test_writes_stay_inside_out_and_workspace(case):
     assert (obuf[:G_OUT] == sentinel).all() and (obuf[-G_OUT:] == sentinel).all()
     assert (wbuf[:G_WS] == 0xA5).all() and (wbuf[-G_WS:] == 0xA5).all()
     assert pa.read_status(ws) == 0
+    if need > pa.WORKSPACE_HEADER_BYTES:
+        _merge_counts_are_zero(ws)
     compare(out, run_oracle(wl), c.kv_dtype, case)
 
 

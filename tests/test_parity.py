@@ -44,18 +44,27 @@ def test_reduced_workloads(idx, partition_pages):
 
 
 # Partition sizes that put a row's slot count (prefix partitions plus the
-# sequence's own) in each regime of the combine: at most 16 (one batch of
-# partial rows), 17..32 (a second batch), exactly 32, and more than 32 (the
-# slots read 32 at a time).
+# sequence's own) in each regime of the combine kernel: at most 16 (one batch
+# of partial rows), 17..32 (a second batch), exactly 32, and more than 32 (the
+# slots read 32 at a time), on the reduced workloads and on a batch of 1040
+# (sequence, kv head) units.
 SLOT_REGIMES = {
     3: [(9, "<=16"), (5, "17..32"), (4, ">32")],
     5: [(64, "<=16"), (8, "17..32"), (5, "32"), (4, ">32")],
+    "many units": [(3, "<=16"), (2, "17..32"), (1, ">32")],
+    "many units, prefix": [(4, "<=16"), (2, "17..32"), (1, ">32")],
 }
+MANY_UNITS = W.PagedConfig("1040 units", num_seqs=260, num_heads=8, num_kv_heads=4, head_size=64,
+                           block_size=16, num_blocks=260 * 38 + 16, seq_len_lo=300,
+                           seq_len_hi=600, seed=4242)
+MANY_UNITS_PREFIX = MANY_UNITS.replace(name="1040 units, prefix", shared_prefix_blocks=8,
+                                       seq_len_lo=400)
 
 
-@pytest.mark.parametrize("idx", sorted(SLOT_REGIMES))
+@pytest.mark.parametrize("idx", list(SLOT_REGIMES), ids=str)
 def test_combine_slot_count_regimes(idx):
-    cfg = REDUCED[idx]
+    cfg = {"many units": MANY_UNITS, "many units, prefix": MANY_UNITS_PREFIX}.get(idx)
+    cfg = cfg if cfg is not None else REDUCED[idx]
     wl = W.make_workload(cfg, DEV)
     ref = run_oracle(wl)
     for pp, regime in SLOT_REGIMES[idx]:
@@ -66,6 +75,7 @@ def test_combine_slot_count_regimes(idx):
         ok = {"<=16": slots <= 16, "17..32": 16 < slots < 32, "32": slots == 32,
               ">32": slots > 32}[regime]
         assert ok, (pp, regime, slots)
+        assert plan["combine"] == 1
         out = torch.full_like(wl.query, float("nan"))
         run_gpu(wl, out=out, partition_pages=pp, shared_prefix_blocks=cfg.shared_prefix_blocks)
         torch.cuda.synchronize()
@@ -172,6 +182,16 @@ PREFIX_CASES = {
                                   head_size=64, block_size=16, num_blocks=20 + 3 * 40 + 8,
                                   seq_len_lo=400, seq_len_hi=640, shared_prefix_blocks=20,
                                   seed=31),
+    # group sizes that do not divide 16: a sequence's rows fall in two 16-row
+    # prefix groups
+    "b32_bf16_g5": W.PagedConfig("prefix G=5", num_seqs=7, num_heads=10, num_kv_heads=2,
+                                 head_size=128, block_size=32, num_blocks=3 + 7 * 48 + 8,
+                                 seq_len_lo=100, seq_len_hi=1500, shared_prefix_blocks=3,
+                                 seed=32),
+    "b16_bf16_g3": W.PagedConfig("prefix G=3", num_seqs=11, num_heads=6, num_kv_heads=2,
+                                 head_size=64, block_size=16, num_blocks=12 + 11 * 60 + 8,
+                                 seq_len_lo=200, seq_len_hi=950, shared_prefix_blocks=12,
+                                 seed=33),
 }
 
 

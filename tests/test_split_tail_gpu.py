@@ -149,7 +149,7 @@ def test_full_size_noalloc_matches_workspace_call(idx):
 
 def _tail_counts(ws):
     lo = pa.WORKSPACE_HEADER_BYTES
-    return ws[lo:lo + pa.WORKSPACE_TAIL_COUNTER_BYTES]
+    return ws[lo:lo + pa.WORKSPACE_MERGE_COUNT_BYTES]
 
 
 def test_back_to_back_calls_graph_and_guard_bands():

@@ -54,11 +54,11 @@ def _cover(plan, S, Hq, Hk, D, B, T):
     # tail CTAs follow every whole unit's
     assert all(page_owner[(u, 0)] < n_full for u in range(n_full))
     # partial rows fit the workspace: header, tail counts, (D + 2) floats per row
-    need = (pa.WORKSPACE_HEADER_BYTES + pa.WORKSPACE_TAIL_COUNTER_BYTES
+    need = (pa.WORKSPACE_HEADER_BYTES + pa.WORKSPACE_MERGE_COUNT_BYTES
             + len(rows) * (D + 2) * 4)
     assert max(rows, default=-1) < n_tail * G * tP
     assert plan["workspace_bytes"] >= need
-    assert n_tail <= pa.WORKSPACE_TAIL_COUNTER_BYTES // 4
+    assert n_tail <= pa.WORKSPACE_MERGE_COUNT_BYTES // 4
 
 
 SHAPES = [(S, Hq, Hk, D, B, T) for S, (Hq, Hk), D, B, T in itertools.product(
