@@ -201,6 +201,9 @@ typedef struct pa_plan {
                                  dynamic schedules); 0: none -- whole units, or a
                                  split tail, whose units' last CTAs merge their
                                  rows inside the decode kernel                  */
+    int longest_first;        /* 1: per-sequence CTAs take sequences longest first
+                                 (ranked on the device from seq_lens; at most 256
+                                 sequences, grids of more than one wave of CTAs) */
 } pa_plan;
 
 /*

@@ -64,7 +64,7 @@ class Plan(ctypes.Structure):
                 ("prefix_groups", ctypes.c_int), ("balanced", ctypes.c_int),
                 ("dynamic", ctypes.c_int), ("tail_units", ctypes.c_longlong),
                 ("tail_partitions", ctypes.c_int), ("tail_partition_pages", ctypes.c_int),
-                ("combine", ctypes.c_int)]
+                ("combine", ctypes.c_int), ("longest_first", ctypes.c_int)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}

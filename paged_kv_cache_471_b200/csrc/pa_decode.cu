@@ -161,6 +161,7 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
     pl->tail_partitions = 0;
     pl->tail_partition_pages = 0;
     pl->combine = 0;
+    pl->longest_first = 0;
     if (schedule == PA_SCHEDULE_DYNAMIC) {
         // Persistent warps claiming pages (pa_decode_dynamic.cuh): one wave of
         // CTAs; per query row, a slot per warp that read its unit (at most
@@ -333,6 +334,12 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
     pl->tail_units = tail_units;
     pl->tail_partitions = tail_P;
     pl->tail_partition_pages = tail_PP;
+    // Longest first (ranked on the device) only when the grid takes more than
+    // one wave of CTA slots: in one wave every CTA starts at once and the
+    // order does not matter, and ranking would put the length loads ahead of
+    // every block-table read.
+    pl->longest_first =
+        (num_seqs > 1 && num_seqs <= kMaxRankedSeqs && pl->grid_ctas > slots) ? 1 : 0;
     // Split partials are merged by the combine kernel (merging them in the
     // decode kernel, by each unit's last CTA, measured slower on B200: -1.7%
     // on the long-context workload, -3.9% on a 100 us call); the split tail's
@@ -730,7 +737,7 @@ pa_status pa_decode_ex(void* out, const void* query, const void* key_cache,
     p.prefix_units = static_cast<long long>(num_kv_heads) * pl.prefix_groups * pl.prefix_partitions;
     p.P_total = p_total;
     p.alibi = opts ? opts->alibi_slopes : nullptr;
-    p.longest_first = (!pl.balanced && num_seqs > 1 && num_seqs <= kMaxRankedSeqs) ? 1 : 0;
+    p.longest_first = pl.longest_first;
     p.balanced = pl.balanced;
     p.stall_tx_bytes = 0;
     p.wait_limit_ns = kWaitLimitNs;

@@ -147,6 +147,18 @@ def test_split_tail_only_where_it_applies():
     assert pa.plan(32, 32, 32, 128, 16, 1024, "bf16", **base)["tail_units"] > 0
 
 
+def test_longest_first_only_for_more_than_one_wave():
+    # ranked when the grid takes more than one wave of 444 CTA slots
+    p1, p2, p3, p5 = (_plan(i) for i in (1, 2, 3, 5))
+    assert p1["grid_ctas"] <= 444 and p1["longest_first"] == 0
+    assert p2["longest_first"] == 1 and p3["longest_first"] == 1 and p5["longest_first"] == 1
+    # one sequence, more than 256 sequences, or the balanced schedule: never
+    assert pa.plan(1, 32, 8, 128, 16, 131072, "bf16", num_sms=148)["longest_first"] == 0
+    assert pa.plan(300, 32, 8, 128, 16, 4096, "bf16", num_sms=148)["longest_first"] == 0
+    assert pa.plan(64, 32, 8, 128, 16, 4096, "bf16", num_sms=148,
+                   schedule="balanced")["longest_first"] == 0
+
+
 def test_where_the_split_partials_are_merged():
     """By the combine kernel for split partitions, a shared prefix and the
     balanced and dynamic schedules; a split tail's inside the decode kernel

@@ -83,6 +83,23 @@ def test_combine_slot_count_regimes(idx):
         assert pa.read_status(device=DEV) == 0
 
 
+@pytest.mark.parametrize("schedule", ["auto", "partitioned"])
+def test_longest_first_ranking_with_ties(schedule):
+    """Planned for 2 SMs, the reduced GQA batch (48 units) takes several waves
+    of CTAs, so CTAs take its sequences longest first, ranked on the device;
+    lengths with ties and an empty sequence."""
+    cfg = REDUCED[3]
+    lens = [2100, 100, 2100, 0, 1500, 100]
+    wl = W.make_workload(cfg, DEV, seq_lens=lens)
+    p = pa.plan(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_size, cfg.block_size,
+                cfg.max_seq_len, cfg.kv_dtype, num_sms=2, schedule=schedule)
+    assert p["longest_first"] == 1 and p["num_partitions"] == 1
+    out = torch.full_like(wl.query, float("nan"))
+    run_gpu(wl, out=out, num_sms=2, schedule=schedule)
+    torch.cuda.synchronize()
+    compare(out, run_oracle(wl), cfg.kv_dtype, f"longest first {schedule}")
+
+
 @pytest.mark.parametrize("idx", [1, 3, 4, 5])
 def test_pa_decode_symbol_through_ctypes(idx):
     """The boundary call itself, pa_decode (no options), called through
