@@ -286,10 +286,10 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
     // last, partial wave (units mod CTA slots) are cut into kTailParts
     // partitions each, dispatched after every whole unit, so that the call
     // does not end on a few full-length units streaming alone (measured on
-    // B200: +2.7% and +3.4% on equal-length batches of 1024 units; -0.35% when
-    // the last units are the short ones of mixed lengths; from four waves up
-    // the last wave is a small enough share that the gains and losses even
-    // out, so it is not split there).
+    // B200: +2.4% to +4.0% on equal-length batches of 1024 units; -0.2% to
+    // -0.35% when the last units are the short ones of mixed lengths; from four
+    // waves up the last wave is a small enough share that the gains and losses
+    // even out, so it is not split there).
     long long tail_units = 0;
     int tail_P = 0, tail_PP = 0;
     if (whole_units && !cascade && schedule == PA_SCHEDULE_AUTO && units < 4 * slots) {
