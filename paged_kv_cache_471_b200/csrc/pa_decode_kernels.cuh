@@ -79,7 +79,13 @@ struct DecodeParams {
     int prefix_pages;         // 0: no shared prefix
     int prefix_parts;         // partitions of the prefix
     int prefix_groups;        // 16-row groups of the S*G query rows of a kv head
-    long long prefix_units;   // Hk * prefix_groups * prefix_parts
+    // Prefix CTAs per (kv head, partition): with prefix_shared (at least W
+    // groups), one per W groups, streaming each page once through a ring
+    // shared by its warps (prefix_shared_ring); otherwise one per group, its
+    // warps splitting the pages like a sequence's unit.
+    int prefix_shared;
+    int prefix_cta_groups;
+    long long prefix_units;   // Hk * prefix_cta_groups * prefix_parts
     int P_total;              // partial slots per (seq, q head): prefix_parts + P
     const float* alibi;       // [Hq] ALiBi slopes, or nullptr
     // Failure-path test hook: each page's mbarrier expects stall_tx_bytes more
@@ -986,6 +992,166 @@ __device__ __forceinline__ void merge_slots(const float* ws_o, const float* ws_m
     }
 }
 
+// Shared-prefix units: a CTA streams one partition of one kv head's prefix
+// pages once, through one ring of W * stages page buffers shared by its W
+// warps, and warp w keeps the running state of 16-row group cg * W + w of
+// that kv head's query rows -- so the pages are read once for W groups
+// instead of once per group.  Warp 0 issues every page's copies; a buffer is
+// refilled once every active warp has released it (an "empty" mbarrier with
+// one arrival per active warp, beside the "full" one the copies complete),
+// and a word per buffer tells the warps which of its pages had a legal block
+// id (written before the "full" arrival, so its completion publishes it).
+// Each warp then writes its rows' partials (slot `part`) itself.  Every wait
+// is bounded; one that gives up stops the warp, and warp 0 lets the copies it
+// issued land before the CTA can exit.
+template <class WS, int D, int B, bool FP8, bool PAIR, int W>
+__device__ __forceinline__ void prefix_shared_ring(const DecodeParams& p, uint32_t sbase,
+                                                   uint32_t bars, int kvh, int cg, int part) {
+    constexpr int PAGE = D * B * (FP8 ? 1 : 2);
+    constexpr int NPG = PAIR ? 2 : 1;
+    constexpr int STAGE = 2 * PAGE * NPG;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nsh = W * p.stages;  // shared page buffers
+    const uint32_t full0 = bars, empty0 = bars + 8 * nsh, flags0 = bars + 16 * nsh;
+    const int n_active = min(W, p.prefix_groups - cg * W);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < nsh; ++i) {
+            mbar_init(full0 + 8 * i, 1);
+            mbar_init(empty0 + 8 * i, n_active);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const int rg = cg * W + warp;
+    if (rg >= p.prefix_groups) return;  // no group for this warp (issues nothing)
+
+    const int j0 = part * p.PP;
+    const int j1 = min(p.prefix_pages, j0 + p.PP);
+    const int span = (j1 - j0 + NPG - 1) / NPG;  // stages of this partition
+    const int rows_total = p.S * p.G;
+    auto row_of = [&](int lr) -> long long {
+        const int gi = rg * 16 + lr;
+        if (gi >= rows_total) return -1;
+        return (long long)(gi / p.G) * p.Hq + (long long)kvh * p.G + gi % p.G;
+    };
+    // Warp 0's block-table window: lane l holds stage (wbase + l)'s page.
+    const int32_t* btrow = p.bt;  // the prefix is row 0's first blocks
+    auto load_win = [&](int base, int off) -> int {
+        const int j = j0 + NPG * (base + lane) + off;
+        return j < j1 ? __ldg(btrow + j) : -1;
+    };
+    int win_a = -1, win_b = -1, win_a2 = -1, win_b2 = -1, wbase = 0;
+    if (warp == 0) {
+        win_a = load_win(0, 0);
+        win_b = load_win(32, 0);
+        if constexpr (PAIR) {
+            win_a2 = load_win(0, 1);
+            win_b2 = load_win(32, 1);
+        }
+    }
+    WS wa(lane);
+    wa.fetch_query(p.q, row_of);
+    float k_scale = 1.f, v_scale = 1.f;
+    if constexpr (FP8) {
+        k_scale = __ldg(p.k_scale);
+        v_scale = __ldg(p.v_scale);
+    }
+    wa.set_alibi(nullptr, p.Hq, row_of);
+    const size_t head_off = static_cast<size_t>(kvh) * PAGE;
+    const size_t block_stride = static_cast<size_t>(p.Hk) * PAGE;
+    // Copies of stage i (warp 0 only, stages in increasing order).
+    auto issue = [&](int i) {
+        if (i >= wbase + 32) {
+            win_a = win_b;
+            win_b = load_win(wbase + 64, 0);
+            if constexpr (PAIR) {
+                win_a2 = win_b2;
+                win_b2 = load_win(wbase + 64, 1);
+            }
+            wbase += 32;
+        }
+        const int pb = __shfl_sync(kFull, win_a, i & 31);
+        const int pb2 = PAIR ? __shfl_sync(kFull, win_a2, i & 31) : -1;
+        const int st = i % nsh;
+        const uint32_t bar = full0 + 8 * st;
+        const bool ok = pb >= 0 && static_cast<long long>(pb) < p.num_blocks;
+        const bool has2 = PAIR && j0 + NPG * i + 1 < j1;
+        const bool ok2 = has2 && pb2 >= 0 && static_cast<long long>(pb2) < p.num_blocks;
+        if (lane == 0) {
+            sts32(flags0 + 4 * st, (ok ? 1u : 0u) | (ok2 ? 2u : 0u));
+            const uint32_t bytes = (ok ? 2 * PAGE : 0) + (ok2 ? 2 * PAGE : 0);
+            const uint32_t dst = sbase + static_cast<uint32_t>(st * STAGE);
+            if (bytes) {
+                mbar_arrive_expect_tx(bar, bytes + p.stall_tx_bytes);
+                if (ok) {
+                    const size_t off = static_cast<size_t>(pb) * block_stride + head_off;
+                    bulk_copy_g2s(dst, p.kc + off, PAGE, bar);
+                    bulk_copy_g2s(dst + NPG * PAGE, p.vc + off, PAGE, bar);
+                }
+                if (ok2) {
+                    const size_t off = static_cast<size_t>(pb2) * block_stride + head_off;
+                    bulk_copy_g2s(dst + PAGE, p.kc + off, PAGE, bar);
+                    bulk_copy_g2s(dst + 3 * PAGE, p.vc + off, PAGE, bar);
+                }
+            } else {
+                mbar_arrive(bar);
+            }
+            if (!ok || (has2 && !ok2)) atomicOr(p.status, kDevBadBlock);
+        }
+    };
+    int issued = 0;
+    if (warp == 0) {
+        for (; issued < min(span, nsh); ++issued) issue(issued);
+    }
+    wa.finish_query(p.scale_log2, k_scale, v_scale);
+    wa.reset();
+
+    bool timed_out = false;
+    int k = 0;
+    for (; k < span; ++k) {
+        const int st = k % nsh;
+        const uint32_t ph = static_cast<uint32_t>(k / nsh) & 1u;
+        if (!__all_sync(kFull, mbar_wait_bounded(full0 + 8 * st, ph, p.wait_limit_ns))) {
+            timed_out = true;
+            break;
+        }
+        // Prefix pages are whole blocks: every slot of a legal page is a token
+        // (a stage past the partition's last pair holds one page).
+        const uint32_t fl = lds32(flags0 + 4 * st);
+        const int valid = (fl & 1u) ? B : 0;
+        const int valid2 = (fl & 2u) ? B : 0;
+        const uint32_t kb = sbase + static_cast<uint32_t>(st * STAGE);
+        if (valid == B && (!PAIR || valid2 == B))
+            wa.template page<true, false>(kb, B, B, 0);
+        else
+            wa.template page<false, false>(kb, valid, valid2, 0);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8 * st);
+        if (warp == 0 && issued < span) {
+            // Buffer st is free once every active warp has released stage k.
+            if (!__all_sync(kFull, mbar_wait_bounded(empty0 + 8 * st, ph, p.wait_limit_ns))) {
+                timed_out = true;
+                ++k;  // stage k was consumed
+                break;
+            }
+            issue(issued++);
+        }
+    }
+    if (timed_out) {
+        if (warp == 0) {
+            // Let every copy issued and not yet seen land (bounded) before the
+            // CTA's shared memory can be handed to anyone else.
+            for (int i = k; i < issued; ++i)
+                (void)mbar_wait_bounded(full0 + 8 * (i % nsh),
+                                        static_cast<uint32_t>(i / nsh) & 1u, p.wait_limit_ns);
+        }
+        if (lane == 0) atomicOr(p.status, kDevTimeout);
+    }
+    const int rows_here = min(16, rows_total - rg * 16);
+    wa.write_partial(p.ws_o, p.ws_m, p.ws_l, rows_here,
+                     [&](int h) { return row_of(h) * p.P_total + part; }, timed_out);
+}
+
 // The paired 8-row form with f16 MMAs is held to three CTAs per SM (170
 // registers), the residency of the other 8-row forms.
 // SC: one query head per kv head on the CUDA cores (WarpAttnScalar).
@@ -1103,8 +1269,9 @@ __global__ void __launch_bounds__(W * 32,
         pre = unit < p.prefix_units;
         if (pre) {
             kvh = static_cast<int>(unit % p.Hk);
-            rg = static_cast<int>((unit / p.Hk) % p.prefix_groups);
-            part = static_cast<int>(unit / ((long long)p.Hk * p.prefix_groups));
+            // the row group (or, shared, the group of W row groups)
+            rg = static_cast<int>((unit / p.Hk) % p.prefix_cta_groups);
+            part = static_cast<int>(unit / ((long long)p.Hk * p.prefix_cta_groups));
             s = 0;
         } else {
             long long u = unit - p.prefix_units;
@@ -1159,6 +1326,13 @@ __global__ void __launch_bounds__(W * 32,
     // consumes all it issued).
     const int NS = p.stages;
     const uint32_t sbase = smem_addr(smem);
+    if constexpr (NH == 2 && !SC) {
+        if (pre && p.prefix_shared) {  // (barriers, page flags after the stage area)
+            const int area = max(W * NS * STAGE, merge_smem_bytes<D, NH, W>());
+            prefix_shared_ring<WA, D, B, FP8, PAIR, W>(p, sbase, sbase + area, kvh, rg, part);
+            return;
+        }
+    }
     const uint32_t wstage0 = sbase + static_cast<uint32_t>(warp * NS * STAGE);
     // mbarriers sit after the larger of the page stages and the merge buffer
     // that later overlays them (the host sizes shared memory the same way).

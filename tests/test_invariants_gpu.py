@@ -329,14 +329,18 @@ def test_bad_block_id_and_length_flags():
     assert pa.read_status(ws) == 0
 
 
+@pytest.mark.parametrize("nseq", [3, 17])
 @pytest.mark.parametrize("kv", [W.BF16, W.FP8_E4M3])
 @pytest.mark.parametrize("B", [16, 32])
-def test_one_hot_probe_bit_exact_with_shared_prefix(kv, B):
+def test_one_hot_probe_bit_exact_with_shared_prefix(kv, B, nseq):
     """Cascade decode: the probe token sits in the shared prefix (a shared
-    block, so every sequence sees it) or in a sequence's own pages."""
+    block, so every sequence sees it) or in a sequence's own pages.  With 3
+    sequences a kv head has one 16-row group (a prefix CTA per group); with
+    17, five (prefix CTAs whose warps share one page ring, the last CTA's
+    partly idle)."""
     pref = 5
-    lens = [pref * B + 3, pref * B, 9 * B + 1]
-    cfg = W.PagedConfig(f"probe prefix B={B} {kv}", num_seqs=3, num_heads=8, num_kv_heads=2,
+    lens = ([pref * B + 3, pref * B, 9 * B + 1] * 6)[:nseq]
+    cfg = W.PagedConfig(f"probe prefix B={B} {kv}", num_seqs=nseq, num_heads=8, num_kv_heads=2,
                         head_size=128, block_size=B,
                         num_blocks=pref + sum(-(-t // B) - pref for t in lens) + 6,
                         seq_len_lo=1, seq_len_hi=max(lens), kv_dtype=kv,
@@ -353,10 +357,11 @@ def test_one_hot_probe_bit_exact_with_shared_prefix(kv, B):
     q[:, :, 0] = 4096.0
     wl.query = q
     one = 1.0 if kv == W.BF16 else 0x7E
-    ws = torch.zeros(pa.workspace_size(3, 8, 2, 128, B, max(lens), kv, 2,
+    ws = torch.zeros(pa.workspace_size(nseq, 8, 2, 128, B, max(lens), kv, 2,
                                        shared_prefix_blocks=pref), dtype=torch.uint8, device=DEV)
     out = torch.empty_like(wl.query)
-    for t_star, seqs in [(0, [0, 1, 2]), (pref * B - 1, [0, 1, 2]), (2 * B + 3, [0, 1, 2]),
+    every = list(range(nseq))
+    for t_star, seqs in [(0, every), (pref * B - 1, every), (2 * B + 3, every),
                          (pref * B + 2, [0]), (9 * B, [2])]:
         marks = []
         for s in seqs:
@@ -399,3 +404,28 @@ def test_wait_give_up_path_sets_status_and_leaves_context_usable():
     torch.cuda.synchronize()
     assert pa.read_status(ws) == 0
     compare(good, run_oracle(wl), cfg.kv_dtype, "after a give-up")
+
+
+def test_wait_give_up_path_with_a_shared_prefix():
+    """The prefix units' shared page ring under test_stall_copies: its waits
+    give up too, the call ends with PA_DEV_WAIT_TIMEOUT and a finite output,
+    and a normal call afterwards is correct."""
+    lens = [700, 650, 900, 520, 610]
+    cfg = _cfg(lens=lens, G=4, Hk=2, seed=515).replace(shared_prefix_blocks=20)
+    wl = W.make_workload(cfg, DEV, seq_lens=lens)
+    c = wl.cfg
+    ws = torch.zeros(pa.workspace_size(c.num_seqs, c.num_heads, c.num_kv_heads, c.head_size,
+                                       c.block_size, c.max_seq_len, c.kv_dtype,
+                                       shared_prefix_blocks=20), dtype=torch.uint8, device=DEV)
+    out = torch.full_like(wl.query, float("nan"))
+    pa.decode(out, wl.query, wl.key_cache, wl.value_cache, c.num_kv_heads, c.scale,
+              wl.block_tables, wl.seq_lens, c.block_size, c.max_seq_len, c.kv_dtype,
+              wl.k_scale, wl.v_scale, workspace_tensor=ws, shared_prefix_blocks=20,
+              test_stall_copies=True)
+    torch.cuda.synchronize()
+    assert pa.read_status(ws, clear=True) & pa.PA_DEV_WAIT_TIMEOUT
+    assert torch.isfinite(out.float()).all()
+    good = run_gpu(wl, ws=ws, shared_prefix_blocks=20)
+    torch.cuda.synchronize()
+    assert pa.read_status(ws) == 0
+    compare(good, run_oracle(wl), c.kv_dtype, "prefix after a give-up")

@@ -209,6 +209,18 @@ PREFIX_CASES = {
                                  head_size=64, block_size=16, num_blocks=12 + 11 * 60 + 8,
                                  seq_len_lo=200, seq_len_hi=950, shared_prefix_blocks=12,
                                  seed=33),
+    # at least as many 16-row groups per kv head as warps per CTA: the prefix
+    # CTAs' warps share one page ring (4 groups on 4 warps; 5 groups, the last
+    # CTA with one)
+    "b16_bf16_g8_ring": W.PagedConfig("prefix G=8, shared ring", num_seqs=8, num_heads=16,
+                                      num_kv_heads=2, head_size=128, block_size=16,
+                                      num_blocks=37 + 8 * 70 + 8, seq_len_lo=600,
+                                      seq_len_hi=1100, shared_prefix_blocks=37, seed=34),
+    "b16_fp8_g8_ring": W.PagedConfig("prefix G=8 e4m3, shared ring", num_seqs=9, num_heads=16,
+                                     num_kv_heads=2, head_size=128, block_size=16,
+                                     num_blocks=21 + 9 * 60 + 8, seq_len_lo=400,
+                                     seq_len_hi=950, shared_prefix_blocks=21,
+                                     kv_dtype=W.FP8_E4M3, k_scale=0.05, v_scale=0.05, seed=35),
 }
 
 
