@@ -131,7 +131,9 @@ typedef enum pa_kv_dtype {
  *      PA_SCHEDULE_PARTITIONED: one CTA per (sequence, kv head, partition), as
  *      many waves as that takes; the hardware hands units to SMs as they free
  *      up.  Under PA_SCHEDULE_AUTO, when units are not split and fill two or
- *      three waves of CTA slots, the units of the last, partial wave are cut
+ *      three waves of CTA slots (or more, for pages that go in pairs: e4m3
+ *      pages of 16 tokens, bf16 ones of head size 64), the units of the last,
+ *      partial wave are cut
  *      into partitions whose CTAs follow every whole unit's (the split tail,
  *      pa_plan.tail_units); PA_SCHEDULE_PARTITIONED leaves them whole.
  *      PA_SCHEDULE_BALANCED: one wave of CTAs (grid_ctas = resident CTA

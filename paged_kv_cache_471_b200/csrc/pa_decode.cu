@@ -285,17 +285,18 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         P = (pages_max - prefix + pp - 1) / pp;
         groups = (static_cast<long long>(num_seqs) * (num_heads / num_kv_heads) + 15) / 16;
     }
-    // Split tail: with whole units in two or three waves, the units of the
+    // Split tail: with whole units in two or more waves, the units of the
     // last, partial wave (units mod CTA slots) are cut into kTailParts
     // partitions each, dispatched after every whole unit, so that the call
-    // does not end on a few full-length units streaming alone (measured on
-    // B200: +2.4% to +4.0% on equal-length batches of 1024 units; -0.2% to
-    // -0.35% when the last units are the short ones of mixed lengths; from four
-    // waves up the last wave is a small enough share that the gains and losses
-    // even out, so it is not split there).
+    // does not end on a few full-length units streaming alone.  Measured on
+    // B200: in two or three waves, +2.4% to +4.0% on equal-length batches of
+    // 1024 units and -0.2% to -0.35% when the last units are the short ones of
+    // mixed lengths; from four waves up, +0.65% to +2.5% on batches of paired
+    // pages (e4m3 pages of 16 tokens, bf16 pages of head size 64) and -1.1% to
+    // +0.05% on the others, so there only paired pages are split.
     long long tail_units = 0;
     int tail_P = 0, tail_PP = 0;
-    if (whole_units && !cascade && schedule == PA_SCHEDULE_AUTO && units < 4 * slots) {
+    if (whole_units && !cascade && schedule == PA_SCHEDULE_AUTO && (units < 4 * slots || pair)) {
         const long long r = units % slots;
         const long long tpp = (pages_max + kTailParts - 1) / kTailParts;
         if (r > 0 && r <= kMergeCounts && tpp >= kMinPartitionPages) {

@@ -104,10 +104,11 @@ def test_workspace_size_header_only_without_split():
 
 
 def test_split_tail_plan_and_workspace():
-    """Whole units in two or three waves: the last wave's units (units mod CTA
-    slots) are cut into 4 partitions whose CTAs follow the whole units; the
-    workspace holds, after the header and the split-tail counts, their
-    partials ((D + 2) floats per row and partition), 256-byte aligned."""
+    """Whole units in two or three waves (or more, for paired pages): the
+    last wave's units (units mod CTA slots) are cut into 4 partitions whose
+    CTAs follow the whole units; the workspace holds, after the header and the
+    split-tail counts, their partials ((D + 2) floats per row and partition),
+    256-byte aligned."""
     S, Hq, Hk, D, B, T = 32, 32, 32, 128, 16, 8192
     p = pa.plan(S, Hq, Hk, D, B, T, "bf16", num_sms=148)
     units, slots = S * Hk, 3 * 148
@@ -141,6 +142,10 @@ def test_split_tail_only_where_it_applies():
                    **base)["tail_units"] == 0
     assert pa.plan(16, 32, 32, 128, 16, 4096, "bf16", **base)["tail_units"] == 0
     assert pa.plan(64, 32, 32, 128, 16, 4096, "bf16", **base)["tail_units"] == 0  # 4.6 waves
+    # ... but pages that go in pairs are split from four waves up too
+    assert pa.plan(64, 32, 32, 64, 16, 4096, "bf16", **base)["tail_units"] == 2048 % 444
+    assert pa.plan(256, 32, 8, 128, 16, 16384, "fp8_e4m3", **base)["tail_units"] == 2048 % 444
+    assert pa.plan(256, 32, 8, 128, 32, 16384, "fp8_e4m3", **base)["tail_units"] == 0
     assert pa.plan(111, 12, 3, 128, 16, 4096, "bf16", num_sms=37)["tail_units"] == 0  # 3 x 111
     # tail partitions of fewer than 16 pages are not made
     assert pa.plan(32, 32, 32, 128, 16, 960, "bf16", **base)["tail_units"] == 0
@@ -197,11 +202,13 @@ def test_planner_on_the_five_workloads():
     p1, p2, p3, p4, p5 = (_plan(i) for i in range(1, 6))
     assert all(p["balanced"] == 0 for p in (p1, p2, p3, p4, p5))
     assert p1["num_partitions"] == 1 and p1["partition_pages"] == 16
-    # whole units; in two or three waves, the last wave's units in 4 partitions
+    # whole units; in two or three waves (or more, for paired pages) the last
+    # wave's units in 4 partitions
     assert p2["num_partitions"] == 1 and p2["grid_ctas"] == 64 * 32 and p2["tail_units"] == 0
     assert p3["num_partitions"] == 1  # two waves of units; longest-first order
     assert p3["tail_units"] == 128 * 8 % 444
-    assert p4["num_partitions"] == 1 and p4["grid_ctas"] == 256 * 8 and p4["tail_units"] == 0
+    assert p4["num_partitions"] == 1 and p4["tail_units"] == 256 * 8 % 444  # paired e4m3
+    assert p4["grid_ctas"] == 256 * 8 + 3 * p4["tail_units"]
     assert p1["tail_units"] == 0 and p5["tail_units"] == 0
     assert p5["num_partitions"] >= 4  # 64 (seq, kv head) units cannot fill 148 SMs
     # balanced ranges on request: one wave of CTAs

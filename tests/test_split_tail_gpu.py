@@ -116,11 +116,12 @@ def test_one_workspace_long_then_short():
         compare(out, run_oracle(wl), cfg.kv_dtype, f"split tail reuse {lens[:4]}")
 
 
-@pytest.mark.parametrize("idx", [3])
+@pytest.mark.parametrize("idx", [3, 4])
 def test_full_size_noalloc_matches_workspace_call(idx):
-    """The full GQA batch (1024 units) takes the split tail on this GPU; the
-    allocation-free entry point (same plan, scratch in the library's own
-    array) gives the same bits as a call with a caller workspace."""
+    """The full GQA batch (1024 units) and the FP8 batch (2048 units of paired
+    pages) take the split tail on this GPU; the allocation-free entry point
+    (same plan, scratch in the library's own array) gives the same bits as a
+    call with a caller workspace."""
     cfg = W.WORKLOADS[idx]
     p = pa.plan(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_size, cfg.block_size,
                 cfg.max_seq_len, cfg.kv_dtype)
