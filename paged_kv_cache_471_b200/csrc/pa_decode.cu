@@ -26,8 +26,10 @@ constexpr int kMaxRankedSeqs = 256;  // batches ranked by length on the device
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // a page copy's wait bound
 constexpr unsigned long long kTestWaitLimitNs = 20000000ull;  // with test_stall_copies
 constexpr long long kLongPartitionPages = 256;
-// Split tail: partitions per unit of the last, partial wave of whole units.
+// Split tail: partitions per unit of the last, partial wave of whole units
+// (at least; more when that wave has few units, up to kMaxTailParts).
 constexpr int kTailParts = 4;
+constexpr int kMaxTailParts = 16;
 // Workspace layout: the header (status word, dynamic-schedule words), then
 // the split tail's per-unit merge counts, which nothing else touches (they
 // are 0 between calls), then the plan's partials (or page scan, or unit
@@ -298,11 +300,16 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
     int tail_P = 0, tail_PP = 0;
     if (whole_units && !cascade && schedule == PA_SCHEDULE_AUTO && (units < 4 * slots || pair)) {
         const long long r = units % slots;
-        const long long tpp = (pages_max + kTailParts - 1) / kTailParts;
-        if (r > 0 && r <= kMergeCounts && tpp >= kMinPartitionPages) {
+        // Enough partitions that the tail's CTAs about fill the slots, at least
+        // kTailParts, at most kMaxTailParts, none under kMinPartitionPages.
+        long long tp = r > 0 ? (slots + r - 1) / r : 0;
+        if (tp < kTailParts) tp = kTailParts;
+        if (tp > kMaxTailParts) tp = kMaxTailParts;
+        while (tp > kTailParts && (pages_max + tp - 1) / tp < kMinPartitionPages) --tp;
+        if (r > 0 && r <= kMergeCounts && (pages_max + tp - 1) / tp >= kMinPartitionPages) {
             tail_units = r;
-            tail_P = kTailParts;
-            tail_PP = static_cast<int>(tpp);
+            tail_P = static_cast<int>(tp);
+            tail_PP = static_cast<int>((pages_max + tp - 1) / tp);
         }
     }
     // Short partitions: give each warp a buffer for every page it will read

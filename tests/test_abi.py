@@ -147,6 +147,12 @@ def test_split_tail_only_where_it_applies():
     assert pa.plan(256, 32, 8, 128, 16, 16384, "fp8_e4m3", **base)["tail_units"] == 2048 % 444
     assert pa.plan(256, 32, 8, 128, 32, 16384, "fp8_e4m3", **base)["tail_units"] == 0
     assert pa.plan(111, 12, 3, 128, 16, 4096, "bf16", num_sms=37)["tail_units"] == 0  # 3 x 111
+    # a small last wave gets more partitions (enough to about fill the slots,
+    # at most 16, none under 16 pages)
+    p = pa.plan(224, 32, 8, 128, 16, 16384, "fp8_e4m3", **base)
+    assert (p["tail_units"], p["tail_partitions"], p["tail_partition_pages"]) == (16, 16, 64)
+    p = pa.plan(224, 32, 8, 128, 16, 2048, "fp8_e4m3", **base)  # 128 pages: at most 8
+    assert (p["tail_units"], p["tail_partitions"], p["tail_partition_pages"]) == (16, 8, 16)
     # tail partitions of fewer than 16 pages are not made
     assert pa.plan(32, 32, 32, 128, 16, 960, "bf16", **base)["tail_units"] == 0
     assert pa.plan(32, 32, 32, 128, 16, 1024, "bf16", **base)["tail_units"] > 0

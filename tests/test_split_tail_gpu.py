@@ -252,3 +252,23 @@ def test_wait_give_up_path_with_a_tail():
     torch.cuda.synchronize()
     assert pa.read_status(ws) == 0
     compare(good, run_oracle(wl), cfg.kv_dtype, "split tail after a give-up")
+
+
+def test_small_last_wave_gets_more_partitions():
+    """A last wave of few units is cut into more partitions (up to 16), so
+    that the tail's CTAs about fill the CTA slots; a row then merges up to 16
+    partials."""
+    T = 256 * 16
+    lens = [T, T - 7, 3000, T, 0, 1, 17 * 16 + 3, T] * 5
+    cfg = _mixed(16, lens, seed=808)
+    sms = 26  # 78 slots; 160 units -> 4 in the tail
+    p = _plan(cfg, sms)
+    assert p["tail_units"] == 4 and p["tail_partitions"] == 16, p
+    wl = W.make_workload(cfg, DEV, seq_lens=lens)
+    ws = _ws(cfg, sms)
+    out = torch.full_like(wl.query, float("nan"))
+    run_gpu(wl, out=out, ws=ws, num_sms=sms)
+    torch.cuda.synchronize()
+    assert pa.read_status(ws) == 0
+    assert not _tail_counts(ws).any()
+    compare(out, run_oracle(wl), cfg.kv_dtype, "split tail, 16 partitions")
