@@ -245,6 +245,21 @@ def test_planner_splits_between_one_and_two_waves():
     assert q["grid_ctas"] == 1024 and p["grid_ctas"] == 1024 + 3 * p["tail_units"]
 
 
+def test_split_count_fills_the_last_wave():
+    """Split plans take a partition count whose last wave of CTAs is about
+    62% full (55-70% measured best), among half to twice the count long
+    partitions would give."""
+    slots = 3 * 148
+    for args, kw in [((8, 32, 8, 128, 32, 131072), dict(shared_prefix_blocks=1024)),
+                     ((8, 32, 8, 128, 32, 131072), {}),
+                     ((8, 32, 8, 128, 16, 131072), {}),
+                     ((16, 32, 8, 128, 16, 16384), {})]:
+        p = pa.plan(*args, "bf16", num_sms=148, **kw)
+        w = p["grid_ctas"] / slots
+        assert p["num_partitions"] > 1 and w >= 1.4, (args, p)
+        assert 0.5 <= w - int(w) <= 0.75, (args, p, w)
+
+
 def test_balanced_schedule_limits():
     # forced partitions or a shared prefix rule balanced ranges out
     with pytest.raises(pa.PagedAttentionError):
