@@ -278,10 +278,11 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         // partitions (none under kMinPartitionPages, at least 1.4 waves), the
         // count whose last wave is nearest 62% full, a partition more or
         // less counting as 1%.
-        const long long cta_groups_est =
-            cascade ? ((static_cast<long long>(num_seqs) * (num_heads / num_kv_heads) + 15) / 16 +
-                       W - 1) / W
-                    : 0;
+        // Prefix CTAs per kv head and prefix partition, as counted below: W row
+        // groups per CTA with a shared ring (at least W groups), else one each.
+        const long long groups_est =
+            cascade ? (static_cast<long long>(num_seqs) * (num_heads / num_kv_heads) + 15) / 16 : 0;
+        const long long cta_groups_est = groups_est >= W ? (groups_est + W - 1) / W : groups_est;
         auto grid_for = [&](long long n) {
             const long long q = (pages_max + n - 1) / n;
             if (!cascade) return units * ((pages_max + q - 1) / q);
