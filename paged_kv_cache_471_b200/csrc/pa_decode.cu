@@ -26,6 +26,9 @@ constexpr int kMaxRankedSeqs = 256;  // batches ranked by length on the device
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // a page copy's wait bound
 constexpr unsigned long long kTestWaitLimitNs = 20000000ull;  // with test_stall_copies
 constexpr long long kLongPartitionPages = 256;
+// Partials per query row that the combine kernel merges with one batch of
+// loads (a slot per lane); split plans keep to it where they can.
+constexpr long long kOneRoundSlots = 32;
 // Split tail: partitions per unit of the last, partial wave of whole units
 // (at least; more when that wave has few units, up to kMaxTailParts).
 constexpr int kTailParts = 4;
@@ -275,9 +278,15 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         // last wave of CTAs is about 55-70% full streamed best, and one that
         // spills a few CTAs into a new wave, or fills its last wave to 80% or
         // more, 2-16% worse.  So take, among half to twice that many
-        // partitions (none under kMinPartitionPages, at least 1.4 waves), the
-        // count whose last wave is nearest 62% full, a partition more or
-        // less counting as 1%.
+        // partitions (none under kMinPartitionPages, at least 1.4 waves, at
+        // most kOneRoundSlots partials per row), the count whose last wave is
+        // nearest 62% full, a partition more or less counting as 1%.  Batches
+        // of so few units that no such grid exists (one or two long
+        // sequences) take one partial wave instead, nearest 75% full.
+        // Measured on B200 (8 kv heads), against the same rule without the
+        // partials limit: 1 x 32768 tokens +45%, 2 x 32768 +20%, 1 and 2 x
+        // 131072 with a shared prefix +24% and +4.5%, 4 and 6 x 131072 +3.1%
+        // and +2.5%, 3 x 131072 with a prefix -1.1%.
         // Prefix CTAs per kv head and prefix partition, as counted below: W row
         // groups per CTA with a shared ring (at least W groups), else one each.
         const long long groups_est =
@@ -289,8 +298,13 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
             return units * ((pages_max - prefix + q - 1) / q) +
                    num_kv_heads * cta_groups_est * ((prefix + q - 1) / q);
         };
-        long long best = np;
-        double best_score = -1.0;
+        auto row_slots = [&](long long n) {  // partials per query row
+            const long long q = (pages_max + n - 1) / n;
+            if (!cascade) return (pages_max + q - 1) / q;
+            return (pages_max - prefix + q - 1) / q + (prefix + q - 1) / q;
+        };
+        long long best = np, best_any = np;
+        double best_score = -1.0, any_score = -1.0;
         for (long long n = np / 2 > 1 ? np / 2 : 1; n <= 2 * np; ++n) {
             if ((pages_max + n - 1) / n < kMinPartitionPages) break;
             const double w = static_cast<double>(grid_for(n)) / static_cast<double>(slots);
@@ -298,9 +312,32 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
             const double f = w - static_cast<double>(static_cast<long long>(w));
             const double score = (f > 0.62 ? f - 0.62 : 0.62 - f) +
                                  0.01 * static_cast<double>(n > np ? n - np : np - n);
-            if (best_score < 0.0 || score < best_score) {
+            if (any_score < 0.0 || score < any_score) {
+                best_any = n;
+                any_score = score;
+            }
+            if (row_slots(n) <= kOneRoundSlots && (best_score < 0.0 || score < best_score)) {
                 best = n;
                 best_score = score;
+            }
+        }
+        if (best_score < 0.0) {
+            // One partial wave of at least half the CTA slots (the grid grows
+            // with n), else the multi-wave count without the partials limit
+            // (batches of a handful of units, where one wave at that limit
+            // would leave most of the GPU idle).
+            best = best_any;
+            double best1 = -1.0;
+            for (long long n = 1;; ++n) {
+                if (n > 1 && (pages_max + n - 1) / n < kMinPartitionPages) break;
+                const double w = static_cast<double>(grid_for(n)) / static_cast<double>(slots);
+                if (w >= 1.0 || row_slots(n) > kOneRoundSlots) break;
+                if (w < 0.5) continue;
+                const double score = w > 0.75 ? w - 0.75 : 0.75 - w;
+                if (best1 < 0.0 || score < best1) {
+                    best = n;
+                    best1 = score;
+                }
             }
         }
         np = best;

@@ -260,6 +260,31 @@ def test_split_count_fills_the_last_wave():
         assert 0.5 <= w - int(w) <= 0.75, (args, p, w)
 
 
+def test_split_plans_keep_to_one_combine_round():
+    """At most 32 partials per query row (one batch of loads in the combine)
+    where a grid of 1.4 waves or more allows it; batches too small for that
+    take one partial wave, at least half the CTA slots and nearest 75% full;
+    a handful of units falls back to the multi-wave count without the limit."""
+    slots = 3 * 148
+
+    def per_row(p):
+        return p["num_partitions"] + p["prefix_partitions"]
+
+    # multi-wave grids within the limit (4 and 6 x 131072 tokens, 8 kv heads)
+    for S in (4, 6):
+        p = pa.plan(S, 32, 8, 128, 16, 131072, "bf16", num_sms=148)
+        assert per_row(p) <= 32 and p["grid_ctas"] / slots >= 1.4, (S, p)
+    # one or two long sequences of 8 kv heads: one partial wave
+    for S, T, B, pre in ((1, 32768, 16, 0), (2, 32768, 16, 0), (1, 16384, 16, 0),
+                         (1, 131072, 32, 1024), (2, 131072, 32, 1024)):
+        p = pa.plan(S, 32, 8, 128, B, T, "bf16", num_sms=148, shared_prefix_blocks=pre)
+        w = p["grid_ctas"] / slots
+        assert per_row(p) <= 32 and 0.5 <= w < 1.0, (S, T, p, w)
+    # one kv head: 32 partials would fill 7% of the GPU, so the limit is dropped
+    p = pa.plan(1, 4, 1, 128, 16, 131072, "bf16", num_sms=148)
+    assert per_row(p) > 32 and p["grid_ctas"] / slots > 0.5, p
+
+
 def test_balanced_schedule_limits():
     # forced partitions or a shared prefix rule balanced ranges out
     with pytest.raises(pa.PagedAttentionError):

@@ -95,17 +95,21 @@ def test_e4m3_code_ranges(f8c, scales, what):
 
 def test_half_million_token_sequence():
     """One sequence of 2^19 tokens beside a short one (8 kv heads, block size
-    32, bf16): the planner splits the long sequence into many partitions and
-    the combine merges them.  Every row against the oracle."""
+    32, bf16): the planner splits the long sequence into many partitions (up
+    to the 32 the combine merges in one batch of loads), and a forced partition
+    size splits it into 64; the combine merges them.  Every row against the
+    oracle, both ways."""
     lens = [1 << 19, 1000]
     wl = _workload(W.BF16, seed=504, D=128, B=32, G=4, Hk=8, lens=lens)
     c = wl.cfg
     p = pa.plan(c.num_seqs, c.num_heads, c.num_kv_heads, c.head_size, c.block_size,
                 c.max_seq_len, c.kv_dtype)
-    assert p["num_partitions"] >= 32
-    out = _decode(wl)
-    assert torch.isfinite(out.float()).all()
-    compare(out, run_oracle_all(wl), W.BF16, "2^19-token sequence all rows", full_size=True)
-    assert pa.read_status(device=DEV) == 0
+    assert 16 <= p["num_partitions"] <= 32, p
+    ref = run_oracle_all(wl)
+    for pp, what in ((0, "planned"), (256, "64 partitions")):
+        out = _decode(wl, partition_pages=pp)
+        assert torch.isfinite(out.float()).all()
+        compare(out, ref, W.BF16, f"2^19-token sequence all rows, {what}", full_size=True)
+        assert pa.read_status(device=DEV) == 0
     del wl, out
     torch.cuda.empty_cache()

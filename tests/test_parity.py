@@ -173,6 +173,34 @@ def test_full_size_all_rows(idx):
     torch.cuda.empty_cache()
 
 
+SMALL_LONG = {
+    "1 x 32768, B=16": W.PagedConfig("1 x 32768", num_seqs=1, num_heads=32, num_kv_heads=8,
+                                     head_size=128, block_size=16, num_blocks=2048 + 40,
+                                     seq_len_lo=32768, seq_len_hi=32768, seed=501),
+    "2 x 32768, B=16, ragged": W.PagedConfig("2 x 32768", num_seqs=2, num_heads=32,
+                                             num_kv_heads=8, head_size=128, block_size=16,
+                                             num_blocks=2 * 2048 + 40, seq_len_lo=20001,
+                                             seq_len_hi=32768, seed=502),
+    "2 x 131072, B=32, shared prefix": W.reduced(5, num_seqs=2),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SMALL_LONG))
+def test_small_long_context_batches_all_rows(name):
+    """One or two long sequences: the planner takes one partial wave of CTAs
+    with at most 32 partials per row; every row against the oracle."""
+    cfg = SMALL_LONG[name]
+    plan = pa.plan(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_size,
+                   cfg.block_size, cfg.max_seq_len, cfg.kv_dtype,
+                   shared_prefix_blocks=cfg.shared_prefix_blocks)
+    assert plan["num_partitions"] + plan["prefix_partitions"] <= 32, plan
+    wl = W.make_workload(cfg, DEV)
+    out = run_gpu(wl, shared_prefix_blocks=cfg.shared_prefix_blocks)
+    torch.cuda.synchronize()
+    assert pa.read_status(device=DEV) == 0
+    compare(out, run_oracle(wl), cfg.kv_dtype, f"{name} all rows", full_size=True)
+
+
 def test_full_size_cfg5_without_prefix_declaration():
     """Config 5 decoded as plain per-sequence units (the shared prefix not
     declared: every sequence streams its own copy of the prefix pages)."""
