@@ -292,16 +292,25 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         const long long groups_est =
             cascade ? (static_cast<long long>(num_seqs) * (num_heads / num_kv_heads) + 15) / 16 : 0;
         const long long cta_groups_est = groups_est >= W ? (groups_est + W - 1) / W : groups_est;
-        auto grid_for = [&](long long n) {
+        // Partition size for about n partitions of max_seq_len, evened out
+        // over the pages each sequence splits (its own pages, after a shared
+        // prefix) so that no partition is left much shorter than the others.
+        const long long own = cascade ? pages_max - prefix : pages_max;
+        auto part_pages = [&](long long n) {
             const long long q = (pages_max + n - 1) / n;
+            const long long parts = (own + q - 1) / q;
+            return parts > 0 ? (own + parts - 1) / parts : q;
+        };
+        auto grid_for = [&](long long n) {
+            const long long q = part_pages(n);
             if (!cascade) return units * ((pages_max + q - 1) / q);
-            return units * ((pages_max - prefix + q - 1) / q) +
+            return units * ((own + q - 1) / q) +
                    num_kv_heads * cta_groups_est * ((prefix + q - 1) / q);
         };
         auto row_slots = [&](long long n) {  // partials per query row
-            const long long q = (pages_max + n - 1) / n;
+            const long long q = part_pages(n);
             if (!cascade) return (pages_max + q - 1) / q;
-            return (pages_max - prefix + q - 1) / q + (prefix + q - 1) / q;
+            return (own + q - 1) / q + (prefix + q - 1) / q;
         };
         long long best = np, best_any = np;
         double best_score = -1.0, any_score = -1.0;
@@ -341,7 +350,7 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
             }
         }
         np = best;
-        pp = (pages_max + np - 1) / np;
+        pp = part_pages(np);
     }
     if (pp < 1) pp = 1;
     long long P = pages_max > 0 ? (pages_max + pp - 1) / pp : 1;
