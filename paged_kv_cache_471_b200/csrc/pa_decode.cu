@@ -285,7 +285,7 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         // sequences) take one partial wave instead, nearest 75% full.
         // Measured on B200 (8 kv heads), against the same rule without the
         // partials limit: 1 x 32768 tokens +45%, 2 x 32768 +20%, 1 and 2 x
-        // 131072 with a shared prefix +24% and +4.5%, 4 and 6 x 131072 +3.1%
+        // 131072 with a shared prefix +24% and +7%, 4 and 6 x 131072 +3.1%
         // and +2.5%, 3 x 131072 with a prefix -1.1%.
         // Prefix CTAs per kv head and prefix partition, as counted below: W row
         // groups per CTA with a shared ring (at least W groups), else one each.
