@@ -29,6 +29,9 @@ constexpr long long kLongPartitionPages = 256;
 // Partials per query row that the combine kernel merges with one batch of
 // loads (a slot per lane); split plans keep to it where they can.
 constexpr long long kOneRoundSlots = 32;
+// CTAs of a split plan for a batch of only a handful of (sequence, kv head)
+// units, where one partial wave within kOneRoundSlots would stay small.
+constexpr long long kFewUnitCtas = 128;
 // Split tail: partitions per unit of the last, partial wave of whole units
 // (at least; more when that wave has few units, up to kMaxTailParts).
 constexpr int kTailParts = 4;
@@ -332,9 +335,7 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         }
         if (best_score < 0.0) {
             // One partial wave of at least half the CTA slots (the grid grows
-            // with n), else the multi-wave count without the partials limit
-            // (batches of a handful of units, where one wave at that limit
-            // would leave most of the GPU idle).
+            // with n).
             best = best_any;
             double best1 = -1.0;
             for (long long n = 1;; ++n) {
@@ -346,6 +347,23 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
                 if (best1 < 0.0 || score < best1) {
                     best = n;
                     best1 = score;
+                }
+            }
+            if (best1 < 0.0) {
+                // A handful of units (fewer than 7 on 148 SMs): about
+                // kFewUnitCtas CTAs, with up to max(32, kFewUnitCtas / units)
+                // partials per row.  Measured on B200 with 1, 2 and 4 units of
+                // 32768-131072 tokens: grids of 64-128 CTAs streamed 1.5-2.6x
+                // faster than 432-632 CTAs of 108-432 partials per row, whose
+                // merge takes several rounds of loads.
+                const long long cap_slots =
+                    (kFewUnitCtas + units - 1) / units > kOneRoundSlots
+                        ? (kFewUnitCtas + units - 1) / units
+                        : kOneRoundSlots;
+                for (long long n = 1;; ++n) {
+                    if (n > 1 && (pages_max + n - 1) / n < kMinPartitionPages) break;
+                    if (row_slots(n) > cap_slots) break;
+                    best = n;
                 }
             }
         }

@@ -264,7 +264,8 @@ def test_split_plans_keep_to_one_combine_round():
     """At most 32 partials per query row (one batch of loads in the combine)
     where a grid of 1.4 waves or more allows it; batches too small for that
     take one partial wave, at least half the CTA slots and nearest 75% full;
-    a handful of units falls back to the multi-wave count without the limit."""
+    a handful of units (too few for half a wave within the limit) takes about
+    128 CTAs, with up to max(32, 128 / units) partials per row."""
     slots = 3 * 148
 
     def per_row(p):
@@ -280,9 +281,10 @@ def test_split_plans_keep_to_one_combine_round():
         p = pa.plan(S, 32, 8, 128, B, T, "bf16", num_sms=148, shared_prefix_blocks=pre)
         w = p["grid_ctas"] / slots
         assert per_row(p) <= 32 and 0.5 <= w < 1.0, (S, T, p, w)
-    # one kv head: 32 partials would fill 7% of the GPU, so the limit is dropped
-    p = pa.plan(1, 4, 1, 128, 16, 131072, "bf16", num_sms=148)
-    assert per_row(p) > 32 and p["grid_ctas"] / slots > 0.5, p
+    # 1, 2 and 4 units of one long sequence: 128 CTAs
+    for Hk, rows in ((1, 128), (2, 64), (4, 32)):
+        p = pa.plan(1, 8 * Hk, Hk, 128, 16, 131072, "bf16", num_sms=148)
+        assert per_row(p) == rows and p["grid_ctas"] == 128, (Hk, p)
 
 
 def test_balanced_schedule_limits():
