@@ -287,6 +287,40 @@ def test_split_plans_keep_to_one_combine_round():
         assert per_row(p) == rows and p["grid_ctas"] == 128, (Hk, p)
 
 
+def test_split_plans_cover_every_page_over_many_shapes():
+    """Invariants of every split plan the planner picks, over a grid of batch
+    shapes: the partitions cover each sequence's own pages (after a shared
+    prefix) and the prefix, none of them is empty at max_seq_len, the sizes are
+    even (less than a page of slack per partition), the grid is the per-sequence CTAs plus the prefix CTAs, and the
+    partials per row stay within max(32, 128 / units)."""
+    n_split = 0
+    for S in (1, 2, 3, 5, 8, 13):
+        for Hk, G in ((1, 8), (2, 4), (4, 8), (8, 4), (32, 1)):
+            for B, T in ((16, 2048), (16, 32768), (32, 131072), (16, 100000)):
+                for pre_frac in (0, 4):
+                    pages = -(-T // B)
+                    prefix = pages // pre_frac if pre_frac else 0
+                    p = pa.plan(S, Hk * G, Hk, 128, B, T, "bf16", num_sms=148,
+                                shared_prefix_blocks=prefix)
+                    P, pp, ppre = p["num_partitions"], p["partition_pages"], p["prefix_partitions"]
+                    own = pages - prefix
+                    units = S * Hk
+                    if P <= 1 and not prefix:
+                        continue  # whole units (or the split tail, checked elsewhere)
+                    n_split += 1
+                    what = (S, Hk, G, B, T, prefix, p)
+                    assert P >= 1 and pp >= 1, what
+                    assert P * pp >= own and (P - 1) * pp < own, what  # covers, none empty
+                    assert P * pp - own < P, what  # even: under a page of slack per partition
+                    assert ppre * pp >= prefix and (ppre == 0 or (ppre - 1) * pp < prefix), what
+                    groups = -(-S * G // 16)
+                    W = p["warps_per_cta"]
+                    cta_groups = -(-groups // W) if groups >= W else groups
+                    assert p["grid_ctas"] == units * P + Hk * cta_groups * ppre, what
+                    assert P + ppre <= max(32, -(-128 // units)), what
+    assert n_split > 100
+
+
 def test_balanced_schedule_limits():
     # forced partitions or a shared prefix rule balanced ranges out
     with pytest.raises(pa.PagedAttentionError):
