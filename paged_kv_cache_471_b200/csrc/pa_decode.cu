@@ -315,8 +315,8 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
             if (!cascade) return (pages_max + q - 1) / q;
             return (own + q - 1) / q + (prefix + q - 1) / q;
         };
-        long long best = np, best_any = np;
-        double best_score = -1.0, any_score = -1.0;
+        long long best = np;
+        double best_score = -1.0;
         for (long long n = np / 2 > 1 ? np / 2 : 1; n <= 2 * np; ++n) {
             if ((pages_max + n - 1) / n < kMinPartitionPages) break;
             const double w = static_cast<double>(grid_for(n)) / static_cast<double>(slots);
@@ -324,10 +324,6 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
             const double f = w - static_cast<double>(static_cast<long long>(w));
             const double score = (f > 0.62 ? f - 0.62 : 0.62 - f) +
                                  0.01 * static_cast<double>(n > np ? n - np : np - n);
-            if (any_score < 0.0 || score < any_score) {
-                best_any = n;
-                any_score = score;
-            }
             if (row_slots(n) <= kOneRoundSlots && (best_score < 0.0 || score < best_score)) {
                 best = n;
                 best_score = score;
@@ -336,7 +332,6 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         if (best_score < 0.0) {
             // One partial wave of at least half the CTA slots (the grid grows
             // with n).
-            best = best_any;
             double best1 = -1.0;
             for (long long n = 1;; ++n) {
                 if (n > 1 && (pages_max + n - 1) / n < kMinPartitionPages) break;
