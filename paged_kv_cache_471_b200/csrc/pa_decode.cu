@@ -28,9 +28,9 @@ constexpr unsigned long long kTestWaitLimitNs = 20000000ull;  // with test_stall
 constexpr long long kLongPartitionPages = 256;
 // Partials per query row that the combine kernel merges with one batch of
 // loads (a slot per lane); split plans keep to it where they can.
-constexpr long long kOneRoundSlots = 32;
+constexpr long long kOneBatchSlots = 32;
 // CTAs of a split plan for a batch of only a handful of (sequence, kv head)
-// units, where one partial wave within kOneRoundSlots would stay small.
+// units, where one partial wave within kOneBatchSlots would stay small.
 constexpr long long kFewUnitCtas = 128;
 // Split tail: partitions per unit of the last, partial wave of whole units
 // (at least; more when that wave has few units, up to kMaxTailParts).
@@ -282,7 +282,7 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
         // spills a few CTAs into a new wave, or fills its last wave to 80% or
         // more, 2-16% worse.  So take, among half to twice that many
         // partitions (none under kMinPartitionPages, at least 1.4 waves, at
-        // most kOneRoundSlots partials per row), the count whose last wave is
+        // most kOneBatchSlots partials per row), the count whose last wave is
         // nearest 62% full, a partition more or less counting as 1%.  Batches
         // of so few units that no such grid exists (one or two long
         // sequences) take one partial wave instead, nearest 75% full.
@@ -324,7 +324,7 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
             const double f = w - static_cast<double>(static_cast<long long>(w));
             const double score = (f > 0.62 ? f - 0.62 : 0.62 - f) +
                                  0.01 * static_cast<double>(n > np ? n - np : np - n);
-            if (row_slots(n) <= kOneRoundSlots && (best_score < 0.0 || score < best_score)) {
+            if (row_slots(n) <= kOneBatchSlots && (best_score < 0.0 || score < best_score)) {
                 best = n;
                 best_score = score;
             }
@@ -336,7 +336,7 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
             for (long long n = 1;; ++n) {
                 if (n > 1 && (pages_max + n - 1) / n < kMinPartitionPages) break;
                 const double w = static_cast<double>(grid_for(n)) / static_cast<double>(slots);
-                if (w >= 1.0 || row_slots(n) > kOneRoundSlots) break;
+                if (w >= 1.0 || row_slots(n) > kOneBatchSlots) break;
                 if (w < 0.5) continue;
                 const double score = w > 0.75 ? w - 0.75 : 0.75 - w;
                 if (best1 < 0.0 || score < best1) {
@@ -350,11 +350,11 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
                 // partials per row.  Measured on B200 with 1, 2 and 4 units of
                 // 32768-131072 tokens: grids of 64-128 CTAs streamed 1.5-2.6x
                 // faster than 432-632 CTAs of 108-432 partials per row, whose
-                // merge takes several rounds of loads.
+                // merge takes several batches of loads.
                 const long long cap_slots =
-                    (kFewUnitCtas + units - 1) / units > kOneRoundSlots
+                    (kFewUnitCtas + units - 1) / units > kOneBatchSlots
                         ? (kFewUnitCtas + units - 1) / units
-                        : kOneRoundSlots;
+                        : kOneBatchSlots;
                 for (long long n = 1;; ++n) {
                     if (n > 1 && (pages_max + n - 1) / n < kMinPartitionPages) break;
                     if (row_slots(n) > cap_slots) break;

@@ -260,7 +260,7 @@ def test_split_count_fills_the_last_wave():
         assert 0.5 <= w - int(w) <= 0.75, (args, p, w)
 
 
-def test_split_plans_keep_to_one_combine_round():
+def test_split_plans_keep_to_one_combine_load_batch():
     """At most 32 partials per query row (one batch of loads in the combine)
     where a grid of 1.4 waves or more allows it; batches too small for that
     take one partial wave, at least half the CTA slots and nearest 75% full;
