@@ -182,18 +182,30 @@ SMALL_LONG = {
                                              num_blocks=2 * 2048 + 40, seq_len_lo=20001,
                                              seq_len_hi=32768, seed=502),
     "2 x 131072, B=32, shared prefix": W.reduced(5, num_seqs=2),
+    # a handful of units: about 128 CTAs, up to 128 / units partials per row
+    "1 x 32768, 1 kv head": W.PagedConfig("1 x 32768, 8/1", num_seqs=1, num_heads=8,
+                                          num_kv_heads=1, head_size=128, block_size=16,
+                                          num_blocks=2048 + 40, seq_len_lo=32768,
+                                          seq_len_hi=32768, seed=503),
+    "1 x 20000, 2 kv heads, B=32": W.PagedConfig("1 x 20000, 16/2", num_seqs=1, num_heads=16,
+                                                 num_kv_heads=2, head_size=128, block_size=32,
+                                                 num_blocks=625 + 40, seq_len_lo=20000,
+                                                 seq_len_hi=20000, seed=504),
 }
 
 
 @pytest.mark.parametrize("name", sorted(SMALL_LONG))
 def test_small_long_context_batches_all_rows(name):
     """One or two long sequences: the planner takes one partial wave of CTAs
-    with at most 32 partials per row; every row against the oracle."""
+    with at most 32 partials per row (or, for a handful of units, about 128
+    CTAs with up to 128 / units partials per row, merged in several batches of
+    loads); every row against the oracle."""
     cfg = SMALL_LONG[name]
     plan = pa.plan(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_size,
                    cfg.block_size, cfg.max_seq_len, cfg.kv_dtype,
                    shared_prefix_blocks=cfg.shared_prefix_blocks)
-    assert plan["num_partitions"] + plan["prefix_partitions"] <= 32, plan
+    units = cfg.num_seqs * cfg.num_kv_heads
+    assert plan["num_partitions"] + plan["prefix_partitions"] <= max(32, -(-128 // units)), plan
     wl = W.make_workload(cfg, DEV)
     out = run_gpu(wl, shared_prefix_blocks=cfg.shared_prefix_blocks)
     torch.cuda.synchronize()
