@@ -30,8 +30,11 @@ constexpr long long kLongPartitionPages = 256;
 // loads (a slot per lane); split plans keep to it where they can.
 constexpr long long kOneBatchSlots = 32;
 // CTAs of a split plan for a batch of only a handful of (sequence, kv head)
-// units, where one partial wave within kOneBatchSlots would stay small.
+// units, where one partial wave within kOneBatchSlots would stay small:
+// kFewUnitCtas per kFewUnitSms SMs (128 on a 148-SM B200), scaled to the SMs
+// the plan is made for.
 constexpr long long kFewUnitCtas = 128;
+constexpr long long kFewUnitSms = 148;
 // Split tail: partitions per unit of the last, partial wave of whole units
 // (at least; more when that wave has few units, up to kMaxTailParts).
 constexpr int kTailParts = 4;
@@ -346,15 +349,16 @@ pa_status plan(pa_plan* pl, int num_seqs, int num_heads, int num_kv_heads, int h
             }
             if (best1 < 0.0) {
                 // A handful of units (fewer than 7 on 148 SMs): about
-                // kFewUnitCtas CTAs, with up to max(32, kFewUnitCtas / units)
-                // partials per row.  Measured on B200 with 1, 2 and 4 units of
-                // 32768-131072 tokens: grids of 64-128 CTAs streamed 1.5-2.6x
-                // faster than 432-632 CTAs of 108-432 partials per row, whose
-                // merge takes several batches of loads.
-                const long long cap_slots =
-                    (kFewUnitCtas + units - 1) / units > kOneBatchSlots
-                        ? (kFewUnitCtas + units - 1) / units
-                        : kOneBatchSlots;
+                // kFewUnitCtas CTAs (128 on 148 SMs), with up to
+                // max(32, that / units) partials per row.  Measured on B200 with
+                // 1, 2 and 4 units of 32768-131072 tokens: grids of 64-128 CTAs
+                // streamed 1.5-2.6x faster than 432-632 CTAs of 108-432
+                // partials per row, whose merge takes several batches of loads.
+                long long few = static_cast<long long>(sms) * kFewUnitCtas / kFewUnitSms;
+                if (few < 1) few = 1;
+                const long long cap_slots = (few + units - 1) / units > kOneBatchSlots
+                                                ? (few + units - 1) / units
+                                                : kOneBatchSlots;
                 for (long long n = 1;; ++n) {
                     if (n > 1 && (pages_max + n - 1) / n < kMinPartitionPages) break;
                     if (row_slots(n) > cap_slots) break;
