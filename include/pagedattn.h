@@ -93,7 +93,12 @@ typedef enum pa_kv_dtype {
  * Tuning knobs; pass NULL for the planner's defaults.
  *  partition_pages: 0 lets the planner choose; > 0 forces split-KV partitions
  *      of that many blocks (the combine kernel merges them).  A value >= the
- *      longest sequence's block count means "no split".
+ *      longest sequence's block count means "no split".  The planner splits
+ *      only batches of fewer than two waves of (sequence, kv head) units; it
+ *      takes a partition count whose last wave of CTAs is about 62% full, at
+ *      most 32 partials per query row where the batch allows it (one or two
+ *      long sequences take one partial wave; a handful of units about 128 CTAs
+ *      on 148 SMs), and partitions of even size over each sequence's pages.
  *  num_sms: 0 queries the current device; > 0 plans for that many SMs
  *      (lets the host plan without a GPU, e.g. to size a workspace).
  *  stages: 0 lets the planner choose; 2..16 forces that many page buffers
